@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Benchmark of the routed mixture-of-experts FFN from low-bit blocks on B200.
+
+Default workload (one JSON line on stdout, rank 0):
+  verify-stack-48L-8tok-q2 -- 1 + 7 token verify batches through a 48-layer MoE-only stack
+  (d_model 2048, expert d_ff 768, 512 routed experts top-10 + 1 shared expert, 2-bit Q2 blocks,
+  ~36 GB resident in HBM), residual add between layers, no norm, fresh seeded x per pass.
+  A step is one pass: 8 tokens through all 48 layers.  Every pass reads ~3.6 GB of distinct
+  expert blocks, far more than the 126 MB L2, so no flush is needed between steps.
+
+Also: --workload decode (1 token through 16 model-scale layers of seeds 0-15, one step = the 16
+layers), --workload codebook (3.5-bit codebook blocks, 48 independent layers on the same x),
+--workload prefill (1,180 / 8,192-token chunks through the stack, grouped GEMM path).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload verify|decode|codebook|prefill]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample, same metric
+
+Multi-GPU: replicas only (each rank holds the full stack and its own token stream; no
+collective on the data path); time = max over ranks, value = all ranks' tokens / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import synth  # noqa: E402
+
+METRIC = "routed-MoE tokens/s (48-layer stack); decode HBM GB/s; prefill TFLOP/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------------ utilities
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = Path(os.environ.get("TMPDIR", "/tmp")) / f"clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path.exists():
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.path.read_text().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def source_hash(*files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        h.update((ROOT / f).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str, src_hash: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    p = ROOT / "profiles" / f"{kernel}_{workload}.md"
+    if not p.exists():
+        return None
+    t = p.read_text()
+    m = re.search(r"source_hash:\s*([0-9a-f]+)", t)
+    b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", t)
+    if not m or not b or m.group(1) != src_hash:
+        return None
+    return float(b.group(1))
+
+
+# ------------------------------------------------------------------------------------ distributed
+def dist_setup(n_gpus):
+    import torch
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------ model setup
+def load_stack(moe, wl, seed, layers, layer_of=lambda i: i, chunk=128):
+    """Generate each layer on the device (seeded hash, byte-identical to the CPU generator) and
+    load it through moe_load_layer from device memory."""
+    import torch
+
+    dev = torch.device("cuda")
+    buf = torch.empty((wl.n_experts, wl.expert_bytes()), dtype=torch.uint8, device=dev)
+    sh = torch.empty((1, wl.expert_bytes(shared=True)), dtype=torch.uint8, device=dev) if wl.n_shared else None
+    for i in range(layers):
+        l = layer_of(i)
+        s = seed if not isinstance(seed, (list, tuple)) else seed[i]
+        for e0 in range(0, wl.n_experts, chunk):
+            ids = range(e0, min(wl.n_experts, e0 + chunk))
+            synth.gen_experts_torch(wl, s, l, ids, buf[e0:e0 + len(ids)])
+        if sh is not None:
+            synth.gen_experts_torch(wl, s, l, [wl.n_experts], sh)
+        router = synth.gen_router_torch(wl, s, l, dev).contiguous()
+        b = synth.gen_bias(wl, s, l)
+        bias = None if b is None else torch.from_numpy(b).to(dev)
+        moe.load_layer(i, router, bias, buf, sh)
+    torch.cuda.synchronize()
+    del buf, sh
+
+
+def make_moe(wl, n_layers, max_tokens, seed=0):
+    import expert_ffn_gemv_b200 as P
+
+    grid = synth.gen_grid(wl, seed) if wl.fmt == synth.FMT_CB35 else None
+    return P.MoE(n_layers=n_layers, d_model=wl.d_model, d_ff=wl.d_ff, n_experts=wl.n_experts, top_k=wl.top_k,
+                 n_shared=wl.n_shared, shared_d_ff=wl.shared_d_ff, fmt=wl.fmt, act_dtype=wl.act_dtype,
+                 router_dtype=wl.router_dtype, out_dtype=P.MOE_F32, max_tokens=max_tokens, codebook_grid=grid,
+                 device=0 if "LOCAL_RANK" not in os.environ else int(os.environ["LOCAL_RANK"]))
+
+
+# ------------------------------------------------------------------------------------ CPU oracle
+def oracle_sample_stack(wl, seed, n_tokens, n_layers_sample, pass_idx=0, threads=0):
+    """Time the fp64 oracle on n_tokens through the first n_layers_sample layers (generation of
+    the sampled layers' bytes is outside the timed part).  Returns (seconds, threads used)."""
+    import oracle
+
+    sys.path.insert(0, str(ROOT / "tests"))
+    from helpers import oracle_layer, supply_from_generator
+
+    x = oracle.to_f64(synth.gen_x(wl, seed, n_tokens, pass_idx), wl.act_dtype)
+    total = 0.0
+    for l in range(n_layers_sample):
+        L = oracle_layer(wl, seed, l, full=False)
+        idx, _, _ = L.route(x)
+        supply_from_generator(wl, seed)(l, L, sorted(set(idx.reshape(-1).tolist())))
+        t0 = time.perf_counter()
+        r = L.forward(x, n_threads=threads)
+        total += time.perf_counter() - t0
+        x = x + r["y"]
+    used = min(n_tokens, threads if threads > 0 else oracle.max_threads())
+    return total, used
+
+
+# ------------------------------------------------------------------------------------ verify stack
+def bench_verify(args, rank, world, local):
+    import torch
+
+    import expert_ffn_gemv_b200 as P
+
+    wl = synth.VERIFY
+    L = args.layers
+    n = wl.n_tokens
+    K, W = args.steps, args.warmup
+    seed = args.seed
+    moe = make_moe(wl, L, 8, seed)
+    t0 = time.time()
+    load_stack(moe, wl, seed, L)
+    load_s = time.time() - t0
+    dev = torch.device("cuda")
+    # fresh x per pass; each rank its own token stream
+    xs = torch.stack([synth.gen_x_torch(wl, seed, n, 1000 * rank + p, dev) for p in range(W + K)]).contiguous()
+    x_in = torch.empty((n, wl.d_model), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((n, wl.d_model), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream()
+    # the timed graph carries event pairs around the gate/up launches only (the roofline kernel)
+    P.moe_profile_enable(moe.h, 1 << P.PROF_GATEUP)
+    with torch.cuda.stream(stream):
+        x_in.copy_(xs[0])
+        moe.forward_stack(0, L, x_in, out)  # eager warm call
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            moe.forward_stack(0, L, x_in, out)
+        for p in range(W):
+            x_in.copy_(xs[p])
+            g.replay()
+        stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for p in range(K):
+                x_in.copy_(xs[W + p])
+                g.replay()
+            ev1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world)
+    # gate/up durations of the last replay (inside the timed region)
+    st_, gu_ms, gu_cnt = P.moe_profile_read(moe.h, P.PROF_GATEUP)
+    if st_ != P.MOE_OK:
+        print(f"profile read: status {st_}: {P.moe_last_error(moe.h)}", file=sys.stderr)
+    # per-kernel breakdown of one eager (untimed) pass of the same input
+    P.moe_profile_enable(moe.h, True)
+    with torch.cuda.stream(stream):
+        x_in.copy_(xs[W + K - 1])
+        moe.forward_stack(0, L, x_in, out)
+    stream.synchronize()
+    kern = {}
+    for kind, name in ((P.PROF_ROUTE, "k_route"), (P.PROF_GATEUP, "k_gateup"), (P.PROF_DOWN, "k_down+k_combine")):
+        _, tot, cnt = P.moe_profile_read(moe.h, kind)
+        kern[name] = (tot, cnt)
+    P.moe_profile_enable(moe.h, False)
+    # routing of every timed pass (deterministic: re-run eagerly, untimed) -> active experts
+    counts = [torch.empty(wl.n_experts, dtype=torch.int32, device=dev) for _ in range(L)]
+    routes = [dict(counts=c) for c in counts]
+    u_all = np.zeros((K, L), dtype=np.int64)
+    with torch.cuda.stream(stream):
+        for p in range(K):
+            x_in.copy_(xs[W + p])
+            moe.forward_stack(0, L, x_in, out, routes=routes)
+            u_all[p] = torch.stack([(c > 0).sum() for c in counts]).cpu().numpy()
+    stream.synchronize()
+    expert_bytes = wl.expert_bytes()
+    mat_bytes = expert_bytes // 3
+    # algorithmic bytes: every active expert's blocks (gate + up + down) + shared, + router
+    router_bytes = wl.n_experts * wl.d_model * 2
+    step_bytes = ((u_all + wl.n_shared) * expert_bytes).sum(axis=1) + L * router_bytes  # per pass
+    gateup_bytes_last = float(((u_all[-1] + wl.n_shared) * 2 * mat_bytes).sum())
+    down_bytes_last = float(((u_all[-1] + wl.n_shared) * mat_bytes).sum())
+
+    tokens = K * n
+    total_tokens = sum_over_ranks(tokens, world)
+    value = total_tokens / (ms / 1e3)
+    pk, pk_kind = peaks()
+    hbm_peak = pk["hbm_gbs"]
+    achieved = gateup_bytes_last / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
+    src = source_hash("expert_ffn_gemv_b200/csrc/decode.cu", "expert_ffn_gemv_b200/csrc/moe_internal.cuh")
+    traffic = profiled_traffic("k_gateup", "verify", src)
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "q2 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
+        "data": "synthetic (seeded integer-hash generator, random-init weights)",
+        "config": {"workload": wl.name, "d_model": wl.d_model, "d_ff": wl.d_ff, "n_experts": wl.n_experts,
+                   "top_k": wl.top_k, "n_shared": wl.n_shared, "layers": L, "tokens_per_pass": n,
+                   "weights": "Q2 2-bit blocks, 10 B / 32 weights", "router_bias": "Zipf(1.1), beta 0.5",
+                   "resident_weight_gb": round(moe.device_bytes() / 1e9, 2),
+                   "l2": "inputs larger than L2: each pass reads ~%.1f GB of distinct expert blocks"
+                         % (step_bytes.mean() / 1e9),
+                   "parallelism": f"replicas x{world}", "cuda_graph": "one pass (48 x 4 kernels) per replay"},
+        "hbm": {"active_expert_and_router_bytes_per_step": float(step_bytes.mean()),
+                "gbs": float(step_bytes.sum() / (ms_local / 1e3) / 1e9),
+                "frac_of_measured_peak": float(step_bytes.sum() / (ms_local / 1e3) / 1e9 / hbm_peak),
+                "mean_active_experts_per_layer": float(u_all.mean() + wl.n_shared)},
+        "roofline": {"kernel": "k_gateup", "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+                     "peak_kind": pk_kind, "unit": "GB/s",
+                     "frac": achieved / hbm_peak if achieved else None, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": gateup_bytes_last / max(gu_cnt, 1),
+                     "avg_launch_us": gu_ms / max(gu_cnt, 1) * 1e3},
+        "kernels_eager_pass_us": {k: round(v[0] * 1e3, 2) for k, v in kern.items()},
+        "down_roofline": {"achieved": down_bytes_last / (kern["k_down+k_combine"][0] / 1e3) / 1e9
+                          if kern["k_down+k_combine"][0] else None, "unit": "GB/s"},
+        "gpu_launches": K * L * 4,
+        "clocks": clk.summary(),
+        "load_seconds": round(load_s, 1),
+    }
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    if not args.no_e2e:
+        xh = xs[W:W + K].cpu().pin_memory()
+        oh = torch.empty((n, wl.d_model), dtype=torch.float32).pin_memory()
+        Ke = min(K, args.e2e_steps)
+        for p in range(2):
+            moe.forward_stack(0, L, xh[p], oh)
+        barrier(world)
+        t0 = time.perf_counter()
+        for p in range(Ke):
+            moe.forward_stack(0, L, xh[p], oh)  # library stages H2D, runs, copies D2H, syncs
+        el = time.perf_counter() - t0
+        el = max_over_ranks(el, world)
+        res["e2e"] = {"value": sum_over_ranks(Ke * n, world) / el, "unit": "tokens/s",
+                      "h2d_bytes_per_step": n * wl.d_model * 2, "d2h_bytes_per_step": n * wl.d_model * 4,
+                      "steps": Ke, "api": "moe_forward_stack(host x, host x_out)"}
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nl = args.cpu_layers
+        sec, used = oracle_sample_stack(wl, seed, n, nl, pass_idx=0)
+        res["cpu_baseline"] = {"value": n * nl / sec / L, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                               "sample": f"{n} tokens through the first {nl} of {L} layers, fp64 C oracle "
+                                         f"(OpenMP over tokens); tokens/s scaled to the {L}-layer stack"}
+    moe.close()
+    return res
+
+
+# ------------------------------------------------------------------------------------ reference arm
+def bench_reference(args):
+    """The fp64 CPU oracle as the reference arm: each step = 8 tokens through one layer of the
+    48-layer verify stack (layer = step mod 48), timed on the host cores."""
+    import oracle
+
+    sys.path.insert(0, str(ROOT / "tests"))
+    from helpers import oracle_layer, supply_from_generator
+
+    wl = synth.VERIFY
+    L, n, seed = args.layers, wl.n_tokens, args.seed
+    cache = {}
+
+    def layer(l):
+        if l not in cache:
+            if len(cache) >= 4:
+                cache.pop(next(iter(cache)))
+            cache[l] = oracle_layer(wl, seed, l, full=False)
+        return cache[l]
+
+    x = oracle.to_f64(synth.gen_x(wl, seed, n, 0), wl.act_dtype)
+    times = []
+    for s in range(args.warmup + args.steps):
+        l = s % L
+        Ll = layer(l)
+        idx, _, _ = Ll.route(x)
+        supply_from_generator(wl, seed)(l, Ll, sorted(set(idx.reshape(-1).tolist())))
+        t0 = time.perf_counter()
+        Ll.forward(x)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times)
+    used = min(n, oracle.max_threads())
+    value = n * len(times) / sec / L
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / len(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded integer-hash generator)",
+        "config": {"workload": wl.name, "layers": L, "tokens_per_pass": n,
+                   "step": "8 tokens through one layer (layer = step mod 48), scaled to the 48-layer stack"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                         "sample": f"{len(times)} steps of 8 tokens x 1 layer"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["verify"], default="verify")
+    ap.add_argument("--layers", type=int, default=48)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-layers", type=int, default=12)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(bench_reference(args)), flush=True)
+        return 0
+    rank, world, local = dist_setup(args.gpus)
+    res = bench_verify(args, rank, world, local)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,219 @@
+// moe_internal.cuh -- device layout, workspace and PTX helpers shared by the library's kernels.
+//
+// Device layout of one weight matrix (R rows x K columns, blocks of 32 along a row):
+// rows are split into tiles of 128 and columns into chunks of 64 weights (two blocks).
+// For every (row tile, chunk) the 128 rows' data are contiguous, row after row:
+//   plane A  [R/128][K/64][128][16 B]  Q2: 2-bit codes, CB35: grid-row indices (16 per chunk)
+//   plane S  [R/128][K/64][128][2 x fp16]  the two block scales of the chunk
+//   plane G  [R/128][K/64][128][2 x u32]   CB35 only: sign masks of the two blocks
+// so a warp whose lanes are 32 consecutive rows reads 512 contiguous bytes of plane A, and a
+// 128-row tile over a run of chunks is one contiguous range (one bulk copy).
+// Bit placement inside a 16-byte Q2 chunk (weights p = 0..63 of the chunk): word p/16, byte
+// p%4, bits 2*((p%16)/4) .. +1.  Masking (word >> 2kk) & 0x03030303 therefore yields the four
+// codes of weights 16w+4kk .. 16w+4kk+3 as bytes 0..3, the operand order of dp2a.
+// CB35 sign word of a block: byte j, bit g is the sign of weight 4g + j, so shifting left by
+// 7 - g puts the signs of group g in the byte msbs, where prmt can replicate them.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kDecodeMaxTokens = 8;   // decode / verify path: 1..8 tokens per call
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 4096;
+constexpr int kTileRows = 128;
+constexpr int kChunk = 64;            // weights per 16-byte code chunk
+constexpr int kDecodeMaxD = 4096;     // decode kernels keep n x D activations in shared memory
+constexpr int kMaxFF = 1024;          // d_ff limit: a CTA quantises a whole h row in registers
+
+// error word bits (host-mapped, OR-ed by device code)
+constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrBadIndex = 2u;
+
+// One group of experts with equal shapes (all routed experts, or the shared expert).
+struct ExpertGroup {
+  uint8_t *a;          // plane A of expert 0, matrix 0
+  __half2 *s;          // plane S
+  uint2 *g;            // plane G (CB35) or nullptr
+  int64_t a_mat;       // bytes of plane A per matrix   = F * D / 4
+  int64_t s_mat;       // half2 per matrix              = F * D / 64
+  int64_t g_mat;       // uint2 per matrix              = F * D / 64
+  int f;               // d_ff of this group
+  int count;           // experts in the group
+};
+
+struct LayerDev {
+  const void *router_w;  // E x D, router dtype
+  const float *bias;     // E
+  ExpertGroup routed;
+  ExpertGroup shared;    // count 0 when there is no shared expert
+  bool loaded;
+};
+
+struct Shape {
+  int d;          // d_model
+  int e;          // n_experts
+  int k;          // top_k
+  int n_shared;   // 0 or 1
+  int fmt;        // MOE_FMT_*
+  int router_bf16;
+};
+
+// Decode workspace (n <= 8 tokens).  u indexes active experts: u = 0 is the shared expert
+// when there is one, routed active experts follow in ascending expert id.  Activations enter
+// the GEMVs as int16 fixed point with a power-of-two factor: the layer input per (token,
+// K-split) (written by the router kernel), the SwiGLU output h per (row, 128-row tile of F)
+// (written where h is produced); each comes with its 32-element block sums.
+struct DecodeWs {
+  float *logits;        // [8][E]
+  int *route_idx;       // [8][k]
+  float *route_w;       // [8][k]
+  int *slotpos;         // [8][k]: u * 8 + i (i = position of the token in expert u's list)
+  int *n_active;        // [1]
+  int *act_expert;      // [umax]: expert id, E for the shared expert
+  int *act_ntok;        // [umax]
+  int *act_tok;         // [umax][8]
+  int16_t *xq;          // [8][D]
+  int *xsum;            // [8][D/32]
+  float *xfac;          // [8][pad4(splits)]
+  int16_t *hq;          // [umax * 8][fmax]
+  int *hsum;            // [umax * 8][fmax/32]
+  float *hfac;          // [umax * 8][hfs]
+  float *gu_part;       // [umax][tmax][splits][2][8][128] gate/up partial sums
+  float *o;             // [umax * 8][D] expert outputs (unweighted)
+  unsigned *route_ticket;   // [1]
+  unsigned *gu_ticket;      // [umax][tmax]
+  int umax;
+  int tmax;             // max(F, F_shared) / 128
+  int fmax;
+  int splits;           // K-splits of the gate/up reduction (d_model / splits columns per CTA)
+  int hfs;              // row stride of hfac: tmax rounded up to a multiple of 4
+  int grid_gu;          // persistent grid of k_gateup / k_down
+  int grid_down;
+};
+
+// ------------------------------------------------------------------------------------------
+// PTX helpers
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completion counted on `bar` (bytes).
+// dst, src 16-byte aligned; bytes a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Bounded wait on an mbarrier phase.  Returns false when `limit` clock cycles pass first.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (static_cast<uint64_t>(clock64() - t0) > limit) return false;
+  }
+  return true;
+}
+
+// Waits for copies a CTA issued before it gives up: a CTA must not exit while a bulk copy
+// still writes its shared memory.  About two seconds at B200 clocks.
+constexpr uint64_t kDrainLimit = 4000000000ull;
+
+__device__ __forceinline__ void flag_error(uint32_t *err, uint32_t bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// prmt in its default mode: a selector nibble with bit 3 set replicates the sign (msb) of the
+// selected byte.  prmt_sign_bytes(t) = 0xFF in byte j where byte j of t has its msb set.
+__device__ __forceinline__ uint32_t prmt_sign_bytes(uint32_t t) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(r) : "r"(t));
+  return r;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+// ------------------------------------------------------------------------------------------
+// launchers (host side, defined in the .cu files)
+// ------------------------------------------------------------------------------------------
+cudaError_t launch_repack(const uint8_t *src, int64_t src_stride, int fmt, int rows, int cols,
+                          int n_mats, int64_t dst_stride, uint8_t *a, __half2 *s, uint2 *g,
+                          cudaStream_t st);
+
+struct DecodeArgs {
+  Shape sh;
+  LayerDev L;
+  DecodeWs ws;
+  const int8_t *grid;        // device 256 x 4 (CB35)
+  const void *x;             // layer input [n][D]
+  int x_bf16;                // 1: x is bf16, 0: fp32
+  int n;                     // tokens
+  void *y;                   // output [n][D]
+  int y_bf16;
+  int residual;              // 1: y = x + MoE(x), else y = MoE(x)
+  float *y_copy;             // optional fp32 copy of y
+  int *out_idx;              // optional user routing outputs
+  float *out_w;
+  int *out_counts;
+  uint32_t *err;
+  uint64_t spin_limit;
+  cudaEvent_t *ev;           // optional timing events: [kind][start, end] for kinds 0..2
+  uint32_t prof_mask;        // kinds whose events are recorded
+};
+
+// kernel classes of the per-kernel event timing
+constexpr int kProfRoute = 0;     // router + top-k (+ routing tables / grouping)
+constexpr int kProfGateUp = 1;    // gate/up GEMV or GEMM + SwiGLU
+constexpr int kProfDown = 2;      // down GEMV or GEMM + combine
+constexpr int kProfKinds = 3;
+
+cudaError_t configure_decode_kernels();
+cudaError_t decode_grid_sizes(int fmt, int d, int splits, int fmax, int umax, int n_shared, int f, int f_shared,
+                              int *grid_gu, int *grid_down);
+cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_wait_test(unsigned *never_set, uint32_t *err, uint64_t spin_limit, cudaStream_t st);
+
+}  // namespace moe

@@ -330,18 +330,51 @@ def _matrix_blocks_torch(wl: Workload, key_base: tuple, rows: int, cols: int, ou
 
 
 def gen_experts_torch(wl: Workload, seed: int, layer: int, experts, out):
-    """Write the interchange bytes of ``experts`` (ids) into ``out`` (uint8 [len, expert bytes])."""
+    """Write the interchange bytes of ``experts`` (ids, all routed or all the shared one) into
+    ``out`` (uint8 [len, expert bytes]); every matrix of the batch is hashed in one pass."""
+    import torch
+
+    experts = list(experts)
+    if not experts:
+        return
+    dev = out.device
     d = wl.d_model
-    for j, e in enumerate(experts):
-        shared = e >= wl.n_experts
-        f = wl.shared_d_ff if shared else wl.d_ff
-        off = 0
-        row = out[j]
-        for m, (r, c) in enumerate(((f, d), (f, d), (d, f))):
-            nbytes = r * c // 32 * wl.block_bytes
-            view = row[off:off + nbytes].view(-1, wl.block_bytes)
-            _matrix_blocks_torch(wl, (seed, wl.wid, layer, T_EXPERT, e, m), r, c, view)
-            off += nbytes
+    shared = experts[0] >= wl.n_experts
+    assert all((e >= wl.n_experts) == shared for e in experts)
+    f = wl.shared_d_ff if shared else wl.d_ff
+    bb = wl.block_bytes
+    stab = _torch_table("scale", scale_table_f16(), dev)
+    nb = f * d // 32  # blocks per matrix (gate, up and down have the same count)
+    off = 0
+    for m in range(3):
+        keys = [(seed, wl.wid, layer, T_EXPERT, e, m) for e in experts]
+
+        def kk(field_id):
+            ks = [stream_key(*k, field_id) for k in keys]
+            k0 = torch.tensor([a for a, _ in ks], dtype=torch.int64, device=dev)[:, None]
+            k1 = torch.tensor([b for _, b in ks], dtype=torch.int64, device=dev)[:, None]
+            return k0, k1
+
+        def words(field_id, count):
+            k0, k1 = kk(field_id)
+            i = torch.arange(count, dtype=torch.int64, device=dev)[None, :]
+            return hash32((hash32(i ^ k0) + k1) & M32)
+
+        view = out[:, off:off + nb * bb].view(len(experts), nb, bb)
+        sc = stab[words(F_SCALE, nb) & 0xFFFF].to(torch.int64)
+        view[:, :, 0] = (sc & 0xFF).to(torch.uint8)
+        view[:, :, 1] = (sc >> 8).to(torch.uint8)
+        del sc
+        if wl.fmt == FMT_Q2:
+            c = words(F_CODES, 2 * nb)
+            view[:, :, 2:10] = _u32_bytes_torch(c).reshape(len(experts), nb, 8)
+        else:
+            ix = words(F_IDX, 2 * nb)
+            view[:, :, 2:10] = _u32_bytes_torch(ix).reshape(len(experts), nb, 8)
+            del ix
+            sg = words(F_SIGN, nb)
+            view[:, :, 10:14] = _u32_bytes_torch(sg).reshape(len(experts), nb, 4)
+        off += nb * bb
 
 
 def gen_router_torch(wl: Workload, seed: int, layer: int, device):

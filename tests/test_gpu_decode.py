@@ -1,0 +1,216 @@
+"""GPU parity of the dequant-fused GEMV path (1..8 tokens) against the fp64 oracle."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from helpers import (TOL_DECODE, compare_routing, load_layer_device, load_layer_host, moe_for, oracle_layer,
+                     rel_l2, route_buffers, supply_from_generator, x_device, x_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+
+    assert torch.cuda.is_available()
+    import expert_ffn_gemv_b200 as P
+
+    P.lib()
+    return torch
+
+
+def _run_layer(torch, moe, wl, seed, n, layer_slot=0, pass_idx=0):
+    x = x_device(wl, seed, n, pass_idx)
+    y = torch.empty((n, wl.d_model), dtype=torch.float32, device="cuda")
+    rb = route_buffers(n, wl.top_k, wl.n_experts)
+    moe.forward(layer_slot, x, y, route=rb)
+    torch.cuda.synchronize()
+    return x, y.cpu().numpy(), {k: v.cpu().numpy() for k, v in rb.items()}
+
+
+def _check_layer(wl, seed, layer, x, y, rb, L=None, tol=TOL_DECODE):
+    if L is None:
+        L = oracle_layer(wl, seed, layer)
+    xs = x_f64(wl, x.view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+               if wl.act_dtype == synth.DT_BF16 else x.cpu().numpy())
+    if not L._experts:
+        idx, _, _ = L.route(xs)
+        supply_from_generator(wl, seed)(layer, L, sorted(set(idx.reshape(-1).tolist())))
+    ref = L.forward(xs)
+    bad, excl = compare_routing(rb["idx"], ref["idx"], ref["margin"], wl.n_experts, rb["counts"])
+    assert bad == 0, f"routing mismatches on {bad} tokens (excluded {excl})"
+    keep = ref["margin"] >= 1e-4
+    assert np.allclose(rb["w"].sum(1), 1.0, atol=1e-5)
+    for t in np.nonzero(keep)[0]:
+        order = {e: j for j, e in enumerate(ref["idx"][t])}
+        w_ref = np.array([ref["w"][t][order[e]] for e in rb["idx"][t]])
+        assert np.allclose(rb["w"][t], w_ref, rtol=1e-5, atol=1e-6)
+    err = rel_l2(y, ref["y"], keep)
+    assert err <= tol, f"max rel L2 {err:.3e} > {tol}"
+    return err, excl
+
+
+def test_tiny_layer_host_buffers(torch_cuda):
+    """d_model 256, d_ff 128, 16 experts, top-2, no shared expert, 4 tokens, fp32 x and router."""
+    torch = torch_cuda
+    wl = synth.TINY
+    moe = moe_for(wl, 1, 8)
+    load_layer_host(moe, 0, wl, 0, 0)
+    x_bits = synth.gen_x(wl, 0, 4)
+    y = np.zeros((4, wl.d_model), dtype=np.float32)
+    moe.forward(0, np.ascontiguousarray(x_bits), y)  # host x and y
+    xd = torch.from_numpy(x_bits).cuda()
+    x, yd, rb = _run_layer(torch, moe, wl, 0, 4)
+    assert np.array_equal(y, yd)
+    _check_layer(wl, 0, 0, xd, yd, rb)
+    moe.close()
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 8])
+def test_small_layer_tokens(torch_cuda, fmt, n):
+    torch = torch_cuda
+    wl = synth.small_workload(fmt=fmt, d_model=512, d_ff=256, n_experts=32, top_k=4, n_shared=1, shared_d_ff=384)
+    moe = moe_for(wl, 1, 8, seed=1)
+    load_layer_device(moe, 0, wl, 1, 0)
+    x, y, rb = _run_layer(torch, moe, wl, 1, n)
+    _check_layer(wl, 1, 0, x, y, rb)
+    moe.close()
+
+
+def test_host_and_device_loads_agree(torch_cuda):
+    torch = torch_cuda
+    wl = synth.small_workload(d_model=256, d_ff=128, n_experts=16, top_k=3)
+    a, b = moe_for(wl, 1, 8), moe_for(wl, 1, 8)
+    load_layer_host(a, 0, wl, 2, 0)
+    load_layer_device(b, 0, wl, 2, 0)
+    _, ya, ra = _run_layer(torch, a, wl, 2, 6)
+    _, yb, rb = _run_layer(torch, b, wl, 2, 6)
+    assert np.array_equal(ya, yb) and np.array_equal(ra["idx"], rb["idx"])
+    a.close()
+    b.close()
+
+
+def test_batch_invariance_bitwise(torch_cuda):
+    """A token's output does not depend on the other tokens of its call."""
+    torch = torch_cuda
+    wl = synth.small_workload(d_model=512, d_ff=256, n_experts=32, top_k=4)
+    moe = moe_for(wl, 1, 8)
+    load_layer_device(moe, 0, wl, 3, 0)
+    x = x_device(wl, 3, 8)
+    y8 = torch.empty((8, wl.d_model), dtype=torch.float32, device="cuda")
+    moe.forward(0, x, y8)
+    for t in (0, 5, 7):
+        y1 = torch.empty((1, wl.d_model), dtype=torch.float32, device="cuda")
+        moe.forward(0, x[t:t + 1].contiguous(), y1)
+        torch.cuda.synchronize()
+        assert torch.equal(y1[0], y8[t])
+    y3 = torch.empty((3, wl.d_model), dtype=torch.float32, device="cuda")
+    moe.forward(0, x[2:5].contiguous(), y3)
+    torch.cuda.synchronize()
+    assert torch.equal(y3, y8[2:5])
+    # repeated calls are bit-reproducible
+    y8b = torch.empty_like(y8)
+    moe.forward(0, x, y8b)
+    torch.cuda.synchronize()
+    assert torch.equal(y8, y8b)
+    moe.close()
+
+
+@pytest.mark.parametrize("seeds", [range(0, 16)])
+def test_decode_layer_model_scale(torch_cuda, seeds):
+    """One token through one model-scale layer (d_model 2048, d_ff 768, 512 experts, top-10 +
+    shared expert, Zipf router bias), seeds 0-15, all 16 layers resident in one handle."""
+    torch = torch_cuda
+    wl = synth.DECODE
+    seeds = list(seeds)
+    moe = moe_for(wl, len(seeds), 8)
+    for i, s in enumerate(seeds):
+        load_layer_device(moe, i, wl, s, 0)
+    worst, excluded = 0.0, 0
+    for i, s in enumerate(seeds):
+        x, y, rb = _run_layer(torch, moe, wl, s, 1, layer_slot=i)
+        L = oracle_layer(wl, s, 0, full=False)
+        err, excl = _check_layer(wl, s, 0, x, y, rb, L=L)
+        worst, excluded = max(worst, err), excluded + excl
+    print(f"decode layer: max rel L2 {worst:.2e}, excluded near-ties {excluded}")
+    moe.close()
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+def test_verify_batch_model_scale(torch_cuda, fmt):
+    """8 tokens (1 + 7 verify batch) through one model-scale layer of each format."""
+    torch = torch_cuda
+    wl = synth.VERIFY if fmt == synth.FMT_Q2 else synth.CODEBOOK
+    moe = moe_for(wl, 1, 8)
+    load_layer_device(moe, 0, wl, 0, 0)
+    for n in (1, 8):
+        x, y, rb = _run_layer(torch, moe, wl, 0, n, pass_idx=n)
+        L = oracle_layer(wl, 0, 0, full=False)
+        _check_layer(wl, 0, 0, x, y, rb, L=L)
+    moe.close()
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+def test_stack_teacher_forced_and_end_to_end(torch_cuda, fmt):
+    """A 3-layer stack of small layers, 8 tokens: per-layer inputs captured on the GPU feed the
+    oracle layer by layer (indices, counts, rel-L2 per layer), and the fp64 oracle stack from
+    the same x is compared with the GPU's final x."""
+    torch = torch_cuda
+    wl = synth.small_workload(fmt=fmt, d_model=512, d_ff=256, n_experts=32, top_k=4, n_layers=3)
+    nl, n, seed = 3, 8, 4
+    moe = moe_for(wl, nl, 8, seed=seed)
+    for l in range(nl):
+        load_layer_device(moe, l, wl, seed, l)
+    x = x_device(wl, seed, n)
+    out = torch.empty((n, wl.d_model), dtype=torch.float32, device="cuda")
+    trace = torch.empty((nl, n, wl.d_model), dtype=torch.float32, device="cuda")
+    routes = [route_buffers(n, wl.top_k, wl.n_experts) for _ in range(nl)]
+    moe.forward_stack(0, nl, x, out, routes=routes, x_trace=trace)
+    torch.cuda.synchronize()
+    tr = trace.cpu().numpy().astype(np.float64)
+    layers = [oracle_layer(wl, seed, l) for l in range(nl)]
+    x0 = x_f64(wl, x.view(torch.int16).cpu().numpy().view(np.uint16))
+    assert np.array_equal(tr[0], x0)
+    any_excl = np.zeros(n, dtype=bool)
+    for l in range(nl):
+        ref = layers[l].forward(tr[l])
+        rb = {k: v.cpu().numpy() for k, v in routes[l].items()}
+        bad, _ = compare_routing(rb["idx"], ref["idx"], ref["margin"], wl.n_experts, rb["counts"])
+        assert bad == 0
+        y_gpu = (tr[l + 1] if l + 1 < nl else out.cpu().numpy().astype(np.float64)) - tr[l]
+        keep = ref["margin"] >= 1e-4
+        any_excl |= ~keep
+        err = rel_l2(y_gpu, ref["y"], keep)
+        print(f"stack fmt={fmt} layer {l}: teacher-forced max rel L2 {err:.2e}")
+        assert err <= TOL_DECODE
+    # End to end from the same x.  The synthetic codebook weights (|w| up to 0.3) make a
+    # norm-free residual stack grow ~100x per layer, which amplifies rounding layer after
+    # layer, so the end-to-end check of that format stops after two layers; the Q2 stack
+    # (small per-layer gain) is checked over all three.
+    n_e2e = nl if fmt == synth.FMT_Q2 else 2
+    ref_out, recs = oracle.stack_forward(layers[:n_e2e], x0)
+    for r in recs:
+        any_excl |= r["margin"] < 1e-4
+    got = out.cpu().numpy() if n_e2e == nl else tr[n_e2e]
+    err = rel_l2(got, ref_out, ~any_excl)
+    print(f"stack fmt={fmt}: end-to-end max rel L2 over {n_e2e} layers {err:.2e}")
+    assert err <= TOL_DECODE
+    moe.close()
+
+
+def test_stack_one_layer_equals_forward_plus_x(torch_cuda):
+    torch = torch_cuda
+    wl = synth.small_workload(d_model=256, d_ff=128, n_experts=16, top_k=2)
+    moe = moe_for(wl, 1, 8)
+    load_layer_device(moe, 0, wl, 5, 0)
+    x = x_device(wl, 5, 4)
+    y = torch.empty((4, wl.d_model), dtype=torch.float32, device="cuda")
+    out = torch.empty_like(y)
+    moe.forward(0, x, y)
+    moe.forward_stack(0, 1, x, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, x.float() + y)
+    moe.close()
