@@ -57,6 +57,7 @@ EXPORTED = [
     "moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack", "moe_check", "moe_destroy",
     "moe_status_string", "moe_last_error", "moe_device_bytes", "moe_debug_set_spin_limit",
     "moe_debug_set_alloc_cap", "moe_debug_wait_test", "moe_profile_enable", "moe_profile_read",
+    "moe_route_noalloc",
 ]
 
 _lib = None
@@ -91,9 +92,10 @@ def lib() -> C.CDLL:
         L.moe_debug_wait_test.argtypes = [P, P]
         L.moe_profile_enable.argtypes = [P, I]
         L.moe_profile_read.argtypes = [P, I, C.POINTER(C.c_float), C.POINTER(I)]
+        L.moe_route_noalloc.argtypes = [P, I, P, I, I, I, P, I, I, P, P, P]
         for name in ("moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack", "moe_check",
                      "moe_destroy", "moe_debug_set_spin_limit", "moe_debug_set_alloc_cap",
-                     "moe_debug_wait_test", "moe_profile_enable", "moe_profile_read"):
+                     "moe_debug_wait_test", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -171,6 +173,13 @@ def moe_profile_read(h, kind: int):
 
 
 PROF_ROUTE, PROF_GATEUP, PROF_DOWN = 0, 1, 2
+
+
+def moe_route_noalloc(router_w: int, router_dtype: int, router_bias: int | None, n_experts: int, d_model: int,
+                      top_k: int, x: int, x_dtype: int, n_tokens: int, topk_idx: int, topk_w: int, stream) -> int:
+    """Handle-less routing that allocates no device memory (device pointers; see include/moe.h)."""
+    return lib().moe_route_noalloc(router_w, router_dtype, router_bias, n_experts, d_model, top_k, x, x_dtype,
+                                   n_tokens, topk_idx, topk_w, stream)
 
 
 # ----------------------------------------------------------------------------------- torch wrapper

@@ -16,7 +16,7 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 OUT_DIR = PKG / "_lib"
 LIB = OUT_DIR / "libmoe_b200.so"
-SOURCES = ["api.cu", "decode.cu", "repack.cu", "prefill.cu"]
+SOURCES = ["api.cu", "decode.cu", "repack.cu", "prefill.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", str(ROOT / "include"), "-I", str(CSRC)]

@@ -143,6 +143,26 @@ uint64_t moe_device_bytes(const moe_handle *h);
 moe_status moe_profile_enable(moe_handle *h, int32_t on);
 moe_status moe_profile_read(moe_handle *h, int32_t kind, float *total_ms, int32_t *launches);
 
+/* Routing for callers that cannot allocate device memory where they route (inside CUDA stream
+ * capture, under a runtime that plans all device memory itself, or in a loop that must not take
+ * cudaMalloc's implicit synchronisation).  The paper has no counterpart of this entry point: it
+ * is the routing step of moe_forward (router logits with fp32 accumulation, top-k with equal
+ * logits resolved to the lower expert index, fp32 softmax over the selected logits) without a
+ * handle.  All pointers are device pointers on the current device: router_w n_experts x d_model
+ * (router_dtype), router_bias n_experts fp32 or NULL, x n_tokens x d_model (x_dtype); outputs
+ * topk_idx / topk_w n_tokens x top_k, descending logit.  It allocates nothing: its scratch (the
+ * logits and an arrival counter, 32 KB) is a static device array that every GPU loading the
+ * library holds until exit.  The first call on a device looks up that array's device address
+ * and sets the kernel's shared-memory limit; make that first call before any stream capture.
+ * Limits: n_tokens <= 8, n_experts <= 1024, d_model <= 4096 (a multiple of 128), top_k <= 32;
+ * larger sizes return MOE_ERR_UNSUPPORTED, malformed arguments MOE_ERR_INVALID_ARGUMENT.
+ * Every call shares the one array and leaves its contents behind; calls whose kernels may
+ * overlap on one device race on it, so keep them in one stream order. */
+moe_status moe_route_noalloc(const void *router_w, int32_t router_dtype, const float *router_bias,
+                             int32_t n_experts, int32_t d_model, int32_t top_k, const void *x,
+                             int32_t x_dtype, int32_t n_tokens, int32_t *topk_idx, float *topk_w,
+                             void *stream);
+
 /* Test hooks.  moe_debug_set_spin_limit: clock cycles a device-side bounded wait may spin
  * before it gives up (0 restores the default of about one second).  moe_debug_set_alloc_cap:
  * fail allocations that would take the handle above `bytes` (0 = no cap). */
