@@ -1,30 +1,37 @@
-// prefill.cuh -- workspace and launcher of the grouped tensor-core path (more than 8 tokens).
+// prefill.cuh -- workspace and launcher of the grouped tensor-core path (more than 8 tokens):
+// prompt chunks of the routed-MoE pages (strata-mlx README, "Prompts": experts multiplied a tile
+// at a time on the matrix units; Strata reads chunks of up to 8,192 tokens).
 #pragma once
 
 #include "moe_internal.cuh"
 
 namespace moe {
 
-// Prompt-chunk workspace.  Assignments (token, slot) are grouped by expert with a counting
-// sort; the shared expert is the group after the routed ones (all tokens, token order).
+constexpr int kPfBN = 128;  // tokens per GEMM tile (MMA N, at most)
+
+// Prompt-chunk workspace.  Assignments (token, slot) are grouped by expert with a counting sort;
+// the shared expert is group E (all tokens, token order).  Rows of the grouped operands are
+// ordered by group; within a group the order is the arrival order of the scatter, which does not
+// change any result (every output row is computed independently of the others).
 struct PrefillWs {
   int max_tokens;
-  int rows_max;          // max_tokens * (k + n_shared): rows of the grouped operands
+  int rows_max;          // max_tokens * (k + n_shared)
   float *logits;         // [n][E]
   int *route_idx;        // [n][k]
   float *route_w;        // [n][k]
-  int *counts;           // [E + 1]   tokens per group (group E = shared)
+  int *counts;           // [E + 1]   rows per group (group E = shared)
   int *offsets;          // [E + 2]   exclusive prefix of counts
   int *fill;             // [E + 1]   scatter cursors
-  int *pos;              // [n][k + 1] sorted row of each assignment (slot k = shared)
-  int *row_token;        // [rows_max] token of each sorted row
-  float *row_w;          // [rows_max] routing weight of each sorted row (1 for shared)
-  int *tile_prefix;      // [E + 2]   prefix over groups of 128-token tiles
-  int *n_tiles;          // [1]
-  __nv_bfloat16 *xs;     // [rows_max][D]   gathered bf16 activations
-  __nv_bfloat16 *hs;     // [rows_max][Fmax] SwiGLU outputs
-  __nv_bfloat16 *outs;   // [rows_max][D]   weighted expert outputs
+  int *pos;              // [n][k + 1] grouped row of each assignment (slot k = shared expert)
+  int *row_token;        // [rows_max] token of each grouped row
+  float *row_w;          // [rows_max] routing weight of each grouped row (1 for the shared expert)
+  int *tile_prefix;      // [E + 2]   prefix over groups of kPfBN-row token tiles
+  int *n_tiles;          // [1]       token tiles of the call
+  __nv_bfloat16 *xs;     // [rows_max + kPfBN][D]   gathered bf16 activations
+  __nv_bfloat16 *hs;     // [rows_max + kPfBN][Fmax] SwiGLU outputs (bf16)
+  __nv_bfloat16 *outs;   // [rows_max][D]   weighted expert outputs (bf16)
   int fmax;
+  int nsm;               // persistent grid of the GEMM kernels
 };
 
 struct PrefillArgs {
