@@ -384,6 +384,187 @@ def bench_verify(args, rank, world, local):
     return res
 
 
+# ------------------------------------------------------------------------------------ other workloads
+def _graph_time(moe, step, prep, W, K, world, local, prof_kind):
+    """Capture step() into a CUDA graph (with event pairs around kernel class prof_kind), replay W
+    warm-up and K timed steps (prep(p) before each), return (ms total max over ranks, kernel ms,
+    kernel launches of the last replay, clocks)."""
+    import torch
+
+    import expert_ffn_gemv_b200 as P
+
+    stream = torch.cuda.Stream()
+    P.moe_profile_enable(moe.h, 1 << prof_kind)
+    with torch.cuda.stream(stream):
+        prep(0)
+        step()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            step()
+        for p in range(W):
+            prep(p)
+            g.replay()
+        stream.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for p in range(K):
+                prep(W + p)
+                g.replay()
+            ev1.record(stream)
+        stream.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    _, kms, kcnt = P.moe_profile_read(moe.h, prof_kind)
+    P.moe_profile_enable(moe.h, False)
+    del g
+    return ms, kms, kcnt, clk.summary()
+
+
+def _base_result(wl, world, K, W, ms, metric_unit, value):
+    return {"metric": METRIC, "value": value, "unit": metric_unit, "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "data": "synthetic (seeded integer-hash generator, random-init weights)"}
+
+
+def bench_decode_layers(args, rank, world, local):
+    """1 token through 16 model-scale layers built from seeds 0-15 (one layer each); a step runs
+    the 16 layers (y_i = MoE_i(x_i)); the 16 layers' ~0.27 GB of active blocks defeat the L2."""
+    import torch
+
+    import expert_ffn_gemv_b200 as P
+
+    wl = synth.DECODE
+    nl = 16
+    moe = make_moe(wl, nl, 8)
+    load_stack(moe, wl, list(range(nl)), nl, layer_of=lambda i: 0)
+    dev = torch.device("cuda")
+    xs = [synth.gen_x_torch(wl, s, 1, 0, dev).contiguous() for s in range(nl)]
+    ys = torch.empty((nl, 1, wl.d_model), dtype=torch.float32, device=dev)
+
+    def step():
+        for i in range(nl):
+            moe.forward(i, xs[i], ys[i])
+
+    K, W = args.steps, args.warmup
+    ms, kms, kcnt, clocks = _graph_time(moe, step, lambda p: None, W, K, world, local, P.PROF_GATEUP)
+    counts = [torch.empty(wl.n_experts, dtype=torch.int32, device=dev) for _ in range(nl)]
+    for i in range(nl):
+        moe.forward(i, xs[i], ys[i], route=dict(counts=counts[i]))
+    u = np.array([int((c > 0).sum()) for c in counts]) + wl.n_shared
+    eb = wl.expert_bytes()
+    step_bytes = float((u * eb).sum())
+    gu_bytes = float((u * 2 * eb // 3).sum())
+    pk, kind = peaks()
+    gbs = step_bytes * K / (ms / 1e3) / 1e9
+    res = _base_result(wl, world, K, W, ms, "GB/s", sum_over_ranks(gbs, world))
+    res.update({"dtype": "q2 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
+                "config": {"workload": wl.name, "layers_per_step": nl, "seeds": "0-15", "tokens": 1,
+                           "bytes": "active-expert blocks (routed + shared) per layer",
+                           "l2": "16 distinct layers per step"},
+                "tokens_per_s_one_layer": K * nl / (ms / 1e3),
+                "us_per_layer": ms * 1e3 / (K * nl),
+                "roofline": {"kernel": "k_gateup", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                             "peak_kind": kind,
+                             "achieved": gu_bytes / (kms / 1e3) / 1e9 if kms else None,
+                             "frac": gu_bytes / (kms / 1e3) / 1e9 / pk["hbm_gbs"] if kms else None,
+                             "avg_launch_us": kms / max(kcnt, 1) * 1e3},
+                "hbm_frac_whole_layer": gbs / pk["hbm_gbs"], "clocks": clocks, "gpu_launches": K * nl * 4})
+    moe.close()
+    return res
+
+
+def bench_codebook(args, rank, world, local):
+    """3.5-bit codebook blocks: 1 and 8 tokens through 48 model-scale layers applied to the same x
+    (no residual chain: the synthetic codebook weights make a norm-free chain overflow)."""
+    import torch
+
+    import expert_ffn_gemv_b200 as P
+
+    wl = synth.CODEBOOK
+    nl = args.layers
+    moe = make_moe(wl, nl, 8)
+    load_stack(moe, wl, args.seed, nl)
+    dev = torch.device("cuda")
+    K, W = args.steps, args.warmup
+    out = {}
+    pk, kind = peaks()
+    for n in (1, 8):
+        x = synth.gen_x_torch(wl, args.seed, n, 0, dev).contiguous()
+        ys = torch.empty((nl, n, wl.d_model), dtype=torch.float32, device=dev)
+
+        def step():
+            for i in range(nl):
+                moe.forward(i, x, ys[i])
+
+        ms, kms, kcnt, clocks = _graph_time(moe, step, lambda p: None, W, K, world, local, P.PROF_GATEUP)
+        counts = [torch.empty(wl.n_experts, dtype=torch.int32, device=dev) for _ in range(nl)]
+        for i in range(nl):
+            moe.forward(i, x, ys[i], route=dict(counts=counts[i]))
+        u = np.array([int((c > 0).sum()) for c in counts]) + wl.n_shared
+        eb = wl.expert_bytes()
+        gbs = float((u * eb).sum()) * K / (ms / 1e3) / 1e9
+        gu = float((u * 2 * eb // 3).sum())
+        out[n] = {"tokens_per_s": sum_over_ranks(n * K / (ms / 1e3), world), "ms_per_step": ms / K, "gbs": gbs,
+                  "frac": gbs / pk["hbm_gbs"], "gateup_gbs": gu / (kms / 1e3) / 1e9 if kms else None,
+                  "clocks": clocks}
+    res = _base_result(wl, world, K, W, out[8]["ms_per_step"] * K, "tokens/s", out[8]["tokens_per_s"])
+    res.update({"dtype": "cb35 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
+                "config": {"workload": wl.name, "layers": nl, "tokens": [1, 8], "chain": "independent layers"},
+                "by_tokens": out, "gpu_launches": K * nl * 4,
+                "roofline": {"kernel": "k_gateup", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                             "peak_kind": kind, "achieved": out[8]["gateup_gbs"],
+                             "frac": out[8]["gateup_gbs"] / pk["hbm_gbs"] if out[8]["gateup_gbs"] else None}})
+    moe.close()
+    return res
+
+
+def bench_prefill(args, rank, world, local):
+    """Prompt chunks (default 8,192 tokens; --chunk 1180 for the short one) through the 48-layer
+    stack, grouped tensor-core path."""
+    import torch
+
+    import expert_ffn_gemv_b200 as P
+
+    wl = synth.PREFILL
+    nl, n = args.layers, args.chunk
+    moe = make_moe(wl, nl, max(n, 9))
+    load_stack(moe, wl, args.seed, nl)
+    dev = torch.device("cuda")
+    K, W = args.steps, args.warmup
+    xs = torch.stack([synth.gen_x_torch(wl, args.seed, n, 1000 * rank + p, dev) for p in range(2)]).contiguous()
+    x_in = torch.empty((n, wl.d_model), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((n, wl.d_model), dtype=torch.float32, device=dev)
+
+    def step():
+        moe.forward_stack(0, nl, x_in, out)
+
+    ms, kms, kcnt, clocks = _graph_time(moe, step, lambda p: x_in.copy_(xs[p % 2]), W, K, world, local,
+                                        P.PROF_GATEUP)
+    rows = n * (wl.top_k + wl.n_shared)
+    flop_gu = 2.0 * rows * 2 * wl.d_ff * wl.d_model        # per layer, gate + up
+    flop_layer = 2.0 * rows * 3 * wl.d_ff * wl.d_model + 2.0 * n * wl.n_experts * wl.d_model
+    pk, kind = peaks()
+    peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    tfl = flop_layer * nl * K / (ms / 1e3) / 1e12
+    gu_tf = flop_gu * kcnt / (kms / 1e3) / 1e12 if kms else None
+    res = _base_result(wl, world, K, W, ms, "tokens/s", sum_over_ranks(n * K / (ms / 1e3), world))
+    res.update({"dtype": "bf16 operands (dequantised q2), f32 accumulate (tcgen05)",
+                "config": {"workload": wl.name, "layers": nl, "chunk_tokens": n,
+                           "l2": "each chunk reads the whole 36 GB stack"},
+                "tflops_whole_step": tfl, "frac_of_sustained_peak": tfl / peak_tf,
+                "roofline": {"kernel": "k_pf_gemm<gate/up>", "bound": "tensor", "unit": "TFLOP/s",
+                             "peak": peak_tf, "peak_kind": kind + " sustained bf16", "achieved": gu_tf,
+                             "frac": gu_tf / peak_tf if gu_tf else None,
+                             "avg_launch_us": kms / max(kcnt, 1) * 1e3, "traffic": None},
+                "clocks": clocks, "gpu_launches": K * nl * 8})
+    moe.close()
+    return res
+
+
 # ------------------------------------------------------------------------------------ reference arm
 def bench_reference(args):
     """The fp64 CPU oracle as the reference arm: each step = 8 tokens through one layer of the
@@ -438,7 +619,8 @@ def main():
     ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["verify"], default="verify")
+    ap.add_argument("--workload", choices=["verify", "decode", "codebook", "prefill"], default="verify")
+    ap.add_argument("--chunk", type=int, default=8192, help="prefill chunk tokens")
     ap.add_argument("--layers", type=int, default=48)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -455,7 +637,9 @@ def main():
         print(json.dumps(bench_reference(args)), flush=True)
         return 0
     rank, world, local = dist_setup(args.gpus)
-    res = bench_verify(args, rank, world, local)
+    fn = {"verify": bench_verify, "decode": bench_decode_layers, "codebook": bench_codebook,
+          "prefill": bench_prefill}[args.workload]
+    res = fn(args, rank, world, local)
     if world > 1:
         import torch.distributed as dist
 

@@ -325,23 +325,33 @@ __device__ __forceinline__ void cp_async_wait() {
 // ------------------------------------------------------------------------------------------
 // grouped GEMM on tcgen05.  MODE 0: gate + up (two A matrices, SwiGLU epilogue -> hs);
 // MODE 1: down (one A matrix, epilogue scales by the row's routing weight -> outs).
-// One CTA per SM walks the (token tile, row tile) list; a 3-stage ring holds, per K-step of 64:
-// the raw blocks (bulk copy), the dequantised bf16 A tiles and the bf16 B tile (cp.async).
+// One CTA per SM walks its (token tile, row tile) list as one stream of K-steps (64 deep).  Three
+// rings run over that stream, continuing across tiles:
+//   raw blocks  (4 slots, bulk copies issued 3 steps ahead; read by the dequantisation),
+//   B tiles     (4 slots, 16-byte cp.async issued 2 steps ahead, 128B-swizzled),
+//   A tiles     (2 slots, bf16 written by the dequantisation, 128B-swizzled).
+// A B slot or an A slot is refilled only once the MMA of two steps earlier has completed, so
+// the tensor core multiplies step j-1 while the threads prepare step j.
 // ------------------------------------------------------------------------------------------
 constexpr int kPfThreads = 256;
-constexpr int kPfStages = 3;
-constexpr int kPfAhead = 2;  // K-steps in flight ahead of the one being multiplied
+constexpr int kRawSlots = 4, kRawAhead = 3;
+constexpr int kBSlots = 4, kBAhead = 2;
+constexpr int kASlots = 2;
 
 template <int FMT, int MODE>
 struct PfPlan {
   static constexpr int NM = MODE == 0 ? 2 : 1;
-  static constexpr int kATile = 128 * 128;   // bytes of one 128 x 64 bf16 tile
-  static constexpr int kBTile = kPfBN * 128;
+  static constexpr int kATile = 128 * 128;     // bytes of one 128 x 64 bf16 tile
+  static constexpr int kBTile = kPfBN * 128;   // kPfBN x 64 bf16
   static constexpr int kRawA = 128 * 16, kRawS = 128 * 4, kRawG = FMT == MOE_FMT_CB35_32 ? 128 * 8 : 0;
-  static constexpr int kRaw = NM * (kRawA + kRawS + kRawG);
-  static constexpr int kStage = NM * kATile + kBTile + ((kRaw + 1023) & ~1023);
-  static constexpr int kHead = 2048;  // barriers and TMEM address [0, 1024), grid table [1024, 2048)
-  static constexpr int kBytes = kHead + 1024 + kPfStages * kStage;  // +1024 for alignment
+  static constexpr int kRawM = kRawA + kRawS + kRawG;       // one matrix
+  static constexpr int kRaw = NM * kRawM;                   // bytes per raw slot
+  static constexpr int kRawSlot = (kRaw + 127) & ~127;
+  static constexpr int kHead = 2048;  // barriers + TMEM address [0, 1024), grid table [1024, 2048)
+  static constexpr int kAOff = kHead;
+  static constexpr int kBOff = kAOff + kASlots * NM * kATile;
+  static constexpr int kRawOff = kBOff + kBSlots * kBTile;
+  static constexpr int kBytes = 1024 + kRawOff + kRawSlots * kRawSlot;  // + 1024 for alignment
   static constexpr uint32_t kTmemCols = MODE == 0 ? 2 * kPfBN : kPfBN;
 };
 
@@ -368,31 +378,71 @@ __device__ __forceinline__ bool pf_tile(const PrefillArgs &a, int tile, int mtil
   return pt.cnt > 0;
 }
 
+// A position in this CTA's stream of K-steps: tile (blockIdx.x + i * gridDim.x) and step s.
+struct PfCursor {
+  int tile, s, nc, eidx;
+  bool shared;
+  PfTile pt;
+  bool valid;
+};
+
+template <int MODE>
+__device__ __forceinline__ void pf_seek(const PrefillArgs &a, int mtiles, int total, PfCursor &c) {
+  c.valid = false;
+  while (c.tile < total) {
+    if (pf_tile(a, c.tile, mtiles, c.pt)) {
+      c.shared = a.sh.n_shared && c.pt.g == a.sh.e;
+      const int f = c.shared ? a.L.shared.f : a.L.routed.f;
+      if (MODE == 1 || c.pt.mt * kTileRows < f) {
+        c.eidx = c.shared ? 0 : c.pt.g;
+        c.nc = (MODE == 0 ? a.sh.d : f) / kChunk;
+        c.s = 0;
+        c.valid = true;
+        return;
+      }
+    }
+    c.tile += gridDim.x;
+  }
+}
+
+template <int MODE>
+__device__ __forceinline__ void pf_next(const PrefillArgs &a, int mtiles, int total, PfCursor &c) {
+  if (!c.valid) return;
+  if (++c.s == c.nc) {
+    c.tile += gridDim.x;
+    pf_seek<MODE>(a, mtiles, total, c);
+  }
+}
+
 template <int FMT, int MODE>
 __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(PrefillArgs a) {
   using PL = PfPlan<FMT, MODE>;
   constexpr int NM = PL::NM;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem);            // [kPfStages]
-  uint64_t *mma_done = raw_full + kPfStages;                           // [kPfStages]
-  uint64_t *acc_full = mma_done + kPfStages;                           // [1]
+  uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem);            // [kRawSlots]
+  uint64_t *mma_done = raw_full + kRawSlots;                           // [kBSlots] (step j -> j % 4)
+  uint64_t *acc_full = mma_done + kBSlots;                             // [1]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 128);
   int8_t *grid_s = reinterpret_cast<int8_t *>(smem + 1024);            // 256 x 4 (CB35)
-  unsigned char *stages = smem + PL::kHead;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int D = a.sh.d, E = a.sh.e;
-
+  const int D = a.sh.d;
   const int fmax = a.ws.fmax;
   const int mtiles = MODE == 0 ? fmax / kTileRows : D / kTileRows;
   const int total = __ldcg(a.ws.n_tiles) * mtiles;
-  if (blockIdx.x >= total) return;
+  const __nv_bfloat16 *bsrc = MODE == 0 ? a.ws.xs : a.ws.hs;
+  const int bstride = MODE == 0 ? D : fmax;
+
+  PfCursor cons, craw, cb;
+  cons.tile = blockIdx.x;
+  pf_seek<MODE>(a, mtiles, total, cons);
+  if (!cons.valid) return;  // no tile for this CTA (uniform)
+  craw = cons;
+  cb = cons;
 
   if (tid == 0) {
-    for (int s = 0; s < kPfStages; ++s) {
-      mbar_init(&raw_full[s], 1);
-      mbar_init(&mma_done[s], 1);
-    }
+    for (int s = 0; s < kRawSlots; ++s) mbar_init(&raw_full[s], 1);
+    for (int s = 0; s < kBSlots; ++s) mbar_init(&mma_done[s], 1);
     mbar_init(acc_full, 1);
     fence_barrier_init();
   }
@@ -408,161 +458,166 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(PrefillArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  uint32_t gstep = 0;      // ring position of the next tile's first K-step
-  uint32_t tiles_done = 0;
-  int64_t last_issued = -1;     // highest ring position whose copies were issued
-  int64_t last_committed = -1;  // highest ring position whose MMAs were committed
-  bool failed = false;
-
-  for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-    PfTile pt;
-    if (!pf_tile(a, tile, mtiles, pt)) continue;
-    const bool shared = a.sh.n_shared && pt.g == E;
-    const ExpertGroup &G = shared ? a.L.shared : a.L.routed;
-    const int eidx = shared ? 0 : pt.g;
-    if (MODE == 0 && pt.mt * kTileRows >= G.f) continue;  // row tile beyond this group's d_ff
-    const int K = MODE == 0 ? D : G.f;
-    const int nc = K / kChunk;                      // K-steps (64 each)
-    const int nN = (pt.cnt + 15) & ~15;             // MMA N for this tile
-    const __nv_bfloat16 *bsrc = MODE == 0 ? a.ws.xs : a.ws.hs;
-    const int bstride = MODE == 0 ? D : fmax;
-    const uint32_t idesc = idesc_bf16(nN);
-
-    // issue the copies of K-step s of this tile into ring slot (gstep0 + s) % kPfStages
-    auto issue = [&](int s, uint32_t ring) {
-      const int b = ring % kPfStages;
-      unsigned char *st = stages + b * PL::kStage;
-      unsigned char *raw = st + NM * PL::kATile + PL::kBTile;
-      if (ring >= kPfStages) {  // the MMA that last read this slot must be done
-        const uint32_t par = ((ring - kPfStages) / kPfStages) & 1u;
-        if (!mbar_wait_bounded(&mma_done[b], par, a.spin_limit)) {
-          flag_error(a.err, kErrTimeout);
-          mbar_wait_bounded(&mma_done[b], par, kDrainLimit);
-        }
-      }
-      if (tid == 0) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&raw_full[b], PL::kRaw);
-        const int64_t slot0 = (static_cast<int64_t>(pt.mt) * nc + s) * kTileRows;
+  // ---- producers
+  auto issue_raw = [&](const PfCursor &c, uint32_t j) {  // thread 0
+    const int slot = j % kRawSlots;
+    unsigned char *raw = smem + PL::kRawOff + slot * PL::kRawSlot;
+    const ExpertGroup &G = c.shared ? a.L.shared : a.L.routed;
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&raw_full[slot], PL::kRaw);
+    const int64_t slot0 = (static_cast<int64_t>(c.pt.mt) * c.nc + c.s) * kTileRows;
 #pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          const int64_t mat = static_cast<int64_t>(eidx) * 3 + (MODE == 0 ? m : 2);
-          unsigned char *rm = raw + m * (PL::kRawA + PL::kRawS + PL::kRawG);
-          bulk_g2s(rm, G.a + mat * G.a_mat + slot0 * 16, PL::kRawA, &raw_full[b]);
-          bulk_g2s(rm + PL::kRawA, G.s + mat * G.s_mat + slot0, PL::kRawS, &raw_full[b]);
-          if (FMT == MOE_FMT_CB35_32) bulk_g2s(rm + PL::kRawA + PL::kRawS, G.g + mat * G.g_mat + slot0, PL::kRawG, &raw_full[b]);
-        }
-      }
-      last_issued = ring;
-      // B tile: kPfBN rows x 128 bytes, swizzled, 16-byte async copies
-      unsigned char *bt = st + NM * PL::kATile;
-      const int k0 = s * kChunk;
+    for (int m = 0; m < NM; ++m) {
+      const int64_t mat = static_cast<int64_t>(c.eidx) * 3 + (MODE == 0 ? m : 2);
+      unsigned char *rm = raw + m * PL::kRawM;
+      bulk_g2s(rm, G.a + mat * G.a_mat + slot0 * 16, PL::kRawA, &raw_full[slot]);
+      bulk_g2s(rm + PL::kRawA, G.s + mat * G.s_mat + slot0, PL::kRawS, &raw_full[slot]);
+      if (FMT == MOE_FMT_CB35_32) bulk_g2s(rm + PL::kRawA + PL::kRawS, G.g + mat * G.g_mat + slot0, PL::kRawG, &raw_full[slot]);
+    }
+  };
+  auto issue_b = [&](const PfCursor &c, uint32_t j) {  // all threads
+    if (c.valid) {
+      unsigned char *bt = smem + PL::kBOff + (j % kBSlots) * PL::kBTile;
+      const int k0 = c.s * kChunk;
 #pragma unroll
       for (int z = 0; z < kPfBN * 8 / kPfThreads; ++z) {
-        const int q = tid + kPfThreads * z, r = q >> 3, c = q & 7;
-        const __nv_bfloat16 *src = bsrc + static_cast<int64_t>(pt.rows0 + r) * bstride + k0 + 8 * c;
-        cp_async16(bt + sw128_off(r, c), src);
+        const int q = tid + kPfThreads * z, r = q >> 3, cc = q & 7;
+        cp_async16(bt + sw128_off(r, cc), bsrc + static_cast<int64_t>(c.pt.rows0 + r) * bstride + k0 + 8 * cc);
       }
-      cp_async_commit();
-    };
-
-    const uint32_t g0 = gstep;
-    for (int s = 0; s < kPfAhead; ++s) {
-      if (s < nc) issue(s, g0 + s);
-      else cp_async_commit();
     }
-    for (int s = 0; s < nc; ++s) {
-      const uint32_t ring = g0 + s;
-      const int b = ring % kPfStages;
-      unsigned char *st = stages + b * PL::kStage;
-      unsigned char *raw = st + NM * PL::kATile + PL::kBTile;
-      if (s + kPfAhead < nc) issue(s + kPfAhead, ring + kPfAhead);
-      else cp_async_commit();
-      cp_async_wait<kPfAhead>();
-      const bool ok = mbar_wait_bounded(&raw_full[b], (ring / kPfStages) & 1u, a.spin_limit);
-      if (__syncthreads_or(!ok)) {
-        // give up: wait (bounded) for every bulk copy still in flight, then leave the tile loop
-        if (tid == 0) flag_error(a.err, kErrTimeout);
-        for (int64_t r = ring; r <= last_issued; ++r)
-          mbar_wait_bounded(&raw_full[r % kPfStages], static_cast<uint32_t>(r / kPfStages) & 1u, kDrainLimit);
-        failed = true;
-        break;
+    cp_async_commit();  // one group per step (empty past the end), so wait_group counts steps
+  };
+
+  uint32_t j_raw = 0, j_b = 0;  // next stream position of each producer
+  for (int i = 0; i < kRawAhead && craw.valid; ++i) {
+    if (tid == 0) issue_raw(craw, j_raw);
+    ++j_raw;
+    pf_next<MODE>(a, mtiles, total, craw);
+  }
+  for (int i = 0; i < kBAhead; ++i) {
+    issue_b(cb, j_b);
+    ++j_b;
+    pf_next<MODE>(a, mtiles, total, cb);
+  }
+
+  uint32_t j = 0, tiles_done = 0;
+  int64_t last_committed = -1;
+  bool failed = false;
+  while (cons.valid) {
+    // the MMA of step j-2 read A slot j % 2 and B slot (j + 2) % 4
+    if (j >= 2) {
+      const uint32_t jm = j - 2;
+      if (!mbar_wait_bounded(&mma_done[jm % kBSlots], (jm / kBSlots) & 1u, a.spin_limit)) {
+        flag_error(a.err, kErrTimeout);
+        mbar_wait_bounded(&mma_done[jm % kBSlots], (jm / kBSlots) & 1u, kDrainLimit);
       }
-      // dequantise: thread -> (row r, block h) of each matrix; 32 weights -> 4 swizzled chunks
-      {
-        const int r = tid & 127, h = tid >> 7;
+    }
+    if (craw.valid) {
+      if (tid == 0) issue_raw(craw, j_raw);
+      ++j_raw;
+      pf_next<MODE>(a, mtiles, total, craw);
+    }
+    issue_b(cb, j_b);
+    ++j_b;
+    pf_next<MODE>(a, mtiles, total, cb);
+    cp_async_wait<kBAhead>();  // this step's B tile has landed
+    const int rslot = j % kRawSlots;
+    const bool ok = mbar_wait_bounded(&raw_full[rslot], (j / kRawSlots) & 1u, a.spin_limit);
+    if (__syncthreads_or(!ok)) {
+      // give up: wait (bounded) for the bulk copies still in flight, then leave
+      if (tid == 0) flag_error(a.err, kErrTimeout);
+      for (uint32_t r = j; r < j_raw; ++r)
+        mbar_wait_bounded(&raw_full[r % kRawSlots], (r / kRawSlots) & 1u, kDrainLimit);
+      failed = true;
+      break;
+    }
+    // dequantise: thread -> (row r, block h) of each matrix; 32 weights -> 4 swizzled chunks
+    unsigned char *at0 = smem + PL::kAOff + (j % kASlots) * NM * PL::kATile;
+    {
+      const unsigned char *raw = smem + PL::kRawOff + rslot * PL::kRawSlot;
+      const int r = tid & 127, h = tid >> 7;
 #pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          const unsigned char *rm = raw + m * (PL::kRawA + PL::kRawS + PL::kRawG);
-          const uint4 A = reinterpret_cast<const uint4 *>(rm)[r];
-          const __half2 sc2 = reinterpret_cast<const __half2 *>(rm + PL::kRawA)[r];
-          const float sc = __half2float(h ? __high2half(sc2) : __low2half(sc2));
-          const uint32_t w0 = h ? A.z : A.x, w1 = h ? A.w : A.y;
-          uint32_t sgn = 0;
-          if (FMT == MOE_FMT_CB35_32) {
-            const uint2 G2 = reinterpret_cast<const uint2 *>(rm + PL::kRawA + PL::kRawS)[r];
-            sgn = h ? G2.y : G2.x;
-          }
-          unsigned char *at = st + m * PL::kATile;
+      for (int m = 0; m < NM; ++m) {
+        const unsigned char *rm = raw + m * PL::kRawM;
+        const uint4 A = reinterpret_cast<const uint4 *>(rm)[r];
+        const __half2 sc2 = reinterpret_cast<const __half2 *>(rm + PL::kRawA)[r];
+        const float sc = __half2float(h ? __high2half(sc2) : __low2half(sc2));
+        const uint32_t w0 = h ? A.z : A.x, w1 = h ? A.w : A.y;
+        uint32_t sgn = 0;
+        if (FMT == MOE_FMT_CB35_32) {
+          const uint2 G2 = reinterpret_cast<const uint2 *>(rm + PL::kRawA + PL::kRawS)[r];
+          sgn = h ? G2.y : G2.x;
+        }
+        unsigned char *at = at0 + m * PL::kATile;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            float v[8];
+        for (int cc = 0; cc < 4; ++cc) {
+          float v[8];
+          if (FMT == MOE_FMT_Q2_32) {
+            // float(2^23 + q) by exponent bias, minus 2^23: the code q exactly; then s (q - 1.5)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const int p = 8 * cc + i;  // weight within the block
-              if (FMT == MOE_FMT_Q2_32) {
-                const uint32_t w = p < 16 ? w0 : w1;
-                const int pw = p & 15, kk = pw >> 2, j = pw & 3;
-                const uint32_t q = (w >> (8 * j + 2 * kk)) & 3u;
-                v[i] = sc * (static_cast<float>(q) - 1.5f);
-              } else {
-                const int g = p >> 2, j = p & 3;
-                const uint32_t iw = g < 4 ? w0 : w1;
-                const uint32_t idx = (iw >> (8 * (g & 3))) & 0xFFu;
-                const float gv = static_cast<float>(grid_s[idx * 4 + j]);
-                const float sg = ((sgn >> (8 * j + g)) & 1u) ? -1.f : 1.f;
-                v[i] = sc * sg * gv;
+              const uint32_t w = p < 16 ? w0 : w1;
+              const int pw = p & 15, kk = pw >> 2, jj = pw & 3;
+              const float q = __uint_as_float(((w >> (8 * jj + 2 * kk)) & 3u) | 0x4B000000u) - 8388608.0f;
+              v[i] = fmaf(sc, q, -1.5f * sc);
+            }
+          } else {
+            // two groups of 4: signed grid bytes (sign mask applied per byte), then s * value
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+              const int g = 2 * cc + gg;
+              const uint32_t iw = g < 4 ? w0 : w1;
+              const uint32_t idx = (iw >> (8 * (g & 3))) & 0xFFu;
+              const uint32_t gw = reinterpret_cast<const uint32_t *>(grid_s)[idx];
+              const uint32_t mk = prmt_sign_bytes(sgn << (7 - g));
+              const uint32_t sb = ((gw ^ mk) + (mk & 0x01010101u)) ^ 0x80808080u;  // signed -> biased bytes
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                const float q = __uint_as_float(((sb >> (8 * jj)) & 0xFFu) | 0x4B000000u) - 8388736.0f;  // 2^23 + 128
+                v[4 * gg + jj] = sc * q;
               }
             }
-            uint4 o;
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]), b3 = __floats2bfloat162_rn(v[6], v[7]);
-            o.x = *reinterpret_cast<uint32_t *>(&b0);
-            o.y = *reinterpret_cast<uint32_t *>(&b1);
-            o.z = *reinterpret_cast<uint32_t *>(&b2);
-            o.w = *reinterpret_cast<uint32_t *>(&b3);
-            *reinterpret_cast<uint4 *>(at + sw128_off(r, 4 * h + cc)) = o;
           }
+          uint4 o;
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]), b3 = __floats2bfloat162_rn(v[6], v[7]);
+          o.x = *reinterpret_cast<uint32_t *>(&b0);
+          o.y = *reinterpret_cast<uint32_t *>(&b1);
+          o.z = *reinterpret_cast<uint32_t *>(&b2);
+          o.w = *reinterpret_cast<uint32_t *>(&b3);
+          *reinterpret_cast<uint4 *>(at + sw128_off(r, 4 * h + cc)) = o;
         }
       }
-      fence_proxy_async_smem();  // generic-proxy writes (dequant, cp.async) -> tensor core reads
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t bt = smem_u32(st + NM * PL::kATile);
+    }
+    fence_proxy_async_smem();  // generic-proxy writes (dequant, cp.async) -> tensor core reads
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t bt = smem_u32(smem + PL::kBOff + (j % kBSlots) * PL::kBTile);
+      const uint32_t idesc = idesc_bf16((cons.pt.cnt + 15) & ~15);
 #pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          const uint32_t at = smem_u32(st + m * PL::kATile);
+      for (int m = 0; m < NM; ++m) {
+        const uint32_t at = smem_u32(at0 + m * PL::kATile);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma(tmem + m * kPfBN, sw128_desc(at + 32 * kk), sw128_desc(bt + 32 * kk), idesc, (s > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&mma_done[b]);
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma(tmem + m * kPfBN, sw128_desc(at + 32 * kk), sw128_desc(bt + 32 * kk), idesc,
+                 (cons.s > 0 || kk > 0) ? 1u : 0u);
       }
-      last_committed = ring;
+      tc_commit(&mma_done[j % kBSlots]);
     }
-    gstep = g0 + nc;
-    if (failed) break;
-    // epilogue
-    if (tid == 0) tc_commit(acc_full);
-    if (!mbar_wait_bounded(acc_full, tiles_done & 1u, a.spin_limit)) {
-      flag_error(a.err, kErrTimeout);
-      mbar_wait_bounded(acc_full, tiles_done & 1u, kDrainLimit);
-    }
-    ++tiles_done;
-    tc_fence_after();
-    {
-      const int q = warp & 3;                 // TMEM lane quarter of this warp
+    last_committed = j;
+    if (cons.s == cons.nc - 1) {
+      // epilogue of the tile
+      if (tid == 0) tc_commit(acc_full);
+      if (!mbar_wait_bounded(acc_full, tiles_done & 1u, a.spin_limit)) {
+        flag_error(a.err, kErrTimeout);
+        mbar_wait_bounded(acc_full, tiles_done & 1u, kDrainLimit);
+      }
+      ++tiles_done;
+      tc_fence_after();
+      const PfTile &pt = cons.pt;
+      const int q = warp & 3;  // TMEM lane quarter of this warp
       const int row = pt.mt * kTileRows + 32 * q + lane;
       const int c_begin = (warp >> 2) * (kPfBN / 2), c_end = c_begin + kPfBN / 2;
       for (int c0 = c_begin; c0 < c_end; c0 += 16) {
@@ -574,29 +629,29 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(PrefillArgs a) {
           float u[16];
           tmem_ld16(ta + kPfBN, u);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (c0 + i < pt.cnt) {
-              const float hv = silu_f(g[i]) * u[i];
-              a.ws.hs[static_cast<int64_t>(pt.rows0 + c0 + i) * fmax + row] = __float2bfloat16_rn(hv);
-            }
-          }
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < pt.cnt)
+              a.ws.hs[static_cast<int64_t>(pt.rows0 + c0 + i) * fmax + row] = __float2bfloat16_rn(silu_f(g[i]) * u[i]);
         } else {
+          float wr[16];  // routing weights of the 16 rows, loaded together
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (c0 + i < pt.cnt) {
-              const int pr = pt.rows0 + c0 + i;
-              a.ws.outs[static_cast<int64_t>(pr) * D + row] = __float2bfloat16_rn(g[i] * __ldcg(a.ws.row_w + pr));
-            }
-          }
+          for (int i = 0; i < 16; ++i) wr[i] = c0 + i < pt.cnt ? __ldcg(a.ws.row_w + pt.rows0 + c0 + i) : 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < pt.cnt)
+              a.ws.outs[static_cast<int64_t>(pt.rows0 + c0 + i) * D + row] = __float2bfloat16_rn(g[i] * wr[i]);
         }
       }
+      tc_fence_before();
+      __syncthreads();
     }
-    tc_fence_before();
-    __syncthreads();
+    ++j;
+    pf_next<MODE>(a, mtiles, total, cons);
   }
+  (void)failed;
   // drain: every committed MMA must be complete before the TMEM is released
   if (last_committed >= 0)
-    mbar_wait_bounded(&mma_done[last_committed % kPfStages], static_cast<uint32_t>(last_committed / kPfStages) & 1u,
+    mbar_wait_bounded(&mma_done[last_committed % kBSlots], static_cast<uint32_t>(last_committed / kBSlots) & 1u,
                       kDrainLimit);
   cp_async_wait<0>();
   tc_fence_before();

@@ -7,7 +7,7 @@
 
 namespace moe {
 
-constexpr int kPfBN = 128;  // tokens per GEMM tile (MMA N, at most)
+constexpr int kPfBN = 256;  // tokens per GEMM tile (MMA N, at most)
 
 // Prompt-chunk workspace.  Assignments (token, slot) are grouped by expert with a counting sort;
 // the shared expert is group E (all tokens, token order).  Rows of the grouped operands are
