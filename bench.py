@@ -151,24 +151,33 @@ def barrier(world):
         dist.barrier()
 
 
+def _reduce_device():
+    import torch
+    import torch.distributed as dist
+
+    return torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+
+
 def max_over_ranks(v: float, world: int) -> float:
+    """Max of a per-rank value (the job's time is the slowest rank's)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 def sum_over_ranks(v: float, world: int) -> float:
+    """Sum of a per-rank value (tokens processed by all replicas)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
