@@ -326,6 +326,13 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
   {
     Carve c{static_cast<char *>(h->ws_mem)};
     plan_workspace(h, c);
+    if (g.max_tokens > kDecodeMaxTokens) {
+      cudaError_t te = make_prefill_tensor_maps(h->pws, g.d_model);
+      if (te != cudaSuccess) {
+        s = cuda_fail(h, te, "tensor maps");
+        goto fail_out;
+      }
+    }
     cudaError_t ge = decode_grid_sizes(g.fmt, g.d_model, h->gu_splits, h->dws.fmax, h->dws.umax, g.n_shared, g.d_ff,
                                        g.shared_d_ff, &h->dws.grid_gu, &h->dws.grid_down);
     if (ge != cudaSuccess) {

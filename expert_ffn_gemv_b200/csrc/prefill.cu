@@ -323,36 +323,39 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // ------------------------------------------------------------------------------------------
-// grouped GEMM on tcgen05.  MODE 0: gate + up (two A matrices, SwiGLU epilogue -> hs);
-// MODE 1: down (one A matrix, epilogue scales by the row's routing weight -> outs).
-// One CTA per SM walks its (token tile, row tile) list as one stream of K-steps (64 deep).  Three
-// rings run over that stream, continuing across tiles:
-//   raw blocks  (4 slots, bulk copies issued 3 steps ahead; read by the dequantisation),
-//   B tiles     (4 slots, 16-byte cp.async issued 2 steps ahead, 128B-swizzled),
-//   A tiles     (2 slots, bf16 written by the dequantisation, 128B-swizzled).
-// A B slot or an A slot is refilled only once the MMA of two steps earlier has completed, so
-// the tensor core multiplies step j-1 while the threads prepare step j.
+// grouped GEMM on tcgen05, warp-specialised.  MODE 0: gate + up (two A matrices, SwiGLU
+// epilogue -> hs); MODE 1: down (one A matrix, epilogue x routing weight -> outs).
+// One CTA per SM walks its (token tile, row tile) list as one stream of 64-deep K-steps through a
+// ring of stages.  Warp roles:
+//   warp 12       producer: per stage, the raw blocks of the A matrices (bulk copies) and the B
+//                 tile (one 2-D TMA load, 128-byte swizzle) on one "full" barrier
+//   warps 4..11   dequantisation: raw blocks -> bf16 A tiles (128-byte swizzle), then "a_ready"
+//   warp 13       MMA: tcgen05.mma kind::f16, M = 128, N <= 256, fp32 accumulators in TMEM;
+//                 the commit of a stage's MMAs frees the stage ("empty")
+//   warps 0..3    epilogue: TMEM -> registers -> SwiGLU / weight -> global (bf16)
+// Accumulators: MODE 0 uses all 512 TMEM columns (gate + up at N = 256), MODE 1 double-buffers
+// (2 x 256 columns) so the epilogue of a tile overlaps the next tile's MMAs.  Every wait is
+// bounded; a role that gives up raises a shared abort flag that ends the others' waits.
 // ------------------------------------------------------------------------------------------
-constexpr int kPfThreads = 256;
-constexpr int kRawSlots = 4, kRawAhead = 3;
-constexpr int kBSlots = 4, kBAhead = 2;
-constexpr int kASlots = 2;
+constexpr int kPfWarps = 14;
+constexpr int kPfThreads = 32 * kPfWarps;
+constexpr int kWarpEpi0 = 0, kWarpDeq0 = 4, kWarpProd = 12, kWarpMma = 13;
+constexpr int kDeqThreads = 256;
 
 template <int FMT, int MODE>
 struct PfPlan {
   static constexpr int NM = MODE == 0 ? 2 : 1;
-  static constexpr int kATile = 128 * 128;     // bytes of one 128 x 64 bf16 tile
-  static constexpr int kBTile = kPfBN * 128;   // kPfBN x 64 bf16
+  static constexpr int kStages = MODE == 0 ? 3 : 4;
+  static constexpr int kAcc = MODE == 0 ? 1 : 2;               // accumulator buffers
+  static constexpr int kATile = 128 * 128;                      // 128 x 64 bf16
+  static constexpr int kBTile = kPfBN * 128;                    // kPfBN x 64 bf16
   static constexpr int kRawA = 128 * 16, kRawS = 128 * 4, kRawG = FMT == MOE_FMT_CB35_32 ? 128 * 8 : 0;
-  static constexpr int kRawM = kRawA + kRawS + kRawG;       // one matrix
-  static constexpr int kRaw = NM * kRawM;                   // bytes per raw slot
-  static constexpr int kRawSlot = (kRaw + 127) & ~127;
-  static constexpr int kHead = 2048;  // barriers + TMEM address [0, 1024), grid table [1024, 2048)
-  static constexpr int kAOff = kHead;
-  static constexpr int kBOff = kAOff + kASlots * NM * kATile;
-  static constexpr int kRawOff = kBOff + kBSlots * kBTile;
-  static constexpr int kBytes = 1024 + kRawOff + kRawSlots * kRawSlot;  // + 1024 for alignment
-  static constexpr uint32_t kTmemCols = MODE == 0 ? 2 * kPfBN : kPfBN;
+  static constexpr int kRawM = kRawA + kRawS + kRawG;
+  static constexpr int kRaw = NM * kRawM;
+  static constexpr int kStage = NM * kATile + kBTile + ((kRaw + 1023) & ~1023);
+  static constexpr int kHead = 2048;  // barriers, flags, TMEM address [0, 1024); grid [1024, 2048)
+  static constexpr int kBytes = 1024 + kHead + kStages * kStage;
+  static constexpr uint32_t kTmemCols = 512;
 };
 
 struct PfTile {
@@ -363,8 +366,7 @@ __device__ __forceinline__ bool pf_tile(const PrefillArgs &a, int tile, int mtil
   const int tt = tile / mtiles;
   pt.mt = tile % mtiles;
   const int G = a.sh.e + a.sh.n_shared;
-  // group g with tile_prefix[g] <= tt < tile_prefix[g + 1]
-  int lo = 0, hi = G;
+  int lo = 0, hi = G;  // group g with tile_prefix[g] <= tt < tile_prefix[g + 1]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (__ldcg(a.ws.tile_prefix + mid) <= tt) lo = mid; else hi = mid;
@@ -378,12 +380,11 @@ __device__ __forceinline__ bool pf_tile(const PrefillArgs &a, int tile, int mtil
   return pt.cnt > 0;
 }
 
-// A position in this CTA's stream of K-steps: tile (blockIdx.x + i * gridDim.x) and step s.
+// A tile of this CTA's list (blockIdx.x + i * gridDim.x) with its K-step count.
 struct PfCursor {
-  int tile, s, nc, eidx;
-  bool shared;
+  int tile, nc, eidx;
+  bool shared, valid;
   PfTile pt;
-  bool valid;
 };
 
 template <int MODE>
@@ -396,7 +397,6 @@ __device__ __forceinline__ void pf_seek(const PrefillArgs &a, int mtiles, int to
       if (MODE == 1 || c.pt.mt * kTileRows < f) {
         c.eidx = c.shared ? 0 : c.pt.g;
         c.nc = (MODE == 0 ? a.sh.d : f) / kChunk;
-        c.s = 0;
         c.valid = true;
         return;
       }
@@ -406,44 +406,71 @@ __device__ __forceinline__ void pf_seek(const PrefillArgs &a, int mtiles, int to
 }
 
 template <int MODE>
-__device__ __forceinline__ void pf_next(const PrefillArgs &a, int mtiles, int total, PfCursor &c) {
-  if (!c.valid) return;
-  if (++c.s == c.nc) {
-    c.tile += gridDim.x;
-    pf_seek<MODE>(a, mtiles, total, c);
+__device__ __forceinline__ void pf_advance(const PrefillArgs &a, int mtiles, int total, PfCursor &c) {
+  c.tile += gridDim.x;
+  pf_seek<MODE>(a, mtiles, total, c);
+}
+
+// Bounded wait that also ends when another role raised the abort flag.
+__device__ __forceinline__ bool pf_wait(uint64_t *bar, uint32_t parity, uint64_t limit, volatile int *abort_flag,
+                                        uint32_t *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (static_cast<uint64_t>(clock64() - t0) > limit) {
+      *abort_flag = 1;
+      flag_error(err, kErrTimeout);
+      return false;
+    }
   }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(PrefillArgs a) {
+__global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant__ PrefillArgs a) {
   using PL = PfPlan<FMT, MODE>;
-  constexpr int NM = PL::NM;
+  constexpr int NM = PL::NM, NS = PL::kStages, NACC = PL::kAcc;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem);            // [kRawSlots]
-  uint64_t *mma_done = raw_full + kRawSlots;                           // [kBSlots] (step j -> j % 4)
-  uint64_t *acc_full = mma_done + kBSlots;                             // [1]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 128);
-  int8_t *grid_s = reinterpret_cast<int8_t *>(smem + 1024);            // 256 x 4 (CB35)
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);   // [NS] producer -> dequant + MMA
+  uint64_t *a_ready = full + NS;                          // [NS] dequant -> MMA
+  uint64_t *empty = a_ready + NS;                         // [NS] MMA commit -> producer
+  uint64_t *acc_full = empty + NS;                        // [NACC] MMA commit -> epilogue
+  uint64_t *acc_empty = acc_full + NACC;                  // [NACC] epilogue -> MMA
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
+  int8_t *grid_s = reinterpret_cast<int8_t *>(smem + 1024);
+  unsigned char *stages = smem + PL::kHead;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int D = a.sh.d;
-  const int fmax = a.ws.fmax;
+  const int D = a.sh.d, fmax = a.ws.fmax;
   const int mtiles = MODE == 0 ? fmax / kTileRows : D / kTileRows;
   const int total = __ldcg(a.ws.n_tiles) * mtiles;
-  const __nv_bfloat16 *bsrc = MODE == 0 ? a.ws.xs : a.ws.hs;
-  const int bstride = MODE == 0 ? D : fmax;
 
-  PfCursor cons, craw, cb;
-  cons.tile = blockIdx.x;
-  pf_seek<MODE>(a, mtiles, total, cons);
-  if (!cons.valid) return;  // no tile for this CTA (uniform)
-  craw = cons;
-  cb = cons;
+  PfCursor first;
+  first.tile = blockIdx.x;
+  pf_seek<MODE>(a, mtiles, total, first);
+  if (!first.valid) return;  // no tile for this CTA (uniform)
 
   if (tid == 0) {
-    for (int s = 0; s < kRawSlots; ++s) mbar_init(&raw_full[s], 1);
-    for (int s = 0; s < kBSlots; ++s) mbar_init(&mma_done[s], 1);
-    mbar_init(acc_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&a_ready[s], kDeqThreads);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < NACC; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    *abort_flag = 0;
     fence_barrier_init();
   }
   if (FMT == MOE_FMT_CB35_32)
@@ -457,183 +484,162 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(PrefillArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint64_t lim = a.spin_limit;
 
-  // ---- producers
-  auto issue_raw = [&](const PfCursor &c, uint32_t j) {  // thread 0
-    const int slot = j % kRawSlots;
-    unsigned char *raw = smem + PL::kRawOff + slot * PL::kRawSlot;
-    const ExpertGroup &G = c.shared ? a.L.shared : a.L.routed;
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&raw_full[slot], PL::kRaw);
-    const int64_t slot0 = (static_cast<int64_t>(c.pt.mt) * c.nc + c.s) * kTileRows;
+  if (warp == kWarpProd) {
+    // ---------------- producer
+    if (lane == 0) {
+      const CUtensorMap *bmap = MODE == 0 ? &a.ws.tmap_xs : &a.ws.tmap_hs;
+      uint32_t it = 0;
+      bool ok = true;
+      for (PfCursor c = first; c.valid && ok; pf_advance<MODE>(a, mtiles, total, c)) {
+        const ExpertGroup &G = c.shared ? a.L.shared : a.L.routed;
+        for (int s = 0; s < c.nc && ok; ++s, ++it) {
+          const int st = it % NS;
+          if (it >= NS && !(ok = pf_wait(&empty[st], ((it / NS) - 1) & 1u, lim, abort_flag, a.err))) break;
+          unsigned char *sb = stages + st * PL::kStage;
+          unsigned char *raw = sb + NM * PL::kATile + PL::kBTile;
+          mbar_arrive_expect_tx(&full[st], PL::kRaw + PL::kBTile);
+          const int64_t slot0 = (static_cast<int64_t>(c.pt.mt) * c.nc + s) * kTileRows;
 #pragma unroll
-    for (int m = 0; m < NM; ++m) {
-      const int64_t mat = static_cast<int64_t>(c.eidx) * 3 + (MODE == 0 ? m : 2);
-      unsigned char *rm = raw + m * PL::kRawM;
-      bulk_g2s(rm, G.a + mat * G.a_mat + slot0 * 16, PL::kRawA, &raw_full[slot]);
-      bulk_g2s(rm + PL::kRawA, G.s + mat * G.s_mat + slot0, PL::kRawS, &raw_full[slot]);
-      if (FMT == MOE_FMT_CB35_32) bulk_g2s(rm + PL::kRawA + PL::kRawS, G.g + mat * G.g_mat + slot0, PL::kRawG, &raw_full[slot]);
-    }
-  };
-  auto issue_b = [&](const PfCursor &c, uint32_t j) {  // all threads
-    if (c.valid) {
-      unsigned char *bt = smem + PL::kBOff + (j % kBSlots) * PL::kBTile;
-      const int k0 = c.s * kChunk;
-#pragma unroll
-      for (int z = 0; z < kPfBN * 8 / kPfThreads; ++z) {
-        const int q = tid + kPfThreads * z, r = q >> 3, cc = q & 7;
-        cp_async16(bt + sw128_off(r, cc), bsrc + static_cast<int64_t>(c.pt.rows0 + r) * bstride + k0 + 8 * cc);
-      }
-    }
-    cp_async_commit();  // one group per step (empty past the end), so wait_group counts steps
-  };
-
-  uint32_t j_raw = 0, j_b = 0;  // next stream position of each producer
-  for (int i = 0; i < kRawAhead && craw.valid; ++i) {
-    if (tid == 0) issue_raw(craw, j_raw);
-    ++j_raw;
-    pf_next<MODE>(a, mtiles, total, craw);
-  }
-  for (int i = 0; i < kBAhead; ++i) {
-    issue_b(cb, j_b);
-    ++j_b;
-    pf_next<MODE>(a, mtiles, total, cb);
-  }
-
-  uint32_t j = 0, tiles_done = 0;
-  int64_t last_committed = -1;
-  bool failed = false;
-  while (cons.valid) {
-    // the MMA of step j-2 read A slot j % 2 and B slot (j + 2) % 4
-    if (j >= 2) {
-      const uint32_t jm = j - 2;
-      if (!mbar_wait_bounded(&mma_done[jm % kBSlots], (jm / kBSlots) & 1u, a.spin_limit)) {
-        flag_error(a.err, kErrTimeout);
-        mbar_wait_bounded(&mma_done[jm % kBSlots], (jm / kBSlots) & 1u, kDrainLimit);
-      }
-    }
-    if (craw.valid) {
-      if (tid == 0) issue_raw(craw, j_raw);
-      ++j_raw;
-      pf_next<MODE>(a, mtiles, total, craw);
-    }
-    issue_b(cb, j_b);
-    ++j_b;
-    pf_next<MODE>(a, mtiles, total, cb);
-    cp_async_wait<kBAhead>();  // this step's B tile has landed
-    const int rslot = j % kRawSlots;
-    const bool ok = mbar_wait_bounded(&raw_full[rslot], (j / kRawSlots) & 1u, a.spin_limit);
-    if (__syncthreads_or(!ok)) {
-      // give up: wait (bounded) for the bulk copies still in flight, then leave
-      if (tid == 0) flag_error(a.err, kErrTimeout);
-      for (uint32_t r = j; r < j_raw; ++r)
-        mbar_wait_bounded(&raw_full[r % kRawSlots], (r / kRawSlots) & 1u, kDrainLimit);
-      failed = true;
-      break;
-    }
-    // dequantise: thread -> (row r, block h) of each matrix; 32 weights -> 4 swizzled chunks
-    unsigned char *at0 = smem + PL::kAOff + (j % kASlots) * NM * PL::kATile;
-    {
-      const unsigned char *raw = smem + PL::kRawOff + rslot * PL::kRawSlot;
-      const int r = tid & 127, h = tid >> 7;
-#pragma unroll
-      for (int m = 0; m < NM; ++m) {
-        const unsigned char *rm = raw + m * PL::kRawM;
-        const uint4 A = reinterpret_cast<const uint4 *>(rm)[r];
-        const __half2 sc2 = reinterpret_cast<const __half2 *>(rm + PL::kRawA)[r];
-        const float sc = __half2float(h ? __high2half(sc2) : __low2half(sc2));
-        const uint32_t w0 = h ? A.z : A.x, w1 = h ? A.w : A.y;
-        uint32_t sgn = 0;
-        if (FMT == MOE_FMT_CB35_32) {
-          const uint2 G2 = reinterpret_cast<const uint2 *>(rm + PL::kRawA + PL::kRawS)[r];
-          sgn = h ? G2.y : G2.x;
+          for (int m = 0; m < NM; ++m) {
+            const int64_t mat = static_cast<int64_t>(c.eidx) * 3 + (MODE == 0 ? m : 2);
+            unsigned char *rm = raw + m * PL::kRawM;
+            bulk_g2s(rm, G.a + mat * G.a_mat + slot0 * 16, PL::kRawA, &full[st]);
+            bulk_g2s(rm + PL::kRawA, G.s + mat * G.s_mat + slot0, PL::kRawS, &full[st]);
+            if (FMT == MOE_FMT_CB35_32)
+              bulk_g2s(rm + PL::kRawA + PL::kRawS, G.g + mat * G.g_mat + slot0, PL::kRawG, &full[st]);
+          }
+          tma_load_2d(sb + NM * PL::kATile, bmap, s * kChunk, c.pt.rows0, &full[st]);
         }
-        unsigned char *at = at0 + m * PL::kATile;
+      }
+      // leave only once every copy this thread issued has landed
+      const uint32_t issued = it;
+      for (uint32_t k = (issued > NS ? issued - NS : 0); k < issued; ++k)
+        mbar_wait_bounded(&full[k % NS], (k / NS) & 1u, kDrainLimit);
+    }
+  } else if (warp >= kWarpDeq0 && warp < kWarpDeq0 + 8) {
+    // ---------------- dequantisation: thread -> (row r, block h) of each matrix
+    const int t = tid - 32 * kWarpDeq0, r = t & 127, h = t >> 7;
+    uint32_t it = 0;
+    bool ok = true;
+    for (PfCursor c = first; c.valid && ok; pf_advance<MODE>(a, mtiles, total, c)) {
+      for (int s = 0; s < c.nc; ++s, ++it) {
+        const int st = it % NS;
+        if (!(ok = pf_wait(&full[st], (it / NS) & 1u, lim, abort_flag, a.err))) break;
+        unsigned char *sb = stages + st * PL::kStage;
+        const unsigned char *raw = sb + NM * PL::kATile + PL::kBTile;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[8];
-          if (FMT == MOE_FMT_Q2_32) {
-            // float(2^23 + q) by exponent bias, minus 2^23: the code q exactly; then s (q - 1.5)
+        for (int m = 0; m < NM; ++m) {
+          const unsigned char *rm = raw + m * PL::kRawM;
+          const uint4 A = reinterpret_cast<const uint4 *>(rm)[r];
+          const __half2 sc2 = reinterpret_cast<const __half2 *>(rm + PL::kRawA)[r];
+          const float sc = __half2float(h ? __high2half(sc2) : __low2half(sc2));
+          const uint32_t w0 = h ? A.z : A.x, w1 = h ? A.w : A.y;
+          uint32_t sgn = 0;
+          if (FMT == MOE_FMT_CB35_32) {
+            const uint2 G2 = reinterpret_cast<const uint2 *>(rm + PL::kRawA + PL::kRawS)[r];
+            sgn = h ? G2.y : G2.x;
+          }
+          unsigned char *at = sb + m * PL::kATile;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int p = 8 * cc + i;  // weight within the block
-              const uint32_t w = p < 16 ? w0 : w1;
-              const int pw = p & 15, kk = pw >> 2, jj = pw & 3;
-              const float q = __uint_as_float(((w >> (8 * jj + 2 * kk)) & 3u) | 0x4B000000u) - 8388608.0f;
-              v[i] = fmaf(sc, q, -1.5f * sc);
-            }
-          } else {
-            // two groups of 4: signed grid bytes (sign mask applied per byte), then s * value
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[8];
+            if (FMT == MOE_FMT_Q2_32) {
+              // float(2^23 + q) by exponent bias, minus 2^23: the code q exactly; then s (q - 1.5)
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-              const int g = 2 * cc + gg;
-              const uint32_t iw = g < 4 ? w0 : w1;
-              const uint32_t idx = (iw >> (8 * (g & 3))) & 0xFFu;
-              const uint32_t gw = reinterpret_cast<const uint32_t *>(grid_s)[idx];
-              const uint32_t mk = prmt_sign_bytes(sgn << (7 - g));
-              const uint32_t sb = ((gw ^ mk) + (mk & 0x01010101u)) ^ 0x80808080u;  // signed -> biased bytes
+              for (int i = 0; i < 8; ++i) {
+                const int p = 8 * cc + i;
+                const uint32_t w = p < 16 ? w0 : w1;
+                const int pw = p & 15, kk = pw >> 2, jj = pw & 3;
+                const float q = __uint_as_float(((w >> (8 * jj + 2 * kk)) & 3u) | 0x4B000000u) - 8388608.0f;
+                v[i] = fmaf(sc, q, -1.5f * sc);
+              }
+            } else {
 #pragma unroll
-              for (int jj = 0; jj < 4; ++jj) {
-                const float q = __uint_as_float(((sb >> (8 * jj)) & 0xFFu) | 0x4B000000u) - 8388736.0f;  // 2^23 + 128
-                v[4 * gg + jj] = sc * q;
+              for (int gg = 0; gg < 2; ++gg) {
+                const int g = 2 * cc + gg;
+                const uint32_t iw = g < 4 ? w0 : w1;
+                const uint32_t idx = (iw >> (8 * (g & 3))) & 0xFFu;
+                const uint32_t gw = reinterpret_cast<const uint32_t *>(grid_s)[idx];
+                const uint32_t mk = prmt_sign_bytes(sgn << (7 - g));
+                const uint32_t sbv = ((gw ^ mk) + (mk & 0x01010101u)) ^ 0x80808080u;  // signed -> biased bytes
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                  v[4 * gg + jj] = sc * (__uint_as_float(((sbv >> (8 * jj)) & 0xFFu) | 0x4B000000u) - 8388736.0f);
               }
             }
+            uint4 o;
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]), b3 = __floats2bfloat162_rn(v[6], v[7]);
+            o.x = *reinterpret_cast<uint32_t *>(&b0);
+            o.y = *reinterpret_cast<uint32_t *>(&b1);
+            o.z = *reinterpret_cast<uint32_t *>(&b2);
+            o.w = *reinterpret_cast<uint32_t *>(&b3);
+            *reinterpret_cast<uint4 *>(at + sw128_off(r, 4 * h + cc)) = o;
           }
-          uint4 o;
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]), b3 = __floats2bfloat162_rn(v[6], v[7]);
-          o.x = *reinterpret_cast<uint32_t *>(&b0);
-          o.y = *reinterpret_cast<uint32_t *>(&b1);
-          o.z = *reinterpret_cast<uint32_t *>(&b2);
-          o.w = *reinterpret_cast<uint32_t *>(&b3);
-          *reinterpret_cast<uint4 *>(at + sw128_off(r, 4 * h + cc)) = o;
         }
+        fence_proxy_async_smem();  // make the generic-proxy stores visible to the tensor core
+        mbar_arrive(&a_ready[st]);
       }
     }
-    fence_proxy_async_smem();  // generic-proxy writes (dequant, cp.async) -> tensor core reads
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t bt = smem_u32(smem + PL::kBOff + (j % kBSlots) * PL::kBTile);
-      const uint32_t idesc = idesc_bf16((cons.pt.cnt + 15) & ~15);
+  } else if (warp == kWarpMma) {
+    // ---------------- MMA issue (one thread)
+    if (lane == 0) {
+      uint32_t it = 0, tl = 0;
+      bool ok = true;
+      for (PfCursor c = first; c.valid && ok; pf_advance<MODE>(a, mtiles, total, c), ++tl) {
+        const int b = tl % NACC;
+        if (tl >= NACC && !(ok = pf_wait(&acc_empty[b], ((tl / NACC) - 1) & 1u, lim, abort_flag, a.err))) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + b * (NM * kPfBN);
+        const uint32_t idesc = idesc_bf16((c.pt.cnt + 15) & ~15);
+        for (int s = 0; s < c.nc; ++s, ++it) {
+          const int st = it % NS;
+          if (!(ok = pf_wait(&full[st], (it / NS) & 1u, lim, abort_flag, a.err))) break;
+          if (!(ok = pf_wait(&a_ready[st], (it / NS) & 1u, lim, abort_flag, a.err))) break;
+          tc_fence_after();
+          unsigned char *sb = stages + st * PL::kStage;
+          const uint32_t bt = smem_u32(sb + NM * PL::kATile);
 #pragma unroll
-      for (int m = 0; m < NM; ++m) {
-        const uint32_t at = smem_u32(at0 + m * PL::kATile);
+          for (int m = 0; m < NM; ++m) {
+            const uint32_t at = smem_u32(sb + m * PL::kATile);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma(tmem + m * kPfBN, sw128_desc(at + 32 * kk), sw128_desc(bt + 32 * kk), idesc,
-                 (cons.s > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma(acc + m * kPfBN, sw128_desc(at + 32 * kk), sw128_desc(bt + 32 * kk), idesc,
+                     (s > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[st]);
+        }
+        if (ok) tc_commit(&acc_full[b]);
       }
-      tc_commit(&mma_done[j % kBSlots]);
+      // every committed MMA must be complete before the TMEM is released
+      if (it > 0) mbar_wait_bounded(&empty[(it - 1) % NS], ((it - 1) / NS) & 1u, kDrainLimit);
     }
-    last_committed = j;
-    if (cons.s == cons.nc - 1) {
-      // epilogue of the tile
-      if (tid == 0) tc_commit(acc_full);
-      if (!mbar_wait_bounded(acc_full, tiles_done & 1u, a.spin_limit)) {
-        flag_error(a.err, kErrTimeout);
-        mbar_wait_bounded(acc_full, tiles_done & 1u, kDrainLimit);
-      }
-      ++tiles_done;
+  } else if (warp < kWarpEpi0 + 4) {
+    // ---------------- epilogue: warp q reads TMEM lanes 32q .. 32q+31 (= rows of the tile)
+    const int q = warp - kWarpEpi0;
+    uint32_t tl = 0;
+    bool ok = true;
+    for (PfCursor c = first; c.valid && ok; pf_advance<MODE>(a, mtiles, total, c), ++tl) {
+      const int b = tl % NACC;
+      if (!(ok = pf_wait(&acc_full[b], (tl / NACC) & 1u, lim, abort_flag, a.err))) break;
       tc_fence_after();
-      const PfTile &pt = cons.pt;
-      const int q = warp & 3;  // TMEM lane quarter of this warp
+      const PfTile &pt = c.pt;
       const int row = pt.mt * kTileRows + 32 * q + lane;
-      const int c_begin = (warp >> 2) * (kPfBN / 2), c_end = c_begin + kPfBN / 2;
-      for (int c0 = c_begin; c0 < c_end; c0 += 16) {
-        if (c0 >= pt.cnt) break;
-        const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + c0;
+      const uint32_t acc = tmem + b * (NM * kPfBN) + (static_cast<uint32_t>(32 * q) << 16);
+      for (int c0 = 0; c0 < pt.cnt; c0 += 16) {
         float g[16];
-        tmem_ld16(ta, g);
+        tmem_ld16(acc + c0, g);
         if (MODE == 0) {
           float u[16];
-          tmem_ld16(ta + kPfBN, u);
+          tmem_ld16(acc + kPfBN + c0, u);
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             if (c0 + i < pt.cnt)
               a.ws.hs[static_cast<int64_t>(pt.rows0 + c0 + i) * fmax + row] = __float2bfloat16_rn(silu_f(g[i]) * u[i]);
         } else {
-          float wr[16];  // routing weights of the 16 rows, loaded together
+          float wr[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) wr[i] = c0 + i < pt.cnt ? __ldcg(a.ws.row_w + pt.rows0 + c0 + i) : 0.f;
 #pragma unroll
@@ -643,17 +649,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(PrefillArgs a) {
         }
       }
       tc_fence_before();
-      __syncthreads();
+      mbar_arrive(&acc_empty[b]);
     }
-    ++j;
-    pf_next<MODE>(a, mtiles, total, cons);
   }
-  (void)failed;
-  // drain: every committed MMA must be complete before the TMEM is released
-  if (last_committed >= 0)
-    mbar_wait_bounded(&mma_done[last_committed % kBSlots], static_cast<uint32_t>(last_committed / kBSlots) & 1u,
-                      kDrainLimit);
-  cp_async_wait<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, PL::kTmemCols);
@@ -720,6 +718,37 @@ static inline void pf_rec(const PrefillArgs &a, int kind, int end, cudaStream_t 
     cudaEventRecordWithFlags(a.ev[2 * kind + end], st, cudaEventRecordExternal);
   else
     cudaEventRecord(a.ev[2 * kind + end], st);
+}
+
+// 2-D tensor map over a bf16 [rows][cols] row-major buffer: boxes of 64 columns x kPfBN rows with
+// the 128-byte swizzle (the UMMA K-major layout); rows past the end read as zeros.
+static cudaError_t make_tmap(CUtensorMap *map, void *base, uint64_t cols, uint64_t rows) {
+  using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    encode = reinterpret_cast<EncodeFn>(fn);
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(kPfBN)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_prefill_tensor_maps(PrefillWs &w, int d_model) {
+  cudaError_t e = make_tmap(&w.tmap_xs, w.xs, static_cast<uint64_t>(d_model), static_cast<uint64_t>(w.rows_max));
+  if (e == cudaSuccess) e = make_tmap(&w.tmap_hs, w.hs, static_cast<uint64_t>(w.fmax), static_cast<uint64_t>(w.rows_max));
+  return e;
 }
 
 cudaError_t launch_prefill_layer(const PrefillArgs &a, cudaStream_t st) {

@@ -3,6 +3,8 @@
 // at a time on the matrix units; Strata reads chunks of up to 8,192 tokens).
 #pragma once
 
+#include <cuda.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -14,6 +16,8 @@ constexpr int kPfBN = 256;  // tokens per GEMM tile (MMA N, at most)
 // ordered by group; within a group the order is the arrival order of the scatter, which does not
 // change any result (every output row is computed independently of the others).
 struct PrefillWs {
+  CUtensorMap tmap_xs;   // TMA view of xs: boxes of 64 columns x kPfBN rows, 128-byte swizzle
+  CUtensorMap tmap_hs;   // TMA view of hs
   int max_tokens;
   int rows_max;          // max_tokens * (k + n_shared)
   float *logits;         // [n][E]
@@ -56,6 +60,7 @@ struct PrefillArgs {
 };
 
 void plan_prefill_workspace(PrefillWs &w, const moe_config &g, char *base, uint64_t &off);
+cudaError_t make_prefill_tensor_maps(PrefillWs &w, int d_model);
 cudaError_t configure_prefill_kernels();
 cudaError_t launch_prefill_layer(const PrefillArgs &a, cudaStream_t st);
 
