@@ -300,7 +300,7 @@ def bench_verify(args, rank, world, local):
         moe.forward_stack(0, L, x_in, out)
     stream.synchronize()
     kern = {}
-    for kind, name in ((P.PROF_ROUTE, "k_route"), (P.PROF_GATEUP, "k_gateup"), (P.PROF_DOWN, "k_down+k_combine")):
+    for kind, name in ((P.PROF_ROUTE, "k_route"), (P.PROF_GATEUP, "k_gemv<gate/up>"), (P.PROF_DOWN, "k_gemv<down>+combine")):
         _, tot, cnt = P.moe_profile_read(moe.h, kind)
         kern[name] = (tot, cnt)
     P.moe_profile_enable(moe.h, False)
@@ -329,7 +329,7 @@ def bench_verify(args, rank, world, local):
     hbm_peak = pk["hbm_gbs"]
     achieved = gateup_bytes_last / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
     src = source_hash("expert_ffn_gemv_b200/csrc/decode.cu", "expert_ffn_gemv_b200/csrc/moe_internal.cuh")
-    traffic = profiled_traffic("k_gateup", "verify", src)
+    traffic = profiled_traffic("k_gemv_gateup", "verify", src)
     res = {
         "metric": METRIC,
         "value": value,
@@ -349,20 +349,20 @@ def bench_verify(args, rank, world, local):
                    "resident_weight_gb": round(moe.device_bytes() / 1e9, 2),
                    "l2": "inputs larger than L2: each pass reads ~%.1f GB of distinct expert blocks"
                          % (step_bytes.mean() / 1e9),
-                   "parallelism": f"replicas x{world}", "cuda_graph": "one pass (48 x 4 kernels) per replay"},
+                   "parallelism": f"replicas x{world}", "cuda_graph": "one pass (48 x 3 kernels) per replay"},
         "hbm": {"active_expert_and_router_bytes_per_step": float(step_bytes.mean()),
                 "gbs": float(step_bytes.sum() / (ms_local / 1e3) / 1e9),
                 "frac_of_measured_peak": float(step_bytes.sum() / (ms_local / 1e3) / 1e9 / hbm_peak),
                 "mean_active_experts_per_layer": float(u_all.mean() + wl.n_shared)},
-        "roofline": {"kernel": "k_gateup", "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+        "roofline": {"kernel": "k_gemv<gate/up>", "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
                      "peak_kind": pk_kind, "unit": "GB/s",
                      "frac": achieved / hbm_peak if achieved else None, "traffic": traffic,
                      "algorithmic_bytes_per_launch": gateup_bytes_last / max(gu_cnt, 1),
                      "avg_launch_us": gu_ms / max(gu_cnt, 1) * 1e3},
         "kernels_eager_pass_us": {k: round(v[0] * 1e3, 2) for k, v in kern.items()},
-        "down_roofline": {"achieved": down_bytes_last / (kern["k_down+k_combine"][0] / 1e3) / 1e9
-                          if kern["k_down+k_combine"][0] else None, "unit": "GB/s"},
-        "gpu_launches": K * L * 4,
+        "down_roofline": {"achieved": down_bytes_last / (kern["k_gemv<down>+combine"][0] / 1e3) / 1e9
+                          if kern["k_gemv<down>+combine"][0] else None, "unit": "GB/s"},
+        "gpu_launches": K * L * 3,
         "clocks": clk.summary(),
         "load_seconds": round(load_s, 1),
     }
@@ -476,12 +476,12 @@ def bench_decode_layers(args, rank, world, local):
                            "l2": "16 distinct layers per step"},
                 "tokens_per_s_one_layer": K * nl / (ms / 1e3),
                 "us_per_layer": ms * 1e3 / (K * nl),
-                "roofline": {"kernel": "k_gateup", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                "roofline": {"kernel": "k_gemv<gate/up>", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
                              "peak_kind": kind,
                              "achieved": gu_bytes / (kms / 1e3) / 1e9 if kms else None,
                              "frac": gu_bytes / (kms / 1e3) / 1e9 / pk["hbm_gbs"] if kms else None,
                              "avg_launch_us": kms / max(kcnt, 1) * 1e3},
-                "hbm_frac_whole_layer": gbs / pk["hbm_gbs"], "clocks": clocks, "gpu_launches": K * nl * 4})
+                "hbm_frac_whole_layer": gbs / pk["hbm_gbs"], "clocks": clocks, "gpu_launches": K * nl * 3})
     moe.close()
     return res
 
@@ -523,8 +523,8 @@ def bench_codebook(args, rank, world, local):
     res = _base_result(wl, world, K, W, out[8]["ms_per_step"] * K, "tokens/s", out[8]["tokens_per_s"])
     res.update({"dtype": "cb35 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
                 "config": {"workload": wl.name, "layers": nl, "tokens": [1, 8], "chain": "independent layers"},
-                "by_tokens": out, "gpu_launches": K * nl * 4,
-                "roofline": {"kernel": "k_gateup", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                "by_tokens": out, "gpu_launches": K * nl * 3,
+                "roofline": {"kernel": "k_gemv<gate/up>", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
                              "peak_kind": kind, "achieved": out[8]["gateup_gbs"],
                              "frac": out[8]["gateup_gbs"] / pk["hbm_gbs"] if out[8]["gateup_gbs"] else None}})
     moe.close()

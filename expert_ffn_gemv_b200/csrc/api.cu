@@ -11,9 +11,6 @@
 
 using namespace moe;
 
-#ifndef MOE_GATEUP_CHUNKS
-#define MOE_GATEUP_CHUNKS 8  // 512 columns of d_model per gate/up CTA
-#endif
 
 struct moe_handle {
   moe_config cfg;
@@ -35,7 +32,6 @@ struct moe_handle {
   uint64_t spin_limit = 2000000000ull; // ~1 s
   uint64_t alloc_cap = 0;
   uint64_t allocated = 0;
-  int gu_splits = 1;
   std::string last_error;
   // per-kernel event timing: events [layer position][kind][start, end]
   bool prof_on = false;
@@ -120,27 +116,34 @@ void plan_workspace(moe_handle *h, Carve &c) {
   w.umax = umax;
   w.fmax = fmax;
   w.tmax = tmax;
-  w.splits = h->gu_splits;
+  // router: 256 (else 128) d_model columns per CTA; K segments of 4 (else 2) chunks
+  w.rk_cols = D % 256 == 0 ? 256 : 128;
+  const int ncd = D / kChunk;
+  w.gu_seg = ncd % 4 == 0 ? 4 : 2;
+  w.gu_nseg = ncd / w.gu_seg;
+  {
+    auto nseg = [](int f) { const int nc = f / kChunk; return nc / (nc % 4 == 0 ? 4 : 2); };
+    w.dn_nseg = nseg(g.d_ff);
+    if (g.n_shared && nseg(g.shared_d_ff) > w.dn_nseg) w.dn_nseg = nseg(g.shared_d_ff);
+  }
+  const int ks = D / w.rk_cols, ngrp = (E + 31) / 32, td = D / kTileRows;
+  w.logit_part = c.take<float>(static_cast<uint64_t>(ks) * kDecodeMaxTokens * E);
   w.logits = c.take<float>(static_cast<uint64_t>(kDecodeMaxTokens) * E);
   w.route_idx = c.take<int>(kDecodeMaxTokens * K);
   w.route_w = c.take<float>(kDecodeMaxTokens * K);
   w.slotpos = c.take<int>(kDecodeMaxTokens * K);
-  w.n_active = c.take<int>(1);
-  w.act_expert = c.take<int>(umax);
-  w.act_ntok = c.take<int>(umax);
-  w.act_tok = c.take<int>(static_cast<uint64_t>(umax) * kDecodeMaxTokens);
-  w.xq = c.take<int16_t>(static_cast<uint64_t>(kDecodeMaxTokens) * D);
-  w.xsum = c.take<int>(static_cast<uint64_t>(kDecodeMaxTokens) * (D / 32));
-  w.xfac = c.take<float>(static_cast<uint64_t>(kDecodeMaxTokens) * ((h->gu_splits + 3) & ~3));
+  w.task_tab = c.take<int>(4 + static_cast<uint64_t>(umax) * 16);
+  w.xrec = c.take<ActRec>(static_cast<uint64_t>(kDecodeMaxTokens) * ncd);
   const uint64_t hrows = static_cast<uint64_t>(umax) * kDecodeMaxTokens;
-  w.hfs = (tmax + 3) & ~3;
-  w.hq = c.take<int16_t>(hrows * fmax);
-  w.hsum = c.take<int>(hrows * (fmax / 32));
-  w.hfac = c.take<float>(hrows * w.hfs);
-  w.gu_part = c.take<float>(static_cast<uint64_t>(umax) * tmax * h->gu_splits * 2 * kDecodeMaxTokens * kTileRows);
+  w.hrec = c.take<ActRec>(hrows * (fmax / kChunk));
+  w.gu_part = c.take<float>(static_cast<uint64_t>(umax) * tmax * w.gu_nseg * 2 * kDecodeMaxTokens * kTileRows);
+  w.dn_part = c.take<float>(static_cast<uint64_t>(umax) * td * w.dn_nseg * kDecodeMaxTokens * kTileRows);
   w.o = c.take<float>(hrows * D);
   w.route_ticket = c.take<unsigned>(1);
+  w.group_ticket = c.take<unsigned>(ngrp);
   w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax);
+  w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td);
+  w.counters = c.take<unsigned>(2);
   const uint64_t nt = static_cast<uint64_t>(g.max_tokens) * D;
   h->res[0] = c.take<float>(nt);
   h->res[1] = c.take<float>(nt);
@@ -155,8 +158,13 @@ moe_status check_device_error(moe_handle *h, cudaStream_t st) {
   if (!e) return MOE_OK;
   __atomic_store_n(h->err_host, 0u, __ATOMIC_RELEASE);
   // a kernel that gave up may have left arrival counters set: clear them
-  cudaMemsetAsync(h->dws.route_ticket, 0, sizeof(unsigned), st);
-  cudaMemsetAsync(h->dws.gu_ticket, 0, sizeof(unsigned) * h->dws.umax * h->dws.tmax, st);
+  const DecodeWs &w = h->dws;
+  const int td = h->cfg.d_model / kTileRows;
+  cudaMemsetAsync(w.route_ticket, 0, sizeof(unsigned), st);
+  cudaMemsetAsync(w.group_ticket, 0, sizeof(unsigned) * ((h->cfg.n_experts + 31) / 32), st);
+  cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax, st);
+  cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td, st);
+  cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * 2, st);
   if (e & kErrTimeout) return fail(h, MOE_ERR_TIMEOUT, "a device-side bounded wait ran out");
   return fail(h, MOE_ERR_DEVICE_FAULT, "a device-side check found an invalid routing index");
 }
@@ -295,11 +303,6 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
   h->sh.n_shared = g.n_shared;
   h->sh.fmt = g.fmt;
   h->sh.router_bf16 = g.router_dtype == MOE_BF16;
-  {
-    const int nc = g.d_model / kChunk;
-    const int cpc = MOE_GATEUP_CHUNKS;  // chunks of 64 columns per gate/up CTA
-    h->gu_splits = nc >= 2 * cpc && nc % cpc == 0 ? nc / cpc : 1;
-  }
   h->layers.assign(g.n_layers, LayerDev{});
   h->layer_mem.assign(g.n_layers, nullptr);
   h->layer_bytes.assign(g.n_layers, 0);
@@ -333,8 +336,7 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
         goto fail_out;
       }
     }
-    cudaError_t ge = decode_grid_sizes(g.fmt, g.d_model, h->gu_splits, h->dws.fmax, h->dws.umax, g.n_shared, g.d_ff,
-                                       g.shared_d_ff, &h->dws.grid_gu, &h->dws.grid_down);
+    cudaError_t ge = decode_grid_sizes(g.fmt, h->dws.umax, &h->dws.grid_gu, &h->dws.grid_dn, &h->dws.min_streams);
     if (ge != cudaSuccess) {
       s = cuda_fail(h, ge, "grid sizing");
       goto fail_out;
@@ -397,6 +399,7 @@ moe_status moe_profile_enable(moe_handle *h, int32_t on) {
   }
   h->prof_on = on != 0;
   h->prof_mask = static_cast<uint32_t>(on) & ((1u << kProfKinds) - 1);
+  prof_reset_used(h);
   return MOE_OK;
 }
 
@@ -583,8 +586,8 @@ moe_status moe_forward(moe_handle *h, int32_t layer, const void *x, void *y, int
     xd = h->x_stage;
   }
   if (yh) yd = h->y_stage;
-  prof_reset_used(h);
-  s = run_layer(h, layer, xd, g.act_dtype == MOE_BF16, yd, g.out_dtype == MOE_BF16, n_tokens, 0, nullptr, route, st);
+  s = run_layer(h, layer, xd, g.act_dtype == MOE_BF16, yd, g.out_dtype == MOE_BF16, n_tokens, 0, nullptr, route, st,
+                layer);
   if (s != MOE_OK) return s;
   if (yh) {
     cudaError_t e = cudaMemcpyAsync(y, h->y_stage, ybytes, cudaMemcpyDeviceToHost, st);
@@ -627,14 +630,13 @@ moe_status moe_forward_stack(moe_handle *h, int32_t first_layer, int32_t n_layer
     if (e != cudaSuccess) return cuda_fail(h, e, "trace copy");
   }
   int pp = 0;
-  prof_reset_used(h);
   for (int i = 0; i < n_layers; ++i) {
     const bool last = i == n_layers - 1;
     void *out = last ? (yh ? h->y_stage : x_out) : static_cast<void *>(h->res[pp]);
     const int out_bf16 = last ? g.out_dtype == MOE_BF16 : 0;
     float *copy = (x_trace && !last) ? x_trace + static_cast<uint64_t>(i + 1) * nd : nullptr;
     s = run_layer(h, first_layer + i, cur, cur_bf16, out, out_bf16, n_tokens, 1, copy,
-                  per_layer_route ? per_layer_route + i : nullptr, st, i);
+                  per_layer_route ? per_layer_route + i : nullptr, st, first_layer + i);
     if (s != MOE_OK) return s;
     cur = out;
     cur_bf16 = 0;

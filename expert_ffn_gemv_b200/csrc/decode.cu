@@ -1,23 +1,31 @@
 // decode.cu -- the dequant-fused GEMV path for 1..8 tokens (decode steps and 1 + 7 token
 // verify batches of the routed-MoE pages: strata-mlx README, "Draft and verify").
 //
-// Four kernels per layer, all on CUDA cores:
-//   k_route   router GEMV (fp32 accumulate) over all experts; meanwhile the first CTAs quantise
-//             the layer input (int16 + one power-of-two factor per token and K-split).  The last
-//             CTA to finish takes the top-k, the fp32 softmax over the selected logits and builds
-//             the active-expert tables (which experts run, which tokens each one serves).
-//   k_gateup  per (active expert, 128-row tile, K-split): the gate and up rows of the tile and
-//             the quantised inputs of the expert's tokens are bulk-copied (cp.async.bulk) into
-//             shared memory, the weights straight from their low-bit planes; thread r owns gate
-//             row r and up row r.  Codes are unpacked with two ALU ops per four weights and
-//             multiplied with the activations by dp2a (int16 x int8 -> int32); the exact integer
-//             block sums are scaled by the fp16 block scale into fp32 accumulators.  The K-split
-//             partials are reduced in a fixed order by the last CTA of the tile, which applies
-//             SwiGLU and quantises h per (token, tile).
-//   k_down    per (active expert, 128 rows of d_model): the same GEMV over h -> o rows.
-//   k_combine y = sum_j w_j o_j + o_shared (+ x for stacks), slots in a fixed order.
-// No fp32 atomics: results are bit-reproducible and independent of which tokens share a call.
+// Three kernels per layer, all on CUDA cores:
+//   k_route   router GEMV over all experts: lane = expert, the tokens' activations broadcast
+//             from shared memory, fp32 accumulation; each CTA takes 32 experts x one K slice,
+//             the last CTA of a 32-expert group adds the slices in slice order.  The CTAs of
+//             group 0 also quantise the layer input into activation records (int16 + block
+//             sums + a power-of-two factor per 128 columns).  The last group to finish takes
+//             the top-k (warp per token, argmax by warp reductions over order-preserving keys),
+//             the fp32 softmax over the selected logits and builds the active-expert tables.
+//   k_gateup  persistent.  A producer warp takes pieces (active expert, 128-row tile, run of K
+//             segments) from a work queue and bulk-copies (cp.async.bulk) the gate and up rows
+//             of the piece straight from their low-bit planes, with the activation records of
+//             the expert's tokens, into a ring of shared-memory stages; four consumer warps
+//             (thread = row) unpack the codes with two ALU ops per four weights and multiply
+//             them with the int16 activations by dp2a (int16 x int8 -> int32).  The exact
+//             integer block sums are scaled by the fp16 block scale into fp32 sums, one per K
+//             segment; the segment sums are added in segment order.  The unit's last piece
+//             applies SwiGLU and quantises h per (token, 128-row tile) into records.
+//   k_down    the same over h -> o rows; the last expert to finish a 128-column tile of the
+//             output sums y = sum_j w_j o_j + o_shared (+ x) over it, slots in a fixed order.
+// No fp32 atomics, and the K segments are fixed by the matrix shapes: results are
+// bit-reproducible and independent of which tokens share a call and of how the work queue
+// split the units among CTAs.
 #include <float.h>
+#include <stdlib.h>
+#include <limits.h>
 
 #include "moe_internal.cuh"
 
@@ -25,24 +33,30 @@ namespace moe {
 
 constexpr int kRouteWarps = 8;
 constexpr int kRouteThreads = 32 * kRouteWarps;
-constexpr int kMaxSplits = 16;
-// Ring depth of the GEMV kernels.  With one stage the grid holds one CTA per possible task, so
-// that several CTAs per SM overlap one another's copies and compute; with two, a persistent grid
-// of (SMs x resident CTAs) walks the tasks with the next task's copies in flight.
-#ifndef MOE_DECODE_STAGES
-#define MOE_DECODE_STAGES 1
-#endif
+constexpr int kRouteExperts = 32;               // experts per router CTA: lane = expert
+constexpr int kRouteMaxCols = 256;              // d_model columns per router CTA (at most)
+constexpr int kQGroup = 128;                    // columns sharing one activation factor
+constexpr int kConsWarps = kTileRows / 32;      // consumer warps: thread = row of the tile
+constexpr int kGemvThreads = kTileRows + 32;    // + one producer warp
+constexpr int kRing = 4;                        // most stages of the bulk-copy ring
 #ifndef MOE_GEMV_MIN_BLOCKS
-#define MOE_GEMV_MIN_BLOCKS 4
+#define MOE_GEMV_MIN_BLOCKS 3                   // resident CTAs per SM the register budget allows
 #endif
-constexpr int kDecodeStages = MOE_DECODE_STAGES;
+#ifndef MOE_GEMV_UNROLL
+#define MOE_GEMV_UNROLL 1                       // chunks of a stage in flight per iteration
+#endif
+constexpr int kGemvUnroll = MOE_GEMV_UNROLL;
+// ring depth: 4 stages for Q2; 3 for CB35, whose stages and grid table are larger, so that two
+// CTAs fit on an SM
+__host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_CB35_32 ? 3 : 4; }
+constexpr int kGuStageChunks = 2;               // gate/up: chunks per stage
+constexpr int kDnStageChunks = 4;               // down: chunks per stage (one K segment)
+constexpr int kPartStride = kDecodeMaxTokens * kTileRows;  // floats per (segment, matrix)
 
 __device__ __forceinline__ float load_act(const void *x, int64_t i, int bf16) {
   if (bf16) return __bfloat162float(static_cast<const __nv_bfloat16 *>(x)[i]);
   return static_cast<const float *>(x)[i];
 }
-
-__host__ __device__ inline int pad4(int v) { return (v + 3) & ~3; }
 
 // power of two 2^e as a float, e in [-126, 127]
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
@@ -66,7 +80,7 @@ __device__ __forceinline__ int fix16(float v, float sc) {
 template <bool RBF16>
 __device__ __forceinline__ void load_row8(const void *w, int64_t off, float (&v)[8]) {
   if (RBF16) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(w) + off));
+    const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(w) + off));
     const uint32_t p[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -75,248 +89,309 @@ __device__ __forceinline__ void load_row8(const void *w, int64_t off, float (&v)
     }
   } else {
     const float4 *f = reinterpret_cast<const float4 *>(static_cast<const float *>(w) + off);
-    const float4 a = __ldg(f), b = __ldg(f + 1);
+    const float4 a = __ldcs(f), b = __ldcs(f + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
 }
 
-// Copy n x D activations (bf16 or fp32) into shared memory as fp32: 16-byte loads, 8 in flight
-// per thread.
-__device__ __forceinline__ void stage_acts_f32(const void *x, int bf16, int count, float *dst) {
-  if (bf16) {
-    const uint4 *src = static_cast<const uint4 *>(x);
-    const int nv = count / 8;
-    for (int v0 = threadIdx.x; v0 < nv; v0 += 8 * blockDim.x) {
-      uint4 q[8];
+// Order-preserving unsigned key of a float (larger float -> larger key); NaN maps to 0, the
+// key that never wins, and 0 also marks an expert already taken.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 0u;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// fp32 softmax over the K selected logits (lane j holds the j-th), results to the tables
+__device__ __forceinline__ void softmax_store(const DecodeArgs &a, int t, int lane, float my_l, float l0, int my_i) {
+  const int K = a.sh.k;
+  float w = lane < K ? __expf(my_l - l0) : 0.f;
+  float sum = w;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int v = v0 + i * blockDim.x;
-        if (v < nv) q[i] = __ldg(src + v);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int v = v0 + i * blockDim.x;
-        if (v < nv) {
-          const uint32_t p[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
-          float4 lo, hi;
-          lo.x = __uint_as_float(p[0] << 16); lo.y = __uint_as_float(p[0] & 0xFFFF0000u);
-          lo.z = __uint_as_float(p[1] << 16); lo.w = __uint_as_float(p[1] & 0xFFFF0000u);
-          hi.x = __uint_as_float(p[2] << 16); hi.y = __uint_as_float(p[2] & 0xFFFF0000u);
-          hi.z = __uint_as_float(p[3] << 16); hi.w = __uint_as_float(p[3] & 0xFFFF0000u);
-          reinterpret_cast<float4 *>(dst)[2 * v] = lo;
-          reinterpret_cast<float4 *>(dst)[2 * v + 1] = hi;
-        }
-      }
-    }
-  } else {
-    const float4 *src = static_cast<const float4 *>(x);
-    const int nv = count / 4;
-    for (int v0 = threadIdx.x; v0 < nv; v0 += 8 * blockDim.x) {
-      float4 q[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int v = v0 + i * blockDim.x;
-        if (v < nv) q[i] = __ldg(src + v);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int v = v0 + i * blockDim.x;
-        if (v < nv) reinterpret_cast<float4 *>(dst)[v] = q[i];
-      }
-    }
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < K) {
+    w = w / sum;
+    a.ws.route_idx[t * K + lane] = my_i;
+    a.ws.route_w[t * K + lane] = w;
+    if (a.out_idx) a.out_idx[t * K + lane] = my_i;
+    if (a.out_w) a.out_w[t * K + lane] = w;
   }
 }
 
-// CTA-wide max over the 256 threads (all threads get it)
-__device__ __forceinline__ float block_max_256(float v, float *red) {
+// Top-k of token t by one warp, logits in registers (lane l holds experts l + 32 q).  Each
+// round takes the largest key by a warp max-reduction and, among the lanes holding it, the
+// lowest expert index by a min-reduction: the order of repeated strict maxima, ties to the
+// lower index.
+template <int VPL>
+__device__ __forceinline__ void topk_regs(const DecodeArgs &a, int t, int lane, int *s_idx) {
+  const int E = a.sh.e, K = a.sh.k;
+  uint32_t key[VPL];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float m = red[0];
+  for (int q = 0; q < VPL; ++q) {
+    const int i = lane + 32 * q;
+    key[q] = i < E ? order_key(__ldcg(a.ws.logits + t * E + i)) : 0u;
+  }
+  float my_l = 0.f, l0 = 0.f;
+  int my_i = 0;
+  for (int j = 0; j < K; ++j) {
+    uint32_t lb = key[0];
 #pragma unroll
-  for (int w = 1; w < kRouteWarps; ++w) m = fmaxf(m, red[w]);
-  __syncthreads();
-  return m;
+    for (int q = 1; q < VPL; ++q) lb = max(lb, key[q]);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, lb);
+    int qm = 0;
+#pragma unroll
+    for (int q = VPL - 1; q >= 0; --q)
+      if (key[q] == m) qm = q;
+    int bi = __reduce_min_sync(0xffffffffu, lb == m ? lane + 32 * qm : INT_MAX);
+    float bv = key_value(m);
+    if (bi >= E || !(bv > -INFINITY)) {  // only non-finite logits left
+      if (lane == 0) flag_error(a.err, kErrBadIndex);
+      bi = j;
+      bv = 0.f;
+    }
+    // clear the winner by selects on every register (a conditional store with a data-dependent
+    // index would move key[] to local memory)
+    const int qb = (bi & 31) == lane ? bi >> 5 : -1;
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) key[q] = q == qb ? 0u : key[q];
+    if (j == 0) l0 = bv;
+    if (lane == j) { my_l = bv; my_i = bi; }
+    if (lane == 0) s_idx[t * K + j] = bi;
+  }
+  softmax_store(a, t, lane, my_l, l0, my_i);
 }
+
+// Top-k of token t by one warp over logits in shared memory (more than 1,024 experts).
+__device__ __forceinline__ void topk_smem(const DecodeArgs &a, int t, int lane, float *row, int *s_idx) {
+  const int E = a.sh.e, K = a.sh.k;
+  for (int i = lane; i < E; i += 32) row[i] = __ldcg(a.ws.logits + t * E + i);
+  __syncwarp();
+  float my_l = 0.f, l0 = 0.f;
+  int my_i = 0;
+  for (int j = 0; j < K; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int i = lane; i < E; i += 32) {
+      const float v = row[i];
+      if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if (bi >= E) {
+      if (lane == 0) flag_error(a.err, kErrBadIndex);
+      bi = j;
+    }
+    if (j == 0) l0 = bv;
+    if (lane == j) { my_l = bv; my_i = bi; }
+    if (lane == 0) { row[bi] = -INFINITY; s_idx[t * K + j] = bi; }
+    __syncwarp();
+  }
+  softmax_store(a, t, lane, my_l, l0, my_i);
+}
+
+// Pieces per unit: about min_streams pieces in flight over the call; units with four or more
+// tokens (several times the arithmetic per byte) are split up to eight ways.  Returns the run
+// length in segments.
+__device__ __forceinline__ int piece_run(int nseg, int units_total, int ntok, int min_streams) {
+  int p = (min_streams + units_total - 1) / units_total;
+  if (ntok >= 4) p = max(p, 8);
+  p = min(max(p, 1), nseg);
+  return (nseg + p - 1) / p;
+}
+
+// Split of one GEMV unit whose K has nc chunks: K segments of 4 (else 2) chunks, cut into
+// pieces of `len` segments.  Returns the packed split; `pieces` the number of pieces.
+__device__ __forceinline__ int unit_split(int nc, int units_total, int ntok, int min_streams, int &pieces) {
+  const int seg = nc % 4 == 0 ? 4 : 2;
+  const int nseg = nc / seg;
+  const int len = piece_run(nseg, units_total, ntok, min_streams);
+  pieces = (nseg + len - 1) / len;
+  return len | (pieces << 8) | (seg << 16) | (nseg << 20);
+}
+
+constexpr int kTabHead = 4;    // ints before the first row of the task table
+constexpr int kTabInts = 16;   // ints per active expert
+constexpr int kMaxActive = kDecodeMaxTokens * kMaxTopK + 1;
 
 template <bool RBF16>
 __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int D = a.sh.d, E = a.sh.e, K = a.sh.k, n = a.n;
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ __align__(16) float xs[kDecodeMaxTokens][kRouteMaxCols];
+  __shared__ float red[kRouteWarps][kDecodeMaxTokens][32];
+  __shared__ int s_idx[kDecodeMaxTokens * kMaxTopK];
+  __shared__ int s_wsum[kRouteWarps];
+  __shared__ int s_cnt[2][kMaxActive];
+  __shared__ int s_last;
+  const int D = a.sh.d, E = a.sh.e, n = a.n;
+  const int CK = a.ws.rk_cols, KS = D / CK;
+  const int grp = blockIdx.x / KS, ks = blockIdx.x - grp * KS, ngrp = gridDim.x / KS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ float red[kRouteWarps];
-  float *xs = reinterpret_cast<float *>(smem);  // [n][D]
-  stage_acts_f32(a.x, a.x_bf16, n * D, xs);
+  const int c0 = ks * CK;
+  // this CTA's router weights (written by no kernel) load while the previous kernel finishes
+  const int re0 = grp * kRouteExperts + lane;  // lane = expert
+  const int cw = CK / kRouteWarps, cb = warp * cw;  // warp = CK/8 columns of the slice
+  float w[4][8];
+  if (re0 < E) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (8 * i < cw) load_row8<RBF16>(a.L.router_w, static_cast<int64_t>(re0) * D + c0 + cb + 8 * i, w[i]);
+  }
+  griddep_wait();
+  griddep_launch();
+  // the work queues of this layer's GEMV kernels start empty (the previous layer is done)
+  if (blockIdx.x == 0 && tid == 0) {
+    a.ws.counters[0] = 0u;
+    a.ws.counters[1] = 0u;
+  }
+
+  // ---- the K slice of the n tokens, as fp32
+  if (a.x_bf16) {
+    const int per = CK / 8;
+    for (int v = tid; v < n * per; v += kRouteThreads) {
+      const int t = v / per, j = v - t * per;
+      const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) +
+                                                            static_cast<int64_t>(t) * D + c0) + j);
+      float4 lo, hi;
+      lo.x = __uint_as_float(q.x << 16); lo.y = __uint_as_float(q.x & 0xFFFF0000u);
+      lo.z = __uint_as_float(q.y << 16); lo.w = __uint_as_float(q.y & 0xFFFF0000u);
+      hi.x = __uint_as_float(q.z << 16); hi.y = __uint_as_float(q.z & 0xFFFF0000u);
+      hi.z = __uint_as_float(q.w << 16); hi.w = __uint_as_float(q.w & 0xFFFF0000u);
+      *reinterpret_cast<float4 *>(&xs[t][8 * j]) = lo;
+      *reinterpret_cast<float4 *>(&xs[t][8 * j + 4]) = hi;
+    }
+  } else {
+    const int per = CK / 4;
+    for (int v = tid; v < n * per; v += kRouteThreads) {
+      const int t = v / per, j = v - t * per;
+      *reinterpret_cast<float4 *>(&xs[t][4 * j]) =
+          __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + static_cast<int64_t>(t) * D + c0) + j);
+    }
+  }
   __syncthreads();
 
-  // ---- input quantisation: CTA p < n * splits takes token p / splits, K-split p % splits
-  {
-    const int S = a.ws.splits, ncols = D / S;
-    const int p = blockIdx.x;
-    if (p < n * S) {
-      const int t = p / S, s = p % S;
-      const float *src = xs + t * D + s * ncols;
-      float mx = 0.f;
-      for (int c = tid; c < ncols; c += kRouteThreads) mx = fmaxf(mx, fabsf(src[c]));
-      mx = block_max_256(mx, red);
+  // ---- input quantisation (group 0): warp per (token, 128-column group), lane = 4 columns
+  if (grp == 0) {
+    const int qpt = CK / kQGroup;
+    for (int p = warp; p < n * qpt; p += kRouteWarps) {
+      const int t = p / qpt, qg = p - t * qpt;
+      const float4 v = *reinterpret_cast<const float4 *>(&xs[t][qg * kQGroup + 4 * lane]);
+      float mx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const int e = fix16_exponent(mx);
       const float sc = pow2f(e);
-      for (int c = tid; c < ncols; c += kRouteThreads) {
-        const int m = fix16(src[c], sc);
-        a.ws.xq[t * D + s * ncols + c] = static_cast<int16_t>(m);
-        int sum = m;  // a warp covers one 32-column block of this pass
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) a.ws.xsum[t * (D / 32) + (s * ncols + c) / 32] = sum;
+      const int q0 = fix16(v.x, sc), q1 = fix16(v.y, sc), q2 = fix16(v.z, sc), q3 = fix16(v.w, sc);
+      ActRec *rec = a.ws.xrec + static_cast<int64_t>(t) * (D / kChunk) + (c0 + qg * kQGroup) / kChunk + (lane >> 4);
+      *reinterpret_cast<uint2 *>(&rec->x[(4 * lane) & 63]) =
+          make_uint2((static_cast<uint32_t>(q0) & 0xFFFFu) | (static_cast<uint32_t>(q1) << 16),
+                     (static_cast<uint32_t>(q2) & 0xFFFFu) | (static_cast<uint32_t>(q3) << 16));
+      int s = q0 + q1 + q2 + q3;  // eight lanes = one 32-column block
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if ((lane & 7) == 0) rec->m[(lane >> 3) & 1] = s;
+      if ((lane & 15) == 0) {
+        rec->f = pow2f(-e) * (a.sh.fmt == MOE_FMT_Q2_32 ? 0.5f : 1.0f);
+        rec->pad = 0u;
       }
-      if (tid == 0) a.ws.xfac[t * pad4(S) + s] = pow2f(-e) * (a.sh.fmt == MOE_FMT_Q2_32 ? 0.5f : 1.0f);
     }
   }
 
-  // ---- router GEMV: warp = expert, fp32 accumulation
-  const int e = blockIdx.x * kRouteWarps + warp;
-  if (e < E) {
+  // ---- router GEMV: lane = expert, warp = CK/8 columns of the slice
+  {
     float acc[kDecodeMaxTokens];
 #pragma unroll
     for (int t = 0; t < kDecodeMaxTokens; ++t) acc[t] = 0.f;
-    const int nch = D / 8;  // 8-element chunks of the row; lane takes c = lane + 32 i
-    for (int c0 = lane; c0 < nch; c0 += 4 * 32) {
-      float w[4][8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (c0 + 32 * i < nch) load_row8<RBF16>(a.L.router_w, static_cast<int64_t>(e) * D + 8 * (c0 + 32 * i), w[i]);
+    if (re0 < E) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int c = c0 + 32 * i;
-        if (c >= nch) break;
+        if (8 * i < cw) {
 #pragma unroll
-        for (int t = 0; t < kDecodeMaxTokens; ++t) {
-          if (t < n) {
-            const float4 x0 = *reinterpret_cast<const float4 *>(xs + t * D + 8 * c);
-            const float4 x1 = *reinterpret_cast<const float4 *>(xs + t * D + 8 * c + 4);
-            float v = acc[t];
-            v = fmaf(w[i][0], x0.x, v); v = fmaf(w[i][1], x0.y, v); v = fmaf(w[i][2], x0.z, v);
-            v = fmaf(w[i][3], x0.w, v); v = fmaf(w[i][4], x1.x, v); v = fmaf(w[i][5], x1.y, v);
-            v = fmaf(w[i][6], x1.z, v); v = fmaf(w[i][7], x1.w, v);
-            acc[t] = v;
+          for (int t = 0; t < kDecodeMaxTokens; ++t) {
+            if (t < n) {
+              const float4 x0 = *reinterpret_cast<const float4 *>(&xs[t][cb + 8 * i]);
+              const float4 x1 = *reinterpret_cast<const float4 *>(&xs[t][cb + 8 * i + 4]);
+              float v = acc[t];
+              v = fmaf(w[i][0], x0.x, v); v = fmaf(w[i][1], x0.y, v); v = fmaf(w[i][2], x0.z, v);
+              v = fmaf(w[i][3], x0.w, v); v = fmaf(w[i][4], x1.x, v); v = fmaf(w[i][5], x1.y, v);
+              v = fmaf(w[i][6], x1.z, v); v = fmaf(w[i][7], x1.w, v);
+              acc[t] = v;
+            }
           }
         }
       }
     }
-    const float bias = a.L.bias[e];
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxTokens; ++t) {
-      if (t < n) {
-        float v = acc[t];
+    for (int t = 0; t < kDecodeMaxTokens; ++t)
+      if (t < n) red[warp][t][lane] = acc[t];
+  }
+  __syncthreads();
+  const int rt = tid >> 5, re = grp * kRouteExperts + lane;  // thread = (token, expert of the group)
+  if (rt < n && re < E) {
+    float s = red[0][rt][lane];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) a.ws.logits[t * E + e] = v + bias;
-      }
-    }
+    for (int w = 1; w < kRouteWarps; ++w) s += red[w][rt][lane];
+    a.ws.logit_part[(static_cast<int64_t>(ks) * kDecodeMaxTokens + rt) * E + re] = s;
   }
 
-  // ---- the last CTA to finish continues with top-k and the routing tables
+  // ---- the last CTA of the group adds the K slices in slice order
   __threadfence();
   __syncthreads();
-  __shared__ int s_last;
-  if (tid == 0) s_last = atomicAdd(a.ws.route_ticket, 1u) == gridDim.x - 1;
+  if (tid == 0) s_last = atomicAdd(a.ws.group_ticket + grp, 1u) == static_cast<unsigned>(KS - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (rt < n && re < E) {
+    float pv[kDecodeMaxD / 128];
+#pragma unroll
+    for (int q = 0; q < kDecodeMaxD / 128; ++q)
+      if (q < KS) pv[q] = __ldcg(a.ws.logit_part + (static_cast<int64_t>(q) * kDecodeMaxTokens + rt) * E + re);
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < kDecodeMaxD / 128; ++q)
+      if (q < KS) s += pv[q];
+    a.ws.logits[rt * E + re] = s + a.L.bias[re];
+  }
+  if (tid == 0) a.ws.group_ticket[grp] = 0u;
+
+  // ---- the last group continues with top-k and the routing tables
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(a.ws.route_ticket, 1u) == static_cast<unsigned>(ngrp - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
 
-  int *mark = reinterpret_cast<int *>(smem);  // [E] (reuses the x area)
-  int *rank = mark + E;                        // [E]
-  float *lg = reinterpret_cast<float *>(rank + E);  // [n][E] (only for E > 1024)
-  __shared__ int s_idx[kDecodeMaxTokens * kMaxTopK];
-  __shared__ int s_wsum[kRouteWarps];
-  for (int i = tid; i < E; i += kRouteThreads) mark[i] = 0;
-
+  const int K = a.sh.k;
+  uint32_t *tokmask = reinterpret_cast<uint32_t *>(smem);  // [E]: bit t = token t chose the expert
+  int *rank = reinterpret_cast<int *>(tokmask + E);          // [E]
+  float *lg = reinterpret_cast<float *>(rank + E);           // [n][E] (more than 1,024 experts)
+  for (int i = tid; i < E; i += kRouteThreads) tokmask[i] = 0u;
   if (warp < n) {
-    const int t = warp;
-    float my_l = -FLT_MAX, l0 = 0.f;
-    int my_i = 0;
-    if (E <= 32 * 32) {
-      // logits of the token in registers: v[j] is expert lane + 32 j
-      float v[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int i = lane + 32 * j;
-        v[j] = i < E ? __ldcg(a.ws.logits + t * E + i) : -INFINITY;
-      }
-      for (int j = 0; j < K; ++j) {
-        float bv = v[0];
-        int bi = lane;
-#pragma unroll
-        for (int q = 1; q < 32; ++q)
-          if (v[q] > bv) { bv = v[q]; bi = lane + 32 * q; }  // strict: the lower index stays
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if (bi >= E || !(bv > -INFINITY)) {  // only non-finite logits left
-          if (lane == 0) flag_error(a.err, kErrBadIndex);
-          bi = j;
-        }
-#pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (bi == lane + 32 * q) v[q] = -INFINITY;
-        if (j == 0) l0 = bv;
-        if (lane == j) { my_l = bv; my_i = bi; }
-        if (lane == 0) s_idx[t * K + j] = bi;
-      }
-    } else {
-      float *row = lg + t * E;
-      for (int i = lane; i < E; i += 32) row[i] = __ldcg(a.ws.logits + t * E + i);
-      __syncwarp();
-      for (int j = 0; j < K; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int i = lane; i < E; i += 32) {
-          const float v = row[i];
-          if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if (bi >= E) {
-          if (lane == 0) flag_error(a.err, kErrBadIndex);
-          bi = j;
-        }
-        if (j == 0) l0 = bv;
-        if (lane == j) { my_l = bv; my_i = bi; }
-        if (lane == 0) { row[bi] = -INFINITY; s_idx[t * K + j] = bi; }
-        __syncwarp();
-      }
-    }
-    // fp32 softmax over the selected logits
-    float w = lane < K ? __expf(my_l - l0) : 0.f;
-    float sum = w;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane < K) {
-      w = w / sum;
-      a.ws.route_idx[t * K + lane] = my_i;
-      a.ws.route_w[t * K + lane] = w;
-      if (a.out_idx) a.out_idx[t * K + lane] = my_i;
-      if (a.out_w) a.out_w[t * K + lane] = w;
-    }
+    if (E <= 128) topk_regs<4>(a, warp, lane, s_idx);
+    else if (E <= 256) topk_regs<8>(a, warp, lane, s_idx);
+    else if (E <= 512) topk_regs<16>(a, warp, lane, s_idx);
+    else if (E <= 1024) topk_regs<32>(a, warp, lane, s_idx);
+    else topk_smem(a, warp, lane, lg + warp * E, s_idx);
   }
   __syncthreads();
-  for (int i = tid; i < n * K; i += kRouteThreads) mark[s_idx[i]] = 1;
+  for (int p = tid; p < n * K; p += kRouteThreads) atomicOr(tokmask + s_idx[p], 1u << (p / K));
   __syncthreads();
-  // block-wide exclusive scan of mark -> rank (ascending expert id)
+  // block-wide exclusive scan of (tokmask != 0) -> rank (ascending expert id)
   {
     const int per = (E + kRouteThreads - 1) / kRouteThreads;
     const int lo = tid * per, hi = min(E, lo + per);
     int local = 0;
-    for (int i = lo; i < hi; ++i) local += mark[i];
+    for (int i = lo; i < hi; ++i) local += tokmask[i] != 0u;
     int inc = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -328,53 +403,88 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
     int base = 0;
     for (int w = 0; w < warp; ++w) base += s_wsum[w];
     int run = base + inc - local;
-    for (int i = lo; i < hi; ++i) { rank[i] = run; run += mark[i]; }
+    for (int i = lo; i < hi; ++i) {
+      rank[i] = run;
+      run += tokmask[i] != 0u;
+    }
     __syncthreads();
   }
+  // active-expert rows of the task table (u = 0: the shared expert; routed experts follow in
+  // ascending id) and the token slots of the combine
   const int ns = a.sh.n_shared;
-  if (tid == 0) {
-    int total = 0;
-    for (int w = 0; w < kRouteWarps; ++w) total += s_wsum[w];
-    *a.ws.n_active = ns + total;
-    if (ns) a.ws.act_expert[0] = E;
-    if (ns) a.ws.act_ntok[0] = n;
+  int total = 0;
+#pragma unroll
+  for (int w = 0; w < kRouteWarps; ++w) total += s_wsum[w];
+  const int na = ns + total;
+  const int TD = D / kTileRows;
+  const int units_gu = ns * (a.L.shared.f / kTileRows) + total * (a.L.routed.f / kTileRows);
+  const int units_dn = na * TD;
+  int *tt = a.ws.task_tab;
+  for (int i = tid; i < E + ns; i += kRouteThreads) {
+    const bool shared = i == E;
+    uint32_t m = shared ? (n == 32 ? 0xFFFFFFFFu : (1u << n) - 1u) : tokmask[i];
+    if (!shared && a.out_counts) a.out_counts[i] = __popc(m);
+    if (!m) continue;
+    const int u = shared ? 0 : ns + rank[i];
+    const int nt = __popc(m);
+    const int F = shared ? a.L.shared.f : a.L.routed.f;
+    int *row = tt + kTabHead + u * kTabInts;
+    row[0] = i;
+    row[1] = nt;
+    int c = 0;
+    while (m) {
+      row[2 + c++] = __ffs(m) - 1;
+      m &= m - 1u;
+    }
+    int pg, pd;
+    row[11] = unit_split(D / kChunk, units_gu, nt, a.ws.min_streams, pg);
+    row[13] = unit_split(F / kChunk, units_dn, nt, a.ws.min_streams, pd);
+    s_cnt[0][u] = (F / kTileRows) * pg;
+    s_cnt[1][u] = pd;
   }
-  if (ns && tid < n) a.ws.act_tok[tid] = tid;
-  for (int i = tid; i < E; i += kRouteThreads)
-    if (mark[i]) a.ws.act_expert[ns + rank[i]] = i;
   for (int p = tid; p < n * K; p += kRouteThreads) {
     const int t = p / K, ex = s_idx[p];
-    const int u = ns + rank[ex];
-    int before = 0, after = 0;
-    for (int q = 0; q < n * K; ++q) {
-      if (s_idx[q] == ex) {
-        const int tq = q / K;
-        before += tq < t;
-        after += tq > t;
-      }
-    }
-    a.ws.slotpos[p] = u * kDecodeMaxTokens + before;
-    a.ws.act_tok[u * kDecodeMaxTokens + before] = t;
-    if (after == 0) a.ws.act_ntok[u] = before + 1;
+    a.ws.slotpos[p] = (ns + rank[ex]) * kDecodeMaxTokens + __popc(tokmask[ex] & ((1u << t) - 1u));
   }
-  if (a.out_counts) {
-    for (int i = tid; i < E; i += kRouteThreads) {
-      int c = 0;
-      if (mark[i])
-        for (int q = 0; q < n * K; ++q) c += s_idx[q] == i;
-      a.out_counts[i] = c;
+  __syncthreads();
+  if (warp == 0) {  // first task of each active expert: exclusive prefix over u
+    int run0 = 0, run1 = 0;
+    for (int u0 = 0; u0 < na; u0 += 32) {
+      const int u = u0 + lane;
+      const int c0v = u < na ? s_cnt[0][u] : 0, c1v = u < na ? s_cnt[1][u] : 0;
+      int i0 = c0v, i1 = c1v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v0 = __shfl_up_sync(0xffffffffu, i0, o), v1 = __shfl_up_sync(0xffffffffu, i1, o);
+        if (lane >= o) {
+          i0 += v0;
+          i1 += v1;
+        }
+      }
+      if (u < na) {
+        tt[kTabHead + u * kTabInts + 10] = run0 + i0 - c0v;
+        tt[kTabHead + u * kTabInts + 12] = run1 + i1 - c1v;
+      }
+      run0 += __shfl_sync(0xffffffffu, i0, 31);
+      run1 += __shfl_sync(0xffffffffu, i1, 31);
+    }
+    if (lane == 0) {
+      tt[0] = na;
+      tt[1] = run0;
+      tt[2] = run1;
+      tt[3] = 0;
     }
   }
   if (tid == 0) *a.ws.route_ticket = 0u;
 }
 
 // ------------------------------------------------------------------------------------------
-// shared pieces of the two GEMV kernels
+// GEMV arithmetic of one ring stage
 // ------------------------------------------------------------------------------------------
 // replicate the 256 x 4 int8 grid 32 times so that lane l reads copy l (bank l): conflict-free
-__device__ void load_grid_table(const int8_t *grid, uint32_t *tab) {
+__device__ __forceinline__ void load_grid_table(const int8_t *grid, uint32_t *tab, int nthreads) {
   const uint32_t *g = reinterpret_cast<const uint32_t *>(grid);
-  for (int row = threadIdx.x; row < 256; row += blockDim.x) {
+  for (int row = threadIdx.x; row < 256; row += nthreads) {
     const uint32_t v = __ldg(g + row);
     uint4 *dst = reinterpret_cast<uint4 *>(tab + row * 32);
 #pragma unroll
@@ -385,7 +495,7 @@ __device__ void load_grid_table(const int8_t *grid, uint32_t *tab) {
 // Unpacked operand bytes of one 32-weight block, 8 words: word q holds the operands of weights
 // 4q .. 4q+3 of the block (bytes 0..3).
 template <int FMT>
-__device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t sgn, const uint32_t *tab,
+__device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t sgn, uint32_t tab,
                                              int lane, uint32_t (&q)[8]) {
   if (FMT == MOE_FMT_Q2_32) {
     // Q2: word w covers weights 16w .. 16w+15; group kk of word w = weights 16w + 4kk + j
@@ -400,7 +510,7 @@ __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t 
     for (int g = 0; g < 8; ++g) {
       const uint32_t iw = g < 4 ? w0 : w1;
       const uint32_t idx = (iw >> (8 * (g & 3))) & 0xFFu;
-      const uint32_t gw = tab[idx * 32 + lane];
+      const uint32_t gw = lds_u32(tab + (idx * 32 + lane) * 4);
       const uint32_t m = prmt_sign_bytes(sgn << (7 - g));
       q[g] = (gw ^ m) + (m & 0x01010101u);
     }
@@ -429,487 +539,675 @@ __device__ __forceinline__ float block_value(int S, int M) {
   return FMT == MOE_FMT_Q2_32 ? static_cast<float>(2 * S - 3 * M) : static_cast<float>(S);
 }
 
-struct StageSmem {
-  uint4 *a0, *a1;      // plane A of matrix 0 / 1 (gate / up); a1 unused by k_down
-  __half2 *s0, *s1;
-  uint2 *g0, *g1;
-};
-
-// GEMV of NR matrices (1 or 2) over kc chunks for NT tokens, thread = row of the tile.  The
-// activation factor of (token t, chunk c) is cf[t * cf_stride + (c >> cf_shift)].
-template <int FMT, int NT, int NR>
-__device__ __forceinline__ void gemv_tile(const StageSmem &st, int kc, const int16_t *xq, const int *msum,
-                                          const uint32_t *tab, const float *cf, int cf_stride, int cf_shift,
-                                          float (&acc)[2][kDecodeMaxTokens]) {
-  const int r = threadIdx.x, lane = r & 31;
-  const int ncols = kc * kChunk;
-#pragma unroll 1
-  for (int c = 0; c < kc; ++c) {
-    uint4 A[2];
-    float2 sc[2];
-    uint2 G[2] = {make_uint2(0, 0), make_uint2(0, 0)};
-    A[0] = st.a0[c * kTileRows + r];
-    sc[0] = __half22float2(st.s0[c * kTileRows + r]);
-    if (FMT == MOE_FMT_CB35_32) G[0] = st.g0[c * kTileRows + r];
-    if (NR == 2) {
-      A[1] = st.a1[c * kTileRows + r];
-      sc[1] = __half22float2(st.s1[c * kTileRows + r]);
-      if (FMT == MOE_FMT_CB35_32) G[1] = st.g1[c * kTileRows + r];
-    }
-    float cacc[NR][NT];
-#pragma unroll
-    for (int m = 0; m < NR; ++m)
-#pragma unroll
-      for (int t = 0; t < NT; ++t) cacc[m][t] = 0.f;
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      uint32_t q[NR][8];
-#pragma unroll
-      for (int m = 0; m < NR; ++m) {
-        const uint32_t w0 = b ? A[m].z : A[m].x, w1 = b ? A[m].w : A[m].y;
-        unpack_block<FMT>(w0, w1, b ? G[m].y : G[m].x, tab, lane, q[m]);
-      }
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const int4 *xp = reinterpret_cast<const int4 *>(xq + t * ncols + c * kChunk + 32 * b);
-        const int4 p[4] = {xp[0], xp[1], xp[2], xp[3]};
-        const int M = FMT == MOE_FMT_Q2_32 ? msum[t * (2 * kc) + 2 * c + b] : 0;
-#pragma unroll
-        for (int m = 0; m < NR; ++m) {
-          const int S = block_dot(q[m], p);
-          cacc[m][t] = fmaf(block_value<FMT>(S, M), b ? sc[m].y : sc[m].x, cacc[m][t]);
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const float f = cf[t * cf_stride + (c >> cf_shift)];
-#pragma unroll
-      for (int m = 0; m < NR; ++m) acc[m][t] = fmaf(cacc[m][t], f, acc[m][t]);
-    }
-  }
-}
-
-template <int FMT, int NR>
-__device__ __forceinline__ void gemv_dispatch(int nt, const StageSmem &st, int kc, const int16_t *xq,
-                                              const int *msum, const uint32_t *tab, const float *cf,
-                                              int cf_stride, int cf_shift, float (&acc)[2][kDecodeMaxTokens]) {
-  switch (nt) {
-    case 1: gemv_tile<FMT, 1, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-    case 2: gemv_tile<FMT, 2, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-    case 3: gemv_tile<FMT, 3, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-    case 4: gemv_tile<FMT, 4, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-    case 5: gemv_tile<FMT, 5, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-    case 6: gemv_tile<FMT, 6, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-    case 7: gemv_tile<FMT, 7, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-    default: gemv_tile<FMT, 8, NR>(st, kc, xq, msum, tab, cf, cf_stride, cf_shift, acc); break;
-  }
-}
-
-// ------------------------------------------------------------------------------------------
-// persistent GEMV kernels: each CTA walks the task list (task = blockIdx.x + i * gridDim.x)
-// with a two-stage bulk-copy ring, so that the next task's weight tile and activation rows are
-// in flight while the current task computes.
-// ------------------------------------------------------------------------------------------
 __host__ __device__ inline int align128(int v) { return (v + 127) & ~127; }
 
-// one stage: weights of nr matrices over kc chunks + activations of up to 8 tokens
-struct StagePlan {
-  int a, s, g, xq, msum, fac, bytes;
+// Shared memory of the GEMV kernels:
+//   [RingHdr][task table][stage 0] .. [stage kRing-1][grid table (CB35)]
+// A stage holds, for up to CMAX chunks: plane A [NR][CMAX][128][16 B], plane S [NR][CMAX][128]
+// [4 B], plane G [NR][CMAX][128][8 B] (CB35), then the records [8 tokens][CMAX][144 B].
+struct RingPlan {
+  int table, stage0, a, s, g, rec, stage, tab, total;
 };
 
-__host__ __device__ inline StagePlan stage_plan(int fmt, int nr, int kc, int fac_per_tok) {
-  StagePlan p;
-  int off = 0;
-  p.a = off;
-  off += align128(nr * kc * kTileRows * 16);
-  p.s = off;
-  off += align128(nr * kc * kTileRows * 4);
-  p.g = off;
-  if (fmt == MOE_FMT_CB35_32) off += align128(nr * kc * kTileRows * 8);
-  p.xq = off;
-  off += align128(kDecodeMaxTokens * kc * kChunk * 2);
-  p.msum = off;
-  off += align128(kDecodeMaxTokens * kc * 2 * 4);
-  p.fac = off;
-  off += align128(kDecodeMaxTokens * fac_per_tok * 4);
-  p.bytes = off;
-  return p;
-}
+// Per-stage description written by the producer before it arms the stage's barrier.
+struct StageInfo {
+  int task;    // -1: no more work
+  int u;       // active expert
+  int mt;      // 128-row tile
+  int seg;     // K segment of the stage
+  int ntok;
+  int nch;     // chunks in the stage
+  int flags;   // k* bits | pieces of the unit << 8 | K segments of the unit << 16
+  int c0;      // first chunk of the stage
+};
+constexpr int kPieceStart = 1, kSegStart = 2, kSegEnd = 4, kPieceEnd = 8;
+__device__ __forceinline__ int info_pieces(int flags) { return (flags >> 8) & 0xFF; }
+__device__ __forceinline__ int info_nseg(int flags) { return flags >> 16; }
 
-// kernel shared memory: [2 mbarriers + flags (128 B)][task table][stage 0][stage 1][grid table]
-// (one stage when the ring depth NST is 1: the next task is issued after the current one)
-struct PersistPlan {
-  int table, stage0, stage1, tab, total;
-  StagePlan st;
+struct RingHdr {
+  uint64_t full[kRing];
+  uint64_t empty[kRing];
+  uint64_t cbar;  // barrier of the consumer warps (kConsWarps arrivals)
+  StageInfo info[kRing];
+  int n_active;
+  volatile int abort;
+  int flag[2];
+  float wmax[2][kConsWarps][kDecodeMaxTokens];
+  float tot[2][kDecodeMaxTokens][kTileRows];  // running unit sums of an unsplit unit (thread = row)
 };
 
-__host__ __device__ inline PersistPlan persist_plan(int fmt, int nr, int kc, int fac_per_tok, int umax, int nst) {
-  PersistPlan p;
-  p.st = stage_plan(fmt, nr, kc, fac_per_tok);
-  int off = 128;
-  p.table = off;
-  off += align128((1 + umax * (2 + kDecodeMaxTokens)) * 4);
+__host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax, int umax) {
+  RingPlan p;
+  p.table = align128(static_cast<int>(sizeof(RingHdr)));
+  int off = p.table + align128((kTabHead + kTabInts * umax) * 4);
   p.stage0 = off;
-  off += p.st.bytes;
-  p.stage1 = nst > 1 ? off : p.stage0;
-  if (nst > 1) off += p.st.bytes;
+  int so = 0;
+  p.a = so;
+  so += align128(nr * cmax * kTileRows * 16);
+  p.s = so;
+  so += align128(nr * cmax * kTileRows * 4);
+  p.g = so;
+  if (fmt == MOE_FMT_CB35_32) so += align128(nr * cmax * kTileRows * 8);
+  p.rec = so;
+  so += align128(kDecodeMaxTokens * cmax * static_cast<int>(sizeof(ActRec)));
+  p.stage = so;
+  off += ring_depth(fmt) * so;
   p.tab = off;
   if (fmt == MOE_FMT_CB35_32) off += 256 * 32 * 4;
   p.total = off;
   return p;
 }
 
-// Task table in shared memory: [n_active][expert of u][ntok of u][8 tokens of u]
-struct TaskTable {
-  int *base;
-  int umax;
-  __device__ int n_active() const { return base[0]; }
-  __device__ int expert(int u) const { return base[1 + u]; }
-  __device__ int ntok(int u) const { return base[1 + umax + u]; }
-  __device__ int tok(int u, int i) const { return base[1 + 2 * umax + u * kDecodeMaxTokens + i]; }
+// Tokens T0 .. T0+TN-1 of chunk c: NR rows (thread = row of the tile) against the tokens'
+// records; the chunk sums are scaled by the chunk's activation factor into acc.  `rec` is the
+// shared address of the stage's records ([token][CMAX chunks][144 B]).
+template <int FMT, int T0, int TN, int NR, int CMAX>
+__device__ __forceinline__ void chunk_tokens(const uint4 (&A)[NR], const float2 (&sc)[NR], const uint2 (&G)[NR],
+                                             uint32_t rec, int c, uint32_t tab, int lane,
+                                             float (&acc)[2][kDecodeMaxTokens]) {
+  constexpr uint32_t kRec = sizeof(ActRec);
+  float cacc[NR][TN];
+#pragma unroll
+  for (int m = 0; m < NR; ++m)
+#pragma unroll
+    for (int t = 0; t < TN; ++t) cacc[m][t] = 0.f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    uint32_t q[NR][8];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+      const uint32_t w0 = b ? A[m].z : A[m].x, w1 = b ? A[m].w : A[m].y;
+      unpack_block<FMT>(w0, w1, b ? G[m].y : G[m].x, tab, lane, q[m]);
+    }
+#pragma unroll
+    for (int t = 0; t < TN; ++t) {
+      const uint32_t ra = rec + ((T0 + t) * CMAX + c) * kRec;
+      const uint4 u0 = lds_u128(ra + 64 * b), u1 = lds_u128(ra + 64 * b + 16), u2 = lds_u128(ra + 64 * b + 32),
+                  u3 = lds_u128(ra + 64 * b + 48);
+      const int4 p[4] = {make_int4(u0.x, u0.y, u0.z, u0.w), make_int4(u1.x, u1.y, u1.z, u1.w),
+                         make_int4(u2.x, u2.y, u2.z, u2.w), make_int4(u3.x, u3.y, u3.z, u3.w)};
+      const int M = FMT == MOE_FMT_Q2_32 ? static_cast<int>(lds_u32(ra + offsetof(ActRec, m) + 4 * b)) : 0;
+#pragma unroll
+      for (int m = 0; m < NR; ++m) {
+        const int S = block_dot(q[m], p);
+        cacc[m][t] = fmaf(block_value<FMT>(S, M), b ? sc[m].y : sc[m].x, cacc[m][t]);
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TN; ++t) {
+    const float f = __uint_as_float(lds_u32(rec + ((T0 + t) * CMAX + c) * kRec + offsetof(ActRec, f)));
+#pragma unroll
+    for (int m = 0; m < NR; ++m) acc[m][T0 + t] = fmaf(cacc[m][t], f, acc[m][T0 + t]);
+  }
+}
+
+// GEMV of NR matrices (1 or 2) over the nch chunks of one stage for tokens T0 .. T0+TN-1.
+template <int FMT, int T0, int TN, int NR, int CMAX>
+__device__ __forceinline__ void gemv_stage(const unsigned char *st, const RingPlan &P, int nch, uint32_t tab,
+                                           float (&acc)[2][kDecodeMaxTokens]) {
+  const int r = threadIdx.x, lane = r & 31;
+  const uint32_t base = smem_u32(st);
+  const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g, rec = base + P.rec;
+#pragma unroll kGemvUnroll
+  for (int c = 0; c < nch; ++c) {
+    uint4 A[NR];
+    float2 sc[NR];
+    uint2 G[NR];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+      const uint32_t row = (m * CMAX + c) * kTileRows + r;
+      A[m] = lds_u128(pa + row * 16);
+      const uint32_t s2 = lds_u32(ps + row * 4);
+      sc[m] = __half22float2(*reinterpret_cast<const __half2 *>(&s2));
+      G[m] = FMT == MOE_FMT_CB35_32 ? lds_u64(pg + row * 8) : make_uint2(0u, 0u);
+    }
+    chunk_tokens<FMT, T0, TN, NR, CMAX>(A, sc, G, rec, c, tab, lane, acc);
+  }
+}
+
+// Up to four tokens per pass over the stage (more tokens take a second pass, unpacking the
+// codes again), which keeps the loop's registers within three CTAs per SM.
+template <int FMT, int NR, int CMAX>
+__device__ __forceinline__ void gemv_dispatch(int nt, const unsigned char *st, const RingPlan &P, int nch,
+                                              uint32_t tab, float (&acc)[2][kDecodeMaxTokens]) {
+  switch (nt < 4 ? nt : 4) {
+    case 1: gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc); break;
+    case 2: gemv_stage<FMT, 0, 2, NR, CMAX>(st, P, nch, tab, acc); break;
+    case 3: gemv_stage<FMT, 0, 3, NR, CMAX>(st, P, nch, tab, acc); break;
+    default: gemv_stage<FMT, 0, 4, NR, CMAX>(st, P, nch, tab, acc); break;
+  }
+  switch (nt) {
+    case 5: gemv_stage<FMT, 4, 1, NR, CMAX>(st, P, nch, tab, acc); break;
+    case 6: gemv_stage<FMT, 4, 2, NR, CMAX>(st, P, nch, tab, acc); break;
+    case 7: gemv_stage<FMT, 4, 3, NR, CMAX>(st, P, nch, tab, acc); break;
+    case 8: gemv_stage<FMT, 4, 4, NR, CMAX>(st, P, nch, tab, acc); break;
+    default: break;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// producer / consumer plumbing
+// ------------------------------------------------------------------------------------------
+// Bounded wait that also gives up when the other role raised the CTA's abort flag.  Uniform
+// over the warp.
+__device__ __forceinline__ bool ring_wait(RingHdr *H, uint64_t *bar, uint32_t parity, uint64_t limit) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!__all_sync(0xffffffffu, ok)) {
+    const long long t0 = clock64();
+    while (!ok) {
+      ok = mbar_try_wait(bar, parity);
+      if (!ok && (H->abort || static_cast<uint64_t>(clock64() - t0) > limit)) break;
+    }
+    ok = __all_sync(0xffffffffu, ok);
+  }
+  return ok;
+}
+
+// Barrier of the four consumer warps (the producer warp runs on), bounded.
+__device__ __forceinline__ bool cons_sync(RingHdr *H, uint32_t &ph, uint64_t limit) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&H->cbar);
+  const bool ok = ring_wait(H, &H->cbar, ph, limit);
+  ph ^= 1u;
+  return ok;
+}
+
+__device__ __forceinline__ void cons_fail(const DecodeArgs &a, RingHdr *H) {
+  if ((threadIdx.x & 31) == 0) {
+    flag_error(a.err, kErrTimeout);
+    H->abort = 1;
+  }
+}
+
+
+// Load the task table (one round of independent loads) and check it.  Returns the task count,
+// or -1 (uniform over the warp) when an entry is out of range.
+template <bool GU>
+__device__ __forceinline__ int producer_tables(const DecodeArgs &a, RingHdr *H, int *tb) {
+  const int lane = threadIdx.x & 31;
+  const int umax = a.ws.umax, E = a.sh.e, D = a.sh.d;
+  const int4 *src = reinterpret_cast<const int4 *>(a.ws.task_tab);
+  int4 *dst = reinterpret_cast<int4 *>(tb);
+  for (int i = lane; i < (kTabHead + kTabInts * umax) / 4; i += 32) dst[i] = __ldcg(src + i);
+  __syncwarp();
+  const int na = tb[0];
+  const int total = GU ? tb[1] : tb[2];
+  bool bad = na < 1 || na > umax || total < 1;
+  for (int u = lane; !bad && u < na; u += 32) {
+    const int *row = tb + kTabHead + u * kTabInts;
+    const int e = row[0], nt = row[1];
+    bool b = e < 0 || e > E || (e == E) != (a.sh.n_shared && u == 0) || nt < 1 || nt > kDecodeMaxTokens;
+    for (int i = 0; !b && i < nt; ++i) b = row[2 + i] < 0 || row[2 + i] >= a.n;
+    if (!b) {
+      const int F = e == E ? a.L.shared.f : a.L.routed.f;
+      const int nc = (GU ? D : F) / kChunk;
+      const int pk = row[GU ? 11 : 13];
+      const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
+      b = (seg != 2 && seg != 4) || nseg * seg != nc || len < 1 || len > nseg || pieces != (nseg + len - 1) / len;
+      const int cnt = GU ? (F / kTileRows) * pieces : pieces;
+      const int base = row[GU ? 10 : 12];
+      const int next = u + 1 < na ? row[kTabInts + (GU ? 10 : 12)] : total;
+      b = b || base + cnt != next || (u == 0 && base != 0);
+    }
+    bad = b;
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad) return -1;
+  if (lane == 0) H->n_active = na;
+  __syncwarp();
+  return GU ? total : total * (D / kTileRows);
+}
+
+// largest u with first-task(u) <= r (first tasks increase with u, first-task(0) = 0)
+template <bool GU>
+__device__ __forceinline__ int find_expert(const int *tb, int na, int r) {
+  int lo = 0, hi = na - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tb[kTabHead + mid * kTabInts + (GU ? 10 : 12)] <= r) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// The producer warp: work queue -> bulk copies into the ring.  Every stage it arms is waited
+// for (bounded) before the warp leaves, so no copy is in flight when the CTA exits.
+template <int FMT, bool GU>
+__device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H) {
+  constexpr int NR = GU ? 2 : 1;
+  constexpr int CMAX = GU ? kGuStageChunks : kDnStageChunks;
+  constexpr int RING = ring_depth(FMT);
+  const int lane = threadIdx.x & 31;
+  const int D = a.sh.d, E = a.sh.e;
+  int *tb = reinterpret_cast<int *>(smem + P.table);
+  unsigned *ctr = a.ws.counters + (GU ? 0 : 1);
+  // gate/up reads the router kernel's tables, so it waits for that kernel first.  The down
+  // kernel's tables and work queue come from the router kernel too (complete before gate/up,
+  // the kernel before down, could start), so down loads them and issues the weight copies of
+  // its first task while gate/up finishes; the h records wait for gate/up.
+  if (GU) griddep_wait();
+  bool waited = GU;
+  int npend = 0, pend_slot[RING], pend_c0[RING];
+  int task = 0;
+  if (lane == 0) task = static_cast<int>(atomicAdd(ctr, 1u));  // in flight while the table loads
+  const int n_tasks = producer_tables<GU>(a, H, tb);
+  bool ok = n_tasks >= 0;
+  if (!ok && lane == 0) flag_error(a.err, kErrBadIndex);
+  const int na = ok ? H->n_active : 0;
+  const int TD = D / kTileRows;
+  const int per_mt = GU ? 0 : (ok ? n_tasks / TD : 0);
+  const uint64_t pol = l2_evict_first_policy();
+  int slot = 0;
+  uint32_t round = 0;
+  int last_round[RING];
+#pragma unroll
+  for (int s = 0; s < RING; ++s) last_round[s] = -1;
+  task = __shfl_sync(0xffffffffu, task, 0);
+  while (ok && task < n_tasks) {
+    int nxt = 0;
+    if (lane == 0) nxt = static_cast<int>(atomicAdd(ctr, 1u));  // fetched while this piece is issued
+    int u, mt, piece;
+    const int *tr = tb + kTabHead;
+    if (GU) {
+      u = find_expert<true>(tb, na, task);
+      const int pieces = (tr[u * kTabInts + 11] >> 8) & 0xFF;
+      const int r = task - tr[u * kTabInts + 10];
+      mt = r / pieces;
+      piece = r - mt * pieces;
+    } else {
+      mt = task / per_mt;
+      const int r = task - mt * per_mt;
+      u = find_expert<false>(tb, na, r);
+      piece = r - tr[u * kTabInts + 12];
+    }
+    const int *row = tr + u * kTabInts;
+    const int e = row[0], ntok = row[1];
+    const int pk = row[GU ? 11 : 13];
+    const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
+    const bool shared = a.sh.n_shared && e == E;
+    const ExpertGroup &G = shared ? a.L.shared : a.L.routed;
+    const int eidx = shared ? 0 : e;
+    const int nc = GU ? D / kChunk : G.f / kChunk;
+    const int cbeg = piece * len * seg, cend = min(nseg, (piece + 1) * len) * seg;
+    const int sch = GU ? kGuStageChunks : seg;
+    for (int c0 = cbeg; c0 < cend; c0 += sch) {
+      if (round > 0) ok = ring_wait(H, &H->empty[slot], (round - 1) & 1u, a.spin_limit);
+      if (!ok) break;
+      const int nch = min(sch, cend - c0);
+      const uint32_t wbytes = nch * kTileRows * (FMT == MOE_FMT_CB35_32 ? 28 : 20);
+      const uint32_t rbytes = nch * static_cast<uint32_t>(sizeof(ActRec));
+      if (lane == 0) {
+        StageInfo &in = H->info[slot];
+        in.task = task;
+        in.u = u;
+        in.mt = mt;
+        in.seg = c0 / seg;
+        in.ntok = ntok;
+        in.nch = nch;
+        in.flags = (c0 == cbeg ? kPieceStart : 0) | (c0 % seg == 0 ? kSegStart : 0) |
+                   ((c0 + nch) % seg == 0 ? kSegEnd : 0) | (c0 + nch == cend ? kPieceEnd : 0) | (pieces << 8) |
+                   (nseg << 16);
+        in.c0 = c0;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&H->full[slot], NR * wbytes + ntok * rbytes);
+      }
+      __syncwarp();
+      unsigned char *st = smem + P.stage0 + slot * P.stage;
+      // copy l of the stage, issued by lane l: NR x (A, S[, G]) weight planes, then one run of
+      // records per token
+      constexpr int kPlanes = FMT == MOE_FMT_CB35_32 ? 3 : 2;
+      if (lane < NR * kPlanes) {
+        const int m = lane / kPlanes, pl = lane - m * kPlanes;
+        const int64_t mat = static_cast<int64_t>(eidx) * 3 + (GU ? m : 2);
+        const int64_t slot0 = (static_cast<int64_t>(mt) * nc + c0) * kTileRows;
+        if (pl == 0)
+          bulk_g2s_hint(st + P.a + m * CMAX * kTileRows * 16, G.a + mat * G.a_mat + slot0 * 16,
+                        nch * kTileRows * 16, &H->full[slot], pol);
+        else if (pl == 1)
+          bulk_g2s_hint(st + P.s + m * CMAX * kTileRows * 4, G.s + mat * G.s_mat + slot0, nch * kTileRows * 4,
+                        &H->full[slot], pol);
+        else
+          bulk_g2s_hint(st + P.g + m * CMAX * kTileRows * 8, G.g + mat * G.g_mat + slot0, nch * kTileRows * 8,
+                        &H->full[slot], pol);
+      }
+      // records of the tokens: one copy per token, lanes NR * kPlanes ..
+      auto issue_records = [&](int sl, int cc0) {
+        const int i = lane - NR * kPlanes;
+        if (i >= 0 && i < ntok) {
+          const ActRec *src = GU ? a.ws.xrec + static_cast<int64_t>(row[2 + i]) * (D / kChunk) + cc0
+                                 : a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + i) * (a.ws.fmax / kChunk) + cc0;
+          bulk_g2s(smem + P.stage0 + sl * P.stage + P.rec + i * CMAX * static_cast<int>(sizeof(ActRec)), src,
+                   min(sch, cend - cc0) * static_cast<uint32_t>(sizeof(ActRec)), &H->full[sl]);
+        }
+      };
+      if (waited) {
+        issue_records(slot, c0);
+      } else {
+#pragma unroll
+        for (int q = 0; q < RING; ++q) {
+          pend_slot[q] = q == npend ? slot : pend_slot[q];
+          pend_c0[q] = q == npend ? c0 : pend_c0[q];
+        }
+        ++npend;
+      }
+#pragma unroll
+      for (int s = 0; s < RING; ++s) last_round[s] = s == slot ? static_cast<int>(round) : last_round[s];
+      if (++slot == RING) {
+        slot = 0;
+        ++round;
+      }
+      if (!waited && (npend == RING || c0 + sch >= cend)) {
+        griddep_wait();  // the previous kernel's records are complete
+        waited = true;
+#pragma unroll
+        for (int q = 0; q < RING; ++q)
+          if (q < npend) issue_records(pend_slot[q], pend_c0[q]);
+        npend = 0;
+      }
+    }
+    task = __shfl_sync(0xffffffffu, nxt, 0);
+  }
+  if (!waited) {  // no work taken before the wait (or a bad table)
+    griddep_wait();
+#pragma unroll
+    for (int q = 0; q < RING; ++q)
+      if (q < npend) ok = false;  // cannot happen: a task's stages flush before the next task
+  }
+  // end of work: one more stage, with no copies, tells the consumers to leave
+  if (ok && round > 0) ok = ring_wait(H, &H->empty[slot], (round - 1) & 1u, a.spin_limit);
+  if (ok) {
+#pragma unroll
+    for (int s = 0; s < RING; ++s) last_round[s] = s == slot ? static_cast<int>(round) : last_round[s];
+  }
+  if (lane == 0) {
+    if (ok) {
+      H->info[slot].task = -1;
+      mbar_arrive(&H->full[slot]);
+    } else {
+      if (n_tasks >= 0) flag_error(a.err, kErrTimeout);
+      H->abort = 1;
+    }
+    // drain: the last phase armed on each stage has completed before the warp leaves
+#pragma unroll
+    for (int s = 0; s < RING; ++s)
+      if (last_round[s] >= 0) mbar_wait_bounded(&H->full[s], static_cast<uint32_t>(last_round[s]) & 1u, kDrainLimit);
+  }
+}
+
+// Sums of a split unit's segment partials in segment order (the last piece of the unit), row r:
+// tot[m][t] = sum_j part[j][m][t][r].  32 loads are in flight at a time.
+template <int NR>
+__device__ __forceinline__ void sum_segments(const float *part, int nseg, int ntok, float (&tot)[2][kDecodeMaxTokens]) {
+  const int r = threadIdx.x;
+  constexpr int kSegStride = NR * kPartStride;
+  constexpr int TPR = 2 / NR;  // tokens per round
+#pragma unroll
+  for (int t0 = 0; t0 < kDecodeMaxTokens; t0 += TPR) {
+    if (t0 < ntok) {
+      float v[TPR][NR][16];
+#pragma unroll
+      for (int i = 0; i < TPR; ++i)
+#pragma unroll
+        for (int m = 0; m < NR; ++m)
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (t0 + i < ntok && j < nseg)
+              v[i][m][j] = __ldcg(part + j * kSegStride + m * kPartStride + (t0 + i) * kTileRows + r);
+#pragma unroll
+      for (int i = 0; i < TPR; ++i)
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < nseg) s += v[i][m][j];
+          if (t0 + i < ntok) tot[m][t0 + i] = s;
+        }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// consumers: gate/up epilogue (SwiGLU + h quantisation) and down epilogue (o + combine)
+// ------------------------------------------------------------------------------------------
+struct ConsState {
+  uint32_t cph;   // parity of the consumer barrier
+  int nflag;      // uses of H->flag
+  int nwmax;      // uses of H->wmax
 };
 
-// Load the routing tables once per CTA and check them; false (same on all threads) if bad.
-__device__ bool load_table(const DecodeArgs &a, TaskTable &tt) {
-  const int umax = a.ws.umax;
-  int *b = tt.base;
-  for (int i = threadIdx.x; i < 1 + umax * (2 + kDecodeMaxTokens); i += blockDim.x) {
-    int v;
-    if (i == 0) v = __ldcg(a.ws.n_active);
-    else if (i < 1 + umax) v = __ldcg(a.ws.act_expert + (i - 1));
-    else if (i < 1 + 2 * umax) v = __ldcg(a.ws.act_ntok + (i - 1 - umax));
-    else v = __ldcg(a.ws.act_tok + (i - 1 - 2 * umax));
-    b[i] = v;
+// Ticket of a split unit; true on the piece that arrives last (uniform over the consumers).
+__device__ __forceinline__ bool unit_ticket(const DecodeArgs &a, RingHdr *H, ConsState &cs, unsigned *ticket,
+                                            unsigned target, bool &ok) {
+  ok = cons_sync(H, cs.cph, a.spin_limit);  // every consumer's partial stores precede the ticket
+  if (!ok) return false;
+  const int fb = cs.nflag++ & 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const bool last = atomicAdd(ticket, 1u) == target;
+    if (last) __threadfence();
+    H->flag[fb] = last;
+  }
+  ok = cons_sync(H, cs.cph, a.spin_limit);
+  return ok && H->flag[fb];
+}
+
+template <int FMT>
+__device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in) {
+  const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
+  const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags);
+  const int nseg = info_nseg(in.flags);
+  float tot[2][kDecodeMaxTokens];
+#pragma unroll
+  for (int t = 0; t < kDecodeMaxTokens; ++t)
+    if (t < ntok) {
+      tot[0][t] = H->tot[0][t][r];
+      tot[1][t] = H->tot[1][t][r];
+    }
+  if (pieces > 1) {
+    unsigned *ticket = a.ws.gu_ticket + u * a.ws.tmax + mt;
+    bool ok;
+    const bool last = unit_ticket(a, H, cs, ticket, static_cast<unsigned>(pieces - 1), ok);
+    if (!ok) return false;
+    if (!last) return true;
+    sum_segments<2>(a.ws.gu_part + static_cast<int64_t>(u * a.ws.tmax + mt) * a.ws.gu_nseg * 2 * kPartStride, nseg,
+                    ntok, tot);
+    if (r == 0) *ticket = 0u;
+  }
+  // SwiGLU, then h of each token quantised over the tile's 128 rows
+  const int wb = cs.nwmax++ & 1;
+  float hv[kDecodeMaxTokens];
+#pragma unroll
+  for (int t = 0; t < kDecodeMaxTokens; ++t) {
+    hv[t] = 0.f;
+    if (t < ntok) {
+      hv[t] = silu_f(tot[0][t]) * tot[1][t];
+      float m = fabsf(hv[t]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) H->wmax[wb][warp][t] = m;
+    }
+  }
+  if (!cons_sync(H, cs.cph, a.spin_limit)) return false;
+  const int fs = a.ws.fmax / kChunk;
+#pragma unroll
+  for (int t = 0; t < kDecodeMaxTokens; ++t) {
+    if (t < ntok) {
+      float mx = H->wmax[wb][0][t];
+#pragma unroll
+      for (int w = 1; w < kConsWarps; ++w) mx = fmaxf(mx, H->wmax[wb][w][t]);
+      const int e = fix16_exponent(mx);
+      const int m = fix16(hv[t], pow2f(e));
+      ActRec *rec = a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + t) * fs + 2 * mt + (r >> 6);
+      rec->x[r & 63] = static_cast<int16_t>(m);
+      int sum = m;  // warp = 32 consecutive rows = one block of the down matrix's K
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) rec->m[warp & 1] = sum;
+      if ((r & 63) == 0) {
+        rec->f = pow2f(-e) * (FMT == MOE_FMT_Q2_32 ? 0.5f : 1.0f);
+        rec->pad = 0u;
+      }
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool dn_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in) {
+  const int r = threadIdx.x;
+  const int D = a.sh.d, TD = D / kTileRows;
+  const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags);
+  float tot[2][kDecodeMaxTokens];
+#pragma unroll
+  for (int t = 0; t < kDecodeMaxTokens; ++t)
+    if (t < ntok) tot[0][t] = H->tot[0][t][r];
+  if (pieces > 1) {
+    unsigned *ticket = a.ws.dn_ticket + u * TD + mt;
+    bool ok;
+    const bool last = unit_ticket(a, H, cs, ticket, static_cast<unsigned>(pieces - 1), ok);
+    if (!ok) return false;
+    if (!last) return true;
+    const int nseg = info_nseg(in.flags);
+    sum_segments<1>(a.ws.dn_part + static_cast<int64_t>(u * TD + mt) * a.ws.dn_nseg * kPartStride, nseg, ntok, tot);
+    if (r == 0) *ticket = 0u;
+  }
+  const int row = mt * kTileRows + r;
+#pragma unroll
+  for (int t = 0; t < kDecodeMaxTokens; ++t)
+    if (t < ntok) a.ws.o[(static_cast<int64_t>(u) * kDecodeMaxTokens + t) * D + row] = tot[0][t];
+  return true;
+}
+
+template <int FMT, bool GU>
+__device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H) {
+  constexpr int NR = GU ? 2 : 1;
+  constexpr int CMAX = GU ? kGuStageChunks : kDnStageChunks;
+  constexpr int RING = ring_depth(FMT);
+  const int r = threadIdx.x, lane = r & 31;
+  const int D = a.sh.d, TD = D / kTileRows;
+  uint32_t *tab = reinterpret_cast<uint32_t *>(smem + P.tab);
+  ConsState cs{0u, 0, 0};
+  if (FMT == MOE_FMT_CB35_32) {
+    load_grid_table(a.grid, tab, kTileRows);
+    if (!cons_sync(H, cs.cph, a.spin_limit)) {
+      cons_fail(a, H);
+      return;
+    }
+  }
+  float seg[2][kDecodeMaxTokens];
+  int slot = 0;
+  uint32_t round = 0;
+  for (;;) {
+    if (!ring_wait(H, &H->full[slot], round & 1u, a.spin_limit)) {
+      cons_fail(a, H);
+      return;
+    }
+    const StageInfo in = H->info[slot];
+    if (in.task < 0) return;
+    const int pieces = info_pieces(in.flags);
+    if ((in.flags & kPieceStart) && pieces == 1) {
+#pragma unroll
+      for (int m = 0; m < NR; ++m)
+#pragma unroll
+        for (int t = 0; t < kDecodeMaxTokens; ++t) H->tot[m][t][r] = 0.f;
+    }
+    if (in.flags & kSegStart) {
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int t = 0; t < kDecodeMaxTokens; ++t) seg[m][t] = 0.f;
+    }
+    gemv_dispatch<FMT, NR, CMAX>(in.ntok, smem + P.stage0 + slot * P.stage, P, in.nch, smem_u32(tab), seg);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&H->empty[slot]);
+    if (in.flags & kSegEnd) {
+      if (pieces > 1) {
+        // segment sum of a split unit -> partial buffer [segment][matrix][token][row]
+        float *part = GU ? a.ws.gu_part + (static_cast<int64_t>(in.u * a.ws.tmax + in.mt) * a.ws.gu_nseg + in.seg) *
+                                              2 * kPartStride
+                         : a.ws.dn_part + (static_cast<int64_t>(in.u * TD + in.mt) * a.ws.dn_nseg + in.seg) * kPartStride;
+#pragma unroll
+        for (int m = 0; m < NR; ++m)
+#pragma unroll
+          for (int t = 0; t < kDecodeMaxTokens; ++t)
+            if (t < in.ntok) part[m * kPartStride + t * kTileRows + r] = seg[m][t];
+      } else {
+#pragma unroll
+        for (int m = 0; m < NR; ++m)
+#pragma unroll
+          for (int t = 0; t < kDecodeMaxTokens; ++t)
+            if (t < in.ntok) H->tot[m][t][r] += seg[m][t];
+      }
+    }
+    if (in.flags & kPieceEnd) {
+      const bool ok = GU ? gu_finish<FMT>(a, H, cs, in) : dn_finish(a, H, cs, in);
+      if (!ok) {
+        cons_fail(a, H);
+        return;
+      }
+    }
+    if (++slot == RING) {
+      slot = 0;
+      ++round;
+    }
+  }
+}
+
+template <int FMT, bool GU>
+__global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const RingPlan P = ring_plan(FMT, GU ? 2 : 1, GU ? kGuStageChunks : kDnStageChunks, a.ws.umax);
+  RingHdr *H = reinterpret_cast<RingHdr *>(smem);
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < ring_depth(FMT); ++s) {
+      mbar_init(&H->full[s], 1);
+      mbar_init(&H->empty[s], kConsWarps);
+    }
+    mbar_init(&H->cbar, kConsWarps);
+    H->abort = 0;
+    fence_barrier_init();
   }
   __syncthreads();
-  const int na = tt.n_active();
-  bool bad = na < 0 || na > umax;
-  for (int u = threadIdx.x; !bad && u < na; u += blockDim.x) {
-    const int e = tt.expert(u), nt = tt.ntok(u);
-    bad = e < 0 || e > a.sh.e || (e == a.sh.e && !a.sh.n_shared) || nt < 1 || nt > kDecodeMaxTokens;
-    for (int i = 0; !bad && i < nt; ++i) bad = tt.tok(u, i) < 0 || tt.tok(u, i) >= a.n;
-  }
-  if (__syncthreads_or(bad)) {
-    if (threadIdx.x == 0) flag_error(a.err, kErrBadIndex);
-    return false;
-  }
-  return true;
-}
-
-struct StageView {
-  StageSmem w;
-  int16_t *xq;
-  int *msum;
-  float *fac;
-};
-
-__device__ __forceinline__ StageView stage_view(unsigned char *base, const StagePlan &p, int kc) {
-  StageView v;
-  v.w.a0 = reinterpret_cast<uint4 *>(base + p.a);
-  v.w.a1 = v.w.a0 + kc * kTileRows;
-  v.w.s0 = reinterpret_cast<__half2 *>(base + p.s);
-  v.w.s1 = v.w.s0 + kc * kTileRows;
-  v.w.g0 = reinterpret_cast<uint2 *>(base + p.g);
-  v.w.g1 = v.w.g0 + kc * kTileRows;
-  v.xq = reinterpret_cast<int16_t *>(base + p.xq);
-  v.msum = reinterpret_cast<int *>(base + p.msum);
-  v.fac = reinterpret_cast<float *>(base + p.fac);
-  return v;
-}
-
-// Wait for a stage's copies (parity `ph`), bounded; uniform result.  On a timeout the CTA
-// reports it and waits (bounded again) for the copies it issued before it leaves.
-__device__ __forceinline__ bool wait_stage(const DecodeArgs &a, uint64_t *bar, uint32_t ph, uint64_t *other,
-                                           uint32_t other_ph, bool other_pending) {
-  const bool ok = mbar_wait_bounded(bar, ph, a.spin_limit);
-  if (__syncthreads_or(!ok)) {
-    if (threadIdx.x == 0) flag_error(a.err, kErrTimeout);
-    mbar_wait_bounded(bar, ph, kDrainLimit);
-    if (other_pending) mbar_wait_bounded(other, other_ph, kDrainLimit);
-    return false;
-  }
-  return true;
-}
-
-// ------------------------------------------------------------------------------------------
-// gate / up + SwiGLU + h quantisation.  Task = (active expert u, 128-row tile mt, K-split s).
-// ------------------------------------------------------------------------------------------
-struct GuTask {
-  int u, mt, s;
-};
-
-__device__ __forceinline__ GuTask gu_task(int task, int Ts, int Tr, int S, int ns) {
-  GuTask t;
-  if (task < Ts * S) {
-    t.u = 0; t.mt = task / S; t.s = task % S;
+  if (threadIdx.x >= kTileRows) {
+    producer<FMT, GU>(a, smem, P, H);
   } else {
-    const int b = task - Ts * S;
-    t.u = ns + b / (Tr * S);
-    const int r = b % (Tr * S);
-    t.mt = r / S; t.s = r % S;
-  }
-  return t;
-}
-
-template <int FMT>
-__device__ __forceinline__ void gu_issue(const DecodeArgs &a, const TaskTable &tt, const GuTask &k,
-                                         const StageView &v, uint64_t *bar, int kc, int sfs) {
-  const int D = a.sh.d, nc = D / kChunk, ncols = kc * kChunk;
-  const int e = tt.expert(k.u), ntok = tt.ntok(k.u);
-  const bool shared = a.sh.n_shared && e == a.sh.e;
-  const ExpertGroup &G = shared ? a.L.shared : a.L.routed;
-  const int eidx = shared ? 0 : e;
-  const int64_t slot0 = (static_cast<int64_t>(k.mt) * nc + static_cast<int64_t>(k.s) * kc) * kTileRows;
-  const uint32_t abytes = kc * kTileRows * 16, sbytes = kc * kTileRows * 4, gbytes = kc * kTileRows * 8;
-  const uint32_t xbytes = ncols * 2, mbytes = 2 * kc * 4, fbytes = sfs * 4;
-  fence_proxy_async_smem();  // the stage was last read by generic loads
-  mbar_arrive_expect_tx(bar, 2 * (abytes + sbytes) + (FMT == MOE_FMT_CB35_32 ? 2 * gbytes : 0) +
-                                 ntok * (xbytes + mbytes + fbytes));
-#pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const int64_t mat = static_cast<int64_t>(eidx) * 3 + m;
-    bulk_g2s(m ? (void *)v.w.a1 : (void *)v.w.a0, G.a + mat * G.a_mat + slot0 * 16, abytes, bar);
-    bulk_g2s(m ? (void *)v.w.s1 : (void *)v.w.s0, G.s + mat * G.s_mat + slot0, sbytes, bar);
-    if (FMT == MOE_FMT_CB35_32)
-      bulk_g2s(m ? (void *)v.w.g1 : (void *)v.w.g0, G.g + mat * G.g_mat + slot0, gbytes, bar);
-  }
-  for (int i = 0; i < ntok; ++i) {
-    const int t = tt.tok(k.u, i);
-    bulk_g2s(v.xq + i * ncols, a.ws.xq + static_cast<int64_t>(t) * D + k.s * ncols, xbytes, bar);
-    bulk_g2s(v.msum + i * 2 * kc, a.ws.xsum + static_cast<int64_t>(t) * (D / 32) + k.s * 2 * kc, mbytes, bar);
-    bulk_g2s(v.fac + i * sfs, a.ws.xfac + static_cast<int64_t>(t) * sfs, fbytes, bar);
-  }
-}
-
-template <int FMT, int NST>
-__global__ void __launch_bounds__(128, MOE_GEMV_MIN_BLOCKS) k_gateup(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int S = a.ws.splits, D = a.sh.d, kc = D / kChunk / S, sfs = pad4(S);
-  const int ns = a.sh.n_shared;
-  const int Ts = ns ? a.L.shared.f / kTileRows : 0, Tr = a.L.routed.f / kTileRows;
-  const PersistPlan P = persist_plan(FMT, 2, kc, sfs, a.ws.umax, NST);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-  __shared__ int s_flag;
-  __shared__ float wmax[4][kDecodeMaxTokens];
-  TaskTable tt{reinterpret_cast<int *>(smem + P.table), a.ws.umax};
-  const StageView sv[2] = {stage_view(smem + P.stage0, P.st, kc), stage_view(smem + P.stage1, P.st, kc)};
-  uint32_t *tab = reinterpret_cast<uint32_t *>(smem + P.tab);
-  if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    fence_barrier_init();
-  }
-  if (FMT == MOE_FMT_CB35_32) load_grid_table(a.grid, tab);
-  if (!load_table(a, tt)) return;
-  const int n_tasks = Ts * S + (tt.n_active() - ns) * Tr * S;
-  int task = blockIdx.x;
-  if (task >= n_tasks) return;
-  if (threadIdx.x == 0) gu_issue<FMT>(a, tt, gu_task(task, Ts, Tr, S, ns), sv[0], &bars[0], kc, sfs);
-  uint32_t ph[2] = {0u, 0u};
-  const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
-  for (int it = 0; task < n_tasks; ++it, task += gridDim.x) {
-    const int cur = NST > 1 ? (it & 1) : 0;
-    const int next = task + gridDim.x;
-    if (NST > 1 && threadIdx.x == 0 && next < n_tasks)
-      gu_issue<FMT>(a, tt, gu_task(next, Ts, Tr, S, ns), sv[cur ^ 1], &bars[cur ^ 1], kc, sfs);
-    if (!wait_stage(a, &bars[cur], ph[cur], &bars[cur ^ 1], ph[cur ^ 1], NST > 1 && next < n_tasks)) return;
-    ph[cur] ^= 1u;
-    const GuTask k = gu_task(task, Ts, Tr, S, ns);
-    const int ntok = tt.ntok(k.u);
-    const StageView &v = sv[cur];
-
-    float acc[2][kDecodeMaxTokens];
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-      for (int t = 0; t < kDecodeMaxTokens; ++t) acc[m][t] = 0.f;
-    gemv_dispatch<FMT, 2>(ntok, v.w, kc, v.xq, v.msum, tab, v.fac + k.s, sfs, 31, acc);
-
-    bool have = true;
-    if (S > 1) {
-      // K-split partials; the last split of the tile to finish reduces them in split order
-      constexpr int kPartStride = 2 * kDecodeMaxTokens * kTileRows;  // floats per K-split
-      float *part = a.ws.gu_part + ((static_cast<int64_t>(k.u) * a.ws.tmax + k.mt) * S) * kPartStride;
-      float *ps = part + static_cast<int64_t>(k.s) * kPartStride;
-#pragma unroll
-      for (int t = 0; t < kDecodeMaxTokens; ++t) {
-        if (t < ntok) {
-          ps[t * kTileRows + r] = acc[0][t];
-          ps[(kDecodeMaxTokens + t) * kTileRows + r] = acc[1][t];
-        }
-      }
-      __threadfence();
-      __syncthreads();
-      unsigned *ticket = a.ws.gu_ticket + k.u * a.ws.tmax + k.mt;
-      if (threadIdx.x == 0) s_flag = atomicAdd(ticket, 1u) == static_cast<unsigned>(S - 1);
-      __syncthreads();
-      have = s_flag;
-      if (have) {
-        __threadfence();
-#pragma unroll
-        for (int t = 0; t < kDecodeMaxTokens; ++t) {
-          if (t < ntok) {
-            float gv[kMaxSplits], uv[kMaxSplits];
-#pragma unroll
-            for (int q = 0; q < kMaxSplits; ++q) {
-              if (q < S) {
-                const float *pq = part + static_cast<int64_t>(q) * kPartStride;
-                gv[q] = __ldcg(pq + t * kTileRows + r);
-                uv[q] = __ldcg(pq + (kDecodeMaxTokens + t) * kTileRows + r);
-              }
-            }
-            float g = 0.f, u = 0.f;
-#pragma unroll
-            for (int q = 0; q < kMaxSplits; ++q)
-              if (q < S) { g += gv[q]; u += uv[q]; }
-            acc[0][t] = g;
-            acc[1][t] = u;
-          }
-        }
-        if (threadIdx.x == 0) *ticket = 0u;
-      }
-    }
-    if (have) {
-      // SwiGLU, then h of each token quantised over the tile's 128 rows
-      float hv[kDecodeMaxTokens];
-#pragma unroll
-      for (int t = 0; t < kDecodeMaxTokens; ++t) {
-        hv[t] = t < ntok ? silu_f(acc[0][t]) * acc[1][t] : 0.f;
-        float m = fabsf(hv[t]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) wmax[warp][t] = m;
-      }
-      __syncthreads();
-      const int f = k.mt * kTileRows + r;
-      const int fs = a.ws.fmax / 32;
-#pragma unroll
-      for (int t = 0; t < kDecodeMaxTokens; ++t) {
-        if (t < ntok) {
-          const float mx = fmaxf(fmaxf(wmax[0][t], wmax[1][t]), fmaxf(wmax[2][t], wmax[3][t]));
-          const int e = fix16_exponent(mx);
-          const int m = fix16(hv[t], pow2f(e));
-          const int64_t row = static_cast<int64_t>(k.u) * kDecodeMaxTokens + t;
-          a.ws.hq[row * a.ws.fmax + f] = static_cast<int16_t>(m);
-          int sum = m;  // warp = 32 consecutive rows = one block of the down matrix's K
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-          if (lane == 0) a.ws.hsum[row * fs + f / 32] = sum;
-          if (r == 0) a.ws.hfac[row * a.ws.hfs + k.mt] = pow2f(-e) * (FMT == MOE_FMT_Q2_32 ? 0.5f : 1.0f);
-        }
-      }
-    }
-    __syncthreads();  // stage `cur` is refilled by the next issue
-    if (NST == 1 && threadIdx.x == 0 && next < n_tasks)
-      gu_issue<FMT>(a, tt, gu_task(next, Ts, Tr, S, ns), sv[0], &bars[0], kc, sfs);
-  }
-}
-
-// ------------------------------------------------------------------------------------------
-// down: o[u, i] = Wd_e h[u, i].  Task = (active expert u, 128-row tile mt of d_model).
-// ------------------------------------------------------------------------------------------
-template <int FMT>
-__device__ __forceinline__ void down_issue(const DecodeArgs &a, const TaskTable &tt, int u, int mt,
-                                           const StageView &v, uint64_t *bar) {
-  const int e = tt.expert(u), ntok = tt.ntok(u);
-  const bool shared = a.sh.n_shared && e == a.sh.e;
-  const ExpertGroup &G = shared ? a.L.shared : a.L.routed;
-  const int eidx = shared ? 0 : e;
-  const int F = G.f, kc = F / kChunk;
-  const int64_t slot0 = static_cast<int64_t>(mt) * kc * kTileRows;
-  const uint32_t abytes = kc * kTileRows * 16, sbytes = kc * kTileRows * 4, gbytes = kc * kTileRows * 8;
-  const uint32_t hbytes = F * 2, mbytes = F / 32 * 4, fbytes = a.ws.hfs * 4;
-  const int fs = a.ws.fmax / 32;
-  fence_proxy_async_smem();
-  mbar_arrive_expect_tx(bar, abytes + sbytes + (FMT == MOE_FMT_CB35_32 ? gbytes : 0) + ntok * (hbytes + mbytes + fbytes));
-  const int64_t mat = static_cast<int64_t>(eidx) * 3 + 2;
-  bulk_g2s(v.w.a0, G.a + mat * G.a_mat + slot0 * 16, abytes, bar);
-  bulk_g2s(v.w.s0, G.s + mat * G.s_mat + slot0, sbytes, bar);
-  if (FMT == MOE_FMT_CB35_32) bulk_g2s(v.w.g0, G.g + mat * G.g_mat + slot0, gbytes, bar);
-  for (int i = 0; i < ntok; ++i) {
-    const int64_t row = static_cast<int64_t>(u) * kDecodeMaxTokens + i;
-    bulk_g2s(v.xq + i * F, a.ws.hq + row * a.ws.fmax, hbytes, bar);
-    bulk_g2s(v.msum + i * 2 * kc, a.ws.hsum + row * fs, mbytes, bar);
-    bulk_g2s(v.fac + i * a.ws.hfs, a.ws.hfac + row * a.ws.hfs, fbytes, bar);
-  }
-}
-
-template <int FMT, int NST>
-__global__ void __launch_bounds__(128, MOE_GEMV_MIN_BLOCKS) k_down(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int D = a.sh.d, TD = D / kTileRows;
-  const int kcmax = a.ws.fmax / kChunk;
-  const PersistPlan P = persist_plan(FMT, 1, kcmax, a.ws.hfs, a.ws.umax, NST);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-  TaskTable tt{reinterpret_cast<int *>(smem + P.table), a.ws.umax};
-  // stage views: per-expert kc differs (shared vs routed); plane offsets use the maximum
-  const StageView sv[2] = {stage_view(smem + P.stage0, P.st, kcmax), stage_view(smem + P.stage1, P.st, kcmax)};
-  uint32_t *tab = reinterpret_cast<uint32_t *>(smem + P.tab);
-  if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    fence_barrier_init();
-  }
-  if (FMT == MOE_FMT_CB35_32) load_grid_table(a.grid, tab);
-  if (!load_table(a, tt)) return;
-  const int n_tasks = tt.n_active() * TD;
-  int task = blockIdx.x;
-  if (task >= n_tasks) return;
-  if (threadIdx.x == 0) down_issue<FMT>(a, tt, task / TD, task % TD, sv[0], &bars[0]);
-  uint32_t ph[2] = {0u, 0u};
-  for (int it = 0; task < n_tasks; ++it, task += gridDim.x) {
-    const int cur = NST > 1 ? (it & 1) : 0;
-    const int next = task + gridDim.x;
-    if (NST > 1 && threadIdx.x == 0 && next < n_tasks)
-      down_issue<FMT>(a, tt, next / TD, next % TD, sv[cur ^ 1], &bars[cur ^ 1]);
-    if (!wait_stage(a, &bars[cur], ph[cur], &bars[cur ^ 1], ph[cur ^ 1], NST > 1 && next < n_tasks)) return;
-    ph[cur] ^= 1u;
-    const int u = task / TD, mt = task % TD;
-    const int e = tt.expert(u), ntok = tt.ntok(u);
-    const int F = (a.sh.n_shared && e == a.sh.e) ? a.L.shared.f : a.L.routed.f;
-    const int kc = F / kChunk;
-    const StageView &v = sv[cur];
-    float acc[2][kDecodeMaxTokens];
-#pragma unroll
-    for (int t = 0; t < kDecodeMaxTokens; ++t) acc[0][t] = acc[1][t] = 0.f;
-    gemv_dispatch<FMT, 1>(ntok, v.w, kc, v.xq, v.msum, tab, v.fac, a.ws.hfs, 1, acc);
-    const int row = mt * kTileRows + threadIdx.x;
-#pragma unroll
-    for (int t = 0; t < kDecodeMaxTokens; ++t)
-      if (t < ntok) a.ws.o[(static_cast<int64_t>(u) * kDecodeMaxTokens + t) * D + row] = acc[0][t];
-    __syncthreads();  // stage `cur` is refilled by the next issue
-    if (NST == 1 && threadIdx.x == 0 && next < n_tasks) down_issue<FMT>(a, tt, next / TD, next % TD, sv[0], &bars[0]);
+    griddep_wait();
+    if (threadIdx.x == 0) griddep_launch();
+    consumer<FMT, GU>(a, smem, P, H);
   }
 }
 
 // ------------------------------------------------------------------------------------------
 // combine: y[t] = sum_j w_tj o[slot(t, j)] + o_shared[t] (+ x[t]), slots in descending-logit
-// order, one thread per output element; every load of a thread is issued before the sum.
+// order.  CTA = (token, 128 columns); every load of a thread is issued before the sum.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_combine(DecodeArgs a) {
+constexpr int kCombineThreads = 128;  // d_model is a multiple of 128
+__global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
+  __shared__ int s_pos[kMaxTopK];
+  __shared__ float s_w[kMaxTopK];
   const int D = a.sh.d, K = a.sh.k;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= static_cast<int64_t>(a.n) * D) return;
-  const int t = static_cast<int>(i / D), d = static_cast<int>(i % D);
-  int pos[kMaxTopK];
-  float w[kMaxTopK], v[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    if (j < K) {
-      pos[j] = __ldcg(a.ws.slotpos + t * K + j);
-      w[j] = __ldcg(a.ws.route_w + t * K + j);
-    }
+  const int cpt = D / kCombineThreads;  // CTAs per token
+  const int t = blockIdx.x / cpt, d = (blockIdx.x - t * cpt) * kCombineThreads + threadIdx.x;
+  griddep_wait();
+  griddep_launch();
+  if (threadIdx.x < K) {
+    s_pos[threadIdx.x] = __ldcg(a.ws.slotpos + t * K + threadIdx.x);
+    s_w[threadIdx.x] = __ldcg(a.ws.route_w + t * K + threadIdx.x);
   }
+  const int64_t i = static_cast<int64_t>(t) * D + d;
   const float xs = a.residual ? load_act(a.x, i, a.x_bf16) : 0.f;
-  const float sh = a.sh.n_shared ? __ldcg(a.ws.o + static_cast<int64_t>(t) * D + d) : 0.f;
+  const float sh = a.sh.n_shared ? __ldcg(a.ws.o + i) : 0.f;  // u = 0 serves token t in slot t
+  __syncthreads();
+  float v[kMaxTopK];
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j)
-    if (j < K) v[j] = __ldcg(a.ws.o + static_cast<int64_t>(pos[j]) * D + d);
+    if (j < K) v[j] = __ldcg(a.ws.o + static_cast<int64_t>(s_pos[j]) * D + d);
   float y = 0.f;
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j)
-    if (j < K) y = fmaf(w[j], v[j], y);
+    if (j < K) y = fmaf(s_w[j], v[j], y);
   y += sh;
   if (a.residual) y = xs + y;
   if (a.y_bf16)
@@ -922,10 +1220,8 @@ __global__ void __launch_bounds__(256) k_combine(DecodeArgs a) {
 // ------------------------------------------------------------------------------------------
 // host launcher
 // ------------------------------------------------------------------------------------------
-static int route_smem_bytes(const DecodeArgs &a) {
-  const int xbytes = a.n * a.sh.d * 4;
-  const int tbytes = 2 * a.sh.e * 4 + (a.sh.e > 1024 ? a.n * a.sh.e * 4 : 0);
-  return xbytes > tbytes ? xbytes : tbytes;
+int route_smem_bytes(int n_experts) {
+  return 2 * n_experts * 4 + (n_experts > 1024 ? kDecodeMaxTokens * n_experts * 4 : 0);
 }
 
 // Under stream capture the records are made external, so that the CUDA graph records the
@@ -940,9 +1236,34 @@ static inline void rec(const DecodeArgs &a, int kind, int end, cudaStream_t st) 
     cudaEventRecord(a.ev[2 * kind + end], st);
 }
 
-// Allow every GEMV kernel the largest dynamic shared memory it can ask for (done once at
-// handle creation, so that launches need no attribute calls, e.g. under stream capture).
+// Programmatic dependent launch of the decode kernels (MOE_DECODE_PDL=0 in the environment
+// turns it off).
+static bool g_pdl = true;
+
+// Launch with programmatic stream serialization: the kernel may begin while the previous kernel
+// in the stream finishes; every decode kernel calls griddep_wait before it reads that kernel's
+// results.
+template <typename... P>
+static cudaError_t launch_pdl(void (*kernel)(P...), int grid, int block, int smem, cudaStream_t st,
+                              const DecodeArgs &a) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+// Allow every kernel the largest dynamic shared memory it can ask for (done once at handle
+// creation, so that launches need no attribute calls, e.g. under stream capture).
 cudaError_t configure_decode_kernels() {
+  const char *pdl = getenv("MOE_DECODE_PDL");
+  g_pdl = !(pdl && pdl[0] == '0');
   int dev = 0, max_optin = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -950,10 +1271,10 @@ cudaError_t configure_decode_kernels() {
   if (e != cudaSuccess) return e;
   const void *ks[] = {(const void *)k_route<true>,
                       (const void *)k_route<false>,
-                      (const void *)k_gateup<MOE_FMT_Q2_32, kDecodeStages>,
-                      (const void *)k_gateup<MOE_FMT_CB35_32, kDecodeStages>,
-                      (const void *)k_down<MOE_FMT_Q2_32, kDecodeStages>,
-                      (const void *)k_down<MOE_FMT_CB35_32, kDecodeStages>};
+                      (const void *)k_gemv<MOE_FMT_Q2_32, true>,
+                      (const void *)k_gemv<MOE_FMT_CB35_32, true>,
+                      (const void *)k_gemv<MOE_FMT_Q2_32, false>,
+                      (const void *)k_gemv<MOE_FMT_CB35_32, false>};
   for (const void *k : ks) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, k);
@@ -965,32 +1286,32 @@ cudaError_t configure_decode_kernels() {
   return cudaSuccess;
 }
 
-cudaError_t decode_grid_sizes(int fmt, int d, int splits, int fmax, int umax, int n_shared, int f, int f_shared,
-                              int *grid_gu, int *grid_down) {
-  const int Ts = n_shared ? f_shared / kTileRows : 0, Tr = f / kTileRows;
-  *grid_gu = Ts * splits + (umax - n_shared) * Tr * splits;
-  *grid_down = umax * (d / kTileRows);
-  if (kDecodeStages == 1) return cudaSuccess;
+static int gemv_smem(int fmt, bool gu, int umax) {
+  return ring_plan(fmt, gu ? 2 : 1, gu ? kGuStageChunks : kDnStageChunks, umax).total;
+}
+
+// Persistent grids: SMs x resident CTAs of each GEMV kernel; min_streams = 2 x SMs.
+cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gu, int *grid_dn, int *min_streams) {
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const int sm_gu = persist_plan(fmt, 2, d / kChunk / splits, pad4(splits), umax, kDecodeStages).total;
-  const int sm_dn = persist_plan(fmt, 1, fmax / kChunk, pad4(fmax / kTileRows), umax, kDecodeStages).total;
   int occ_gu = 0, occ_dn = 0;
+  const int sg = gemv_smem(fmt, true, umax), sd = gemv_smem(fmt, false, umax);
   if (fmt == MOE_FMT_Q2_32) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_gu, k_gateup<MOE_FMT_Q2_32, kDecodeStages>, kTileRows, sm_gu);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_gu, k_gemv<MOE_FMT_Q2_32, true>, kGemvThreads, sg);
     if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_dn, k_down<MOE_FMT_Q2_32, kDecodeStages>, kTileRows, sm_dn);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_dn, k_gemv<MOE_FMT_Q2_32, false>, kGemvThreads, sd);
   } else {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_gu, k_gateup<MOE_FMT_CB35_32, kDecodeStages>, kTileRows, sm_gu);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_gu, k_gemv<MOE_FMT_CB35_32, true>, kGemvThreads, sg);
     if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_dn, k_down<MOE_FMT_CB35_32, kDecodeStages>, kTileRows, sm_dn);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_dn, k_gemv<MOE_FMT_CB35_32, false>, kGemvThreads, sd);
   }
   if (e != cudaSuccess) return e;
   if (occ_gu < 1 || occ_dn < 1) return cudaErrorInvalidConfiguration;
-  if (nsm * occ_gu < *grid_gu) *grid_gu = nsm * occ_gu;
-  if (nsm * occ_dn < *grid_down) *grid_down = nsm * occ_dn;
+  *grid_gu = nsm * occ_gu;
+  *grid_dn = nsm * occ_dn;
+  *min_streams = 2 * nsm;
   return cudaSuccess;
 }
 
@@ -998,41 +1319,33 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
   cudaError_t err;
   // 1. router + input quantisation + top-k + tables
   {
-    int grid = (a.sh.e + kRouteWarps - 1) / kRouteWarps;
-    if (grid < a.n * a.ws.splits) grid = a.n * a.ws.splits;
-    const int sm = route_smem_bytes(a);
+    const int ngrp = (a.sh.e + kRouteExperts - 1) / kRouteExperts;
+    const int grid = ngrp * (a.sh.d / a.ws.rk_cols);
+    const int sm = route_smem_bytes(a.sh.e);
     rec(a, kProfRoute, 0, st);
-    if (a.sh.router_bf16)
-      k_route<true><<<grid, kRouteThreads, sm, st>>>(a);
-    else
-      k_route<false><<<grid, kRouteThreads, sm, st>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = a.sh.router_bf16 ? launch_pdl(k_route<true>, grid, kRouteThreads, sm, st, a)
+                           : launch_pdl(k_route<false>, grid, kRouteThreads, sm, st, a);
+    if (err != cudaSuccess) return err;
     rec(a, kProfRoute, 1, st);
   }
-  // 2. gate/up (persistent)
+  // 2. gate/up + SwiGLU (persistent)
   {
-    const int kc = a.sh.d / kChunk / a.ws.splits;
-    const int sm = persist_plan(a.sh.fmt, 2, kc, pad4(a.ws.splits), a.ws.umax, kDecodeStages).total;
+    const int sm = gemv_smem(a.sh.fmt, true, a.ws.umax);
     rec(a, kProfGateUp, 0, st);
-    if (a.sh.fmt == MOE_FMT_Q2_32)
-      k_gateup<MOE_FMT_Q2_32, kDecodeStages><<<a.ws.grid_gu, kTileRows, sm, st>>>(a);
-    else
-      k_gateup<MOE_FMT_CB35_32, kDecodeStages><<<a.ws.grid_gu, kTileRows, sm, st>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = a.sh.fmt == MOE_FMT_Q2_32 ? launch_pdl(k_gemv<MOE_FMT_Q2_32, true>, a.ws.grid_gu, kGemvThreads, sm, st, a)
+                                    : launch_pdl(k_gemv<MOE_FMT_CB35_32, true>, a.ws.grid_gu, kGemvThreads, sm, st, a);
+    if (err != cudaSuccess) return err;
     rec(a, kProfGateUp, 1, st);
   }
-  // 3. down (persistent) + combine
+  // 3. down + combine (persistent)
   {
-    const int sm = persist_plan(a.sh.fmt, 1, a.ws.fmax / kChunk, a.ws.hfs, a.ws.umax, kDecodeStages).total;
+    const int sm = gemv_smem(a.sh.fmt, false, a.ws.umax);
     rec(a, kProfDown, 0, st);
-    if (a.sh.fmt == MOE_FMT_Q2_32)
-      k_down<MOE_FMT_Q2_32, kDecodeStages><<<a.ws.grid_down, kTileRows, sm, st>>>(a);
-    else
-      k_down<MOE_FMT_CB35_32, kDecodeStages><<<a.ws.grid_down, kTileRows, sm, st>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    const int64_t outs = static_cast<int64_t>(a.n) * a.sh.d;
-    k_combine<<<static_cast<unsigned>((outs + 255) / 256), 256, 0, st>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = a.sh.fmt == MOE_FMT_Q2_32 ? launch_pdl(k_gemv<MOE_FMT_Q2_32, false>, a.ws.grid_dn, kGemvThreads, sm, st, a)
+                                    : launch_pdl(k_gemv<MOE_FMT_CB35_32, false>, a.ws.grid_dn, kGemvThreads, sm, st, a);
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(k_combine, a.n * (a.sh.d / kCombineThreads), kCombineThreads, 0, st, a);
+    if (err != cudaSuccess) return err;
     rec(a, kProfDown, 1, st);
   }
   return cudaSuccess;

@@ -65,37 +65,57 @@ struct Shape {
   int router_bf16;
 };
 
+// GEMV input of one token over one 64-column chunk (the layer input x for gate/up, the SwiGLU
+// output h for down): int16 fixed point, the exact sums of its two 32-element blocks and the
+// power-of-two factor of the chunk's 128-column group (with the 1/2 of the Q2 block value folded
+// in).  Records of consecutive chunks of a token are contiguous, so a run of chunks is one bulk
+// copy.
+struct ActRec {
+  int16_t x[64];
+  int32_t m[2];
+  float f;
+  uint32_t pad;
+};
+static_assert(sizeof(ActRec) == 144, "ActRec is 9 x 16 bytes");
+
 // Decode workspace (n <= 8 tokens).  u indexes active experts: u = 0 is the shared expert
-// when there is one, routed active experts follow in ascending expert id.  Activations enter
-// the GEMVs as int16 fixed point with a power-of-two factor: the layer input per (token,
-// K-split) (written by the router kernel), the SwiGLU output h per (row, 128-row tile of F)
-// (written where h is produced); each comes with its 32-element block sums.
+// when there is one, routed active experts follow in ascending expert id.  A GEMV "unit" is one
+// 128-row tile of one active expert's matrix (pair); its K range is cut into fixed segments of
+// 2 or 4 chunks whose fp32 sums are added in segment order, whether one CTA runs the whole
+// unit or several CTAs each take a run of segments (then the segment sums pass through the
+// partial buffers), so results do not depend on how the work was split.
 struct DecodeWs {
+  float *logit_part;    // [ks][8][E] router sums per K slice
   float *logits;        // [8][E]
   int *route_idx;       // [8][k]
   float *route_w;       // [8][k]
   int *slotpos;         // [8][k]: u * 8 + i (i = position of the token in expert u's list)
-  int *n_active;        // [1]
-  int *act_expert;      // [umax]: expert id, E for the shared expert
-  int *act_ntok;        // [umax]
-  int *act_tok;         // [umax][8]
-  int16_t *xq;          // [8][D]
-  int *xsum;            // [8][D/32]
-  float *xfac;          // [8][pad4(splits)]
-  int16_t *hq;          // [umax * 8][fmax]
-  int *hsum;            // [umax * 8][fmax/32]
-  float *hfac;          // [umax * 8][hfs]
-  float *gu_part;       // [umax][tmax][splits][2][8][128] gate/up partial sums
+  // Task table of the GEMV kernels, written by the router kernel: a header
+  // [n_active, gate/up tasks, down pieces per output tile, 0] and one 16-int row per active
+  // expert u: [expert (E = shared), ntok, tokens 0..7, first gate/up task, gate/up split,
+  // first down piece, down split, 0, 0]; a split packs run length | pieces << 8 |
+  // chunks per segment << 16 | segments << 20.
+  int *task_tab;        // [4 + umax * 16]
+  ActRec *xrec;         // [8][D/64]
+  ActRec *hrec;         // [umax][8][fmax/64]
+  float *gu_part;       // [umax][tmax][gu_nseg][2][8][128] gate/up segment sums
+  float *dn_part;       // [umax][D/128][dn_nseg][8][128]  down segment sums
   float *o;             // [umax * 8][D] expert outputs (unweighted)
   unsigned *route_ticket;   // [1]
+  unsigned *group_ticket;   // [ceil(E/32)]
   unsigned *gu_ticket;      // [umax][tmax]
+  unsigned *dn_ticket;      // [umax][D/128]
+  unsigned *counters;       // [2] work queues of the gate/up and down kernels
   int umax;
   int tmax;             // max(F, F_shared) / 128
   int fmax;
-  int splits;           // K-splits of the gate/up reduction (d_model / splits columns per CTA)
-  int hfs;              // row stride of hfac: tmax rounded up to a multiple of 4
-  int grid_gu;          // persistent grid of k_gateup / k_down
-  int grid_down;
+  int rk_cols;          // router: d_model columns per CTA (128 or 256)
+  int gu_seg;           // gate/up: chunks per K segment (2 or 4)
+  int gu_nseg;          // gate/up: K segments (d_model / 64 / gu_seg)
+  int dn_nseg;          // down: most K segments of any expert
+  int grid_gu;          // persistent grids of the GEMV kernels
+  int grid_dn;
+  int min_streams;      // pieces wanted in flight (about two per SM)
 };
 
 // ------------------------------------------------------------------------------------------
@@ -103,6 +123,24 @@ struct DecodeWs {
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory loads by 32-bit shared address (ld.shared, never a generic load); volatile, so
+// they stay after the barrier waits that order them.
+__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
@@ -148,6 +186,25 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// L2 policy for data read once (the weight blocks): evict first, so that a pass over the
+// expert blocks does not push the small, reused tensors (activations, routing tables, partial
+// sums) and the kernels' code out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// bulk_g2s with an L2 cache policy
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // Bounded wait on an mbarrier phase.  Returns false when `limit` clock cycles pass first.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -161,6 +218,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 // Waits for copies a CTA issued before it gives up: a CTA must not exit while a bulk copy
 // still writes its shared memory.  About two seconds at B200 clocks.
 constexpr uint64_t kDrainLimit = 4000000000ull;
+
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while the previous kernel of the stream still runs.  Before griddep_wait it may only
+// touch data that the previous kernels do not write; griddep_wait returns once they have
+// completed and their writes are visible.  griddep_launch lets the next kernel start early.  Both
+// are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void flag_error(uint32_t *err, uint32_t bit) {
   if (err) atomicOr(err, bit);
@@ -211,8 +276,8 @@ constexpr int kProfDown = 2;      // down GEMV or GEMM + combine
 constexpr int kProfKinds = 3;
 
 cudaError_t configure_decode_kernels();
-cudaError_t decode_grid_sizes(int fmt, int d, int splits, int fmax, int umax, int n_shared, int f, int f_shared,
-                              int *grid_gu, int *grid_down);
+cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gu, int *grid_dn, int *min_streams);
+int route_smem_bytes(int n_experts);
 cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_wait_test(unsigned *never_set, uint32_t *err, uint64_t spin_limit, cudaStream_t st);
 

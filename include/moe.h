@@ -136,10 +136,12 @@ const char *moe_last_error(const moe_handle *h);
 uint64_t moe_device_bytes(const moe_handle *h);
 
 /* Per-kernel CUDA-event timing.  While enabled (on != 0), every forward call records an event
- * pair on its stream around the launches of each selected kernel class (bit k of `on` selects
- * class k; such events are captured into a CUDA graph like the kernels).  moe_profile_read sums the durations recorded by the most recent call for one
- * kernel class -- 0: router + top-k (+ grouping), 1: gate/up + SwiGLU, 2: down + combine --
- * and returns how many launches contributed.  It waits for those events to complete. */
+ * pair on its stream around the launches of each selected kernel class of each layer it runs
+ * (bit k of `on` selects class k; such events are captured into a CUDA graph like the kernels).
+ * moe_profile_read sums, over the layers run since profiling was (re-)enabled, the durations
+ * recorded by the latest call that ran each layer, for one kernel class -- 0: router + top-k
+ * (+ grouping), 1: gate/up + SwiGLU, 2: down + combine -- and returns how many layers
+ * contributed.  It waits for those events to complete. */
 moe_status moe_profile_enable(moe_handle *h, int32_t on);
 moe_status moe_profile_read(moe_handle *h, int32_t kind, float *total_ms, int32_t *launches);
 
