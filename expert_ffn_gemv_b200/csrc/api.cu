@@ -141,8 +141,8 @@ void plan_workspace(moe_handle *h, Carve &c) {
   w.o = c.take<float>(hrows * D);
   w.route_ticket = c.take<unsigned>(1);
   w.group_ticket = c.take<unsigned>(ngrp);
-  w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax);
-  w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td);
+  w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * 4);  // x token groups of a unit
+  w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td * 4);
   w.counters = c.take<unsigned>(2);
   const uint64_t nt = static_cast<uint64_t>(g.max_tokens) * D;
   h->res[0] = c.take<float>(nt);
@@ -162,8 +162,8 @@ moe_status check_device_error(moe_handle *h, cudaStream_t st) {
   const int td = h->cfg.d_model / kTileRows;
   cudaMemsetAsync(w.route_ticket, 0, sizeof(unsigned), st);
   cudaMemsetAsync(w.group_ticket, 0, sizeof(unsigned) * ((h->cfg.n_experts + 31) / 32), st);
-  cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax, st);
-  cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td, st);
+  cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax * 4, st);
+  cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td * 4, st);
   cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * 2, st);
   if (e & kErrTimeout) return fail(h, MOE_ERR_TIMEOUT, "a device-side bounded wait ran out");
   return fail(h, MOE_ERR_DEVICE_FAULT, "a device-side check found an invalid routing index");

@@ -40,18 +40,30 @@ constexpr int kConsWarps = kTileRows / 32;      // consumer warps: thread = row 
 constexpr int kGemvThreads = kTileRows + 32;    // + one producer warp
 constexpr int kRing = 4;                        // most stages of the bulk-copy ring
 #ifndef MOE_GEMV_MIN_BLOCKS
-#define MOE_GEMV_MIN_BLOCKS 3                   // resident CTAs per SM the register budget allows
+#define MOE_GEMV_MIN_BLOCKS 4                   // resident CTAs per SM the register budget allows
 #endif
 #ifndef MOE_GEMV_UNROLL
 #define MOE_GEMV_UNROLL 1                       // chunks of a stage in flight per iteration
 #endif
 constexpr int kGemvUnroll = MOE_GEMV_UNROLL;
+#ifndef MOE_STREAMS_PER_SM
+#define MOE_STREAMS_PER_SM 6                    // GEMV pieces wanted in flight per SM (K split when fewer)
+#endif
 // ring depth: 4 stages for Q2; 3 for CB35, whose stages and grid table are larger, so that two
 // CTAs fit on an SM
 __host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_CB35_32 ? 3 : 4; }
 constexpr int kGuStageChunks = 2;               // gate/up: chunks per stage
 constexpr int kDnStageChunks = 4;               // down: chunks per stage (one K segment)
 constexpr int kPartStride = kDecodeMaxTokens * kTileRows;  // floats per (segment, matrix)
+
+// Q2 block arithmetic.  A block's value is sum_i (q_i - 1.5) m_i = (2S - 3M) / 2 with S = sum q_i m_i
+// and M = sum m_i.  The codes are taken from their words by one mask each, without the shift,
+// so group kk (bits 2kk, 2kk+1 of every byte) enters dp2a as 4^kk q; the four group sums are
+// recombined as 64 S = ((4 A0 + A1) 4 + A2) 4 + A3, and 64 (2S - 3M) = 2 (64 S) + (-192 M) is
+// exact in int32 and in fp32 (a multiple of 64 below 2^30).  Records therefore carry -192 M
+// and the activation factor times (1/2) / 64.
+constexpr int kQ2SumMul = -192;
+constexpr float kQ2Factor = 0.5f / 64.0f;
 
 __device__ __forceinline__ float load_act(const void *x, int64_t i, int bf16) {
   if (bf16) return __bfloat162float(static_cast<const __nv_bfloat16 *>(x)[i]);
@@ -130,12 +142,12 @@ __device__ __forceinline__ void softmax_store(const DecodeArgs &a, int t, int la
 template <int VPL>
 __device__ __forceinline__ void topk_regs(const DecodeArgs &a, int t, int lane, int *s_idx) {
   const int E = a.sh.e, K = a.sh.k;
+  float lv[VPL];  // all loads first (in-range index), then the keys
+#pragma unroll
+  for (int q = 0; q < VPL; ++q) lv[q] = __ldcg(a.ws.logits + t * E + min(lane + 32 * q, E - 1));
   uint32_t key[VPL];
 #pragma unroll
-  for (int q = 0; q < VPL; ++q) {
-    const int i = lane + 32 * q;
-    key[q] = i < E ? order_key(__ldcg(a.ws.logits + t * E + i)) : 0u;
-  }
+  for (int q = 0; q < VPL; ++q) key[q] = lane + 32 * q < E ? order_key(lv[q]) : 0u;
   float my_l = 0.f, l0 = 0.f;
   int my_i = 0;
   for (int j = 0; j < K; ++j) {
@@ -198,22 +210,29 @@ __device__ __forceinline__ void topk_smem(const DecodeArgs &a, int t, int lane, 
   softmax_store(a, t, lane, my_l, l0, my_i);
 }
 
-// Pieces per unit: about min_streams pieces in flight over the call; units with four or more
-// tokens (several times the arithmetic per byte) are split up to eight ways.  Returns the run
-// length in segments.
-__device__ __forceinline__ int piece_run(int nseg, int units_total, int ntok, int min_streams) {
+// Pieces per unit: K is cut only when there are fewer units than about min_streams (e.g. one
+// token's ~11 experts), so that enough pieces are in flight.  Returns the run length in segments.
+__device__ __forceinline__ int piece_run(int nseg, int units_total, int min_streams) {
   int p = (min_streams + units_total - 1) / units_total;
-  if (ntok >= 4) p = max(p, 8);
   p = min(max(p, 1), nseg);
   return (nseg + p - 1) / p;
 }
 
+// Token groups of an active expert: an expert serving three or more tokens is cut into groups of
+// at most two tokens, each a unit of its own over the whole K (the weights are read once per
+// group), which keeps every unit's arithmetic within about 1.6 times that of a one-token unit.
+constexpr int kTokGroup = 2;
+constexpr int kMaxTokGroups = kDecodeMaxTokens / kTokGroup;
+constexpr int kUnitTok = kTokGroup;  // tokens of one GEMV unit (at most)
+__host__ __device__ inline int tok_groups(int ntok) { return ntok >= 3 ? (ntok + kTokGroup - 1) / kTokGroup : 1; }
+__host__ __device__ inline int tok_group_size(int ntok) { return ntok >= 3 ? kTokGroup : ntok; }
+
 // Split of one GEMV unit whose K has nc chunks: K segments of 4 (else 2) chunks, cut into
 // pieces of `len` segments.  Returns the packed split; `pieces` the number of pieces.
-__device__ __forceinline__ int unit_split(int nc, int units_total, int ntok, int min_streams, int &pieces) {
+__device__ __forceinline__ int unit_split(int nc, int units_total, int min_streams, int &pieces) {
   const int seg = nc % 4 == 0 ? 4 : 2;
   const int nseg = nc / seg;
-  const int len = piece_run(nseg, units_total, ntok, min_streams);
+  const int len = piece_run(nseg, units_total, min_streams);
   pieces = (nseg + len - 1) / len;
   return len | (pieces << 8) | (seg << 16) | (nseg << 20);
 }
@@ -230,6 +249,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
   __shared__ int s_idx[kDecodeMaxTokens * kMaxTopK];
   __shared__ int s_wsum[kRouteWarps];
   __shared__ int s_cnt[2][kMaxActive];
+  __shared__ int s_units[2];
   __shared__ int s_last;
   const int D = a.sh.d, E = a.sh.e, n = a.n;
   const int CK = a.ws.rk_cols, KS = D / CK;
@@ -298,9 +318,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       s += __shfl_xor_sync(0xffffffffu, s, 2);
       s += __shfl_xor_sync(0xffffffffu, s, 4);
-      if ((lane & 7) == 0) rec->m[(lane >> 3) & 1] = s;
+      if ((lane & 7) == 0) rec->m[(lane >> 3) & 1] = a.sh.fmt == MOE_FMT_Q2_32 ? kQ2SumMul * s : s;
       if ((lane & 15) == 0) {
-        rec->f = pow2f(-e) * (a.sh.fmt == MOE_FMT_Q2_32 ? 0.5f : 1.0f);
+        rec->f = pow2f(-e) * (a.sh.fmt == MOE_FMT_Q2_32 ? kQ2Factor : 1.0f);
         rec->pad = 0u;
       }
     }
@@ -417,30 +437,45 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
   for (int w = 0; w < kRouteWarps; ++w) total += s_wsum[w];
   const int na = ns + total;
   const int TD = D / kTileRows;
-  const int units_gu = ns * (a.L.shared.f / kTileRows) + total * (a.L.routed.f / kTileRows);
-  const int units_dn = na * TD;
   int *tt = a.ws.task_tab;
+  if (tid == 0) s_units[0] = s_units[1] = 0;
+  __syncthreads();
+  // pass 1: expert, tokens and token groups of each row; unit counts of the call
+  int ug = 0, ud = 0;
   for (int i = tid; i < E + ns; i += kRouteThreads) {
     const bool shared = i == E;
     uint32_t m = shared ? (n == 32 ? 0xFFFFFFFFu : (1u << n) - 1u) : tokmask[i];
     if (!shared && a.out_counts) a.out_counts[i] = __popc(m);
     if (!m) continue;
     const int u = shared ? 0 : ns + rank[i];
-    const int nt = __popc(m);
+    const int nt = __popc(m), ng = tok_groups(nt);
     const int F = shared ? a.L.shared.f : a.L.routed.f;
     int *row = tt + kTabHead + u * kTabInts;
     row[0] = i;
     row[1] = nt;
+    row[14] = ng;
     int c = 0;
     while (m) {
       row[2 + c++] = __ffs(m) - 1;
       m &= m - 1u;
     }
+    s_cnt[0][u] = F;   // d_ff of the row, for pass 2
+    s_cnt[1][u] = ng;
+    ug += (F / kTileRows) * ng;
+    ud += TD * ng;
+  }
+  if (ug) atomicAdd(&s_units[0], ug);
+  if (ud) atomicAdd(&s_units[1], ud);
+  __syncthreads();
+  // pass 2: K splits and task counts per row
+  for (int u = tid; u < na; u += kRouteThreads) {
+    const int F = s_cnt[0][u], ng = s_cnt[1][u];
+    int *row = tt + kTabHead + u * kTabInts;
     int pg, pd;
-    row[11] = unit_split(D / kChunk, units_gu, nt, a.ws.min_streams, pg);
-    row[13] = unit_split(F / kChunk, units_dn, nt, a.ws.min_streams, pd);
-    s_cnt[0][u] = (F / kTileRows) * pg;
-    s_cnt[1][u] = pd;
+    row[11] = unit_split(D / kChunk, s_units[0], a.ws.min_streams, pg);
+    row[13] = unit_split(F / kChunk, s_units[1], a.ws.min_streams, pd);
+    s_cnt[0][u] = (F / kTileRows) * ng * pg;
+    s_cnt[1][u] = ng * pd;
   }
   for (int p = tid; p < n * K; p += kRouteThreads) {
     const int t = p / K, ex = s_idx[p];
@@ -533,10 +568,33 @@ __device__ __forceinline__ int block_dot(const uint32_t (&q)[8], const int4 (&p)
   return s0 + s1;
 }
 
-// block value: Q2 sum (q - 1.5) m = (2S - 3M) / 2 (the 1/2 is in the activation factor); CB35: S
-template <int FMT>
-__device__ __forceinline__ float block_value(int S, int M) {
-  return FMT == MOE_FMT_Q2_32 ? static_cast<float>(2 * S - 3 * M) : static_cast<float>(S);
+// dp2a with signed 16-bit pairs (a) and unsigned bytes (b)
+__device__ __forceinline__ int dp2a_lo_su(int a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi_su(int a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// 64 x the Q2 block sum S = sum q_i m_i from the block's two code words, groups masked in place
+// (see kQ2SumMul); four accumulation chains, one per group.
+__device__ __forceinline__ int q2_block_dot64(uint32_t w0, uint32_t w1, const int4 (&p)[4]) {
+  const int pr[16] = {p[0].x, p[0].y, p[0].z, p[0].w, p[1].x, p[1].y, p[1].z, p[1].w,
+                      p[2].x, p[2].y, p[2].z, p[2].w, p[3].x, p[3].y, p[3].z, p[3].w};
+  int acc[4];
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint32_t m0 = w0 & (0x03030303u << (2 * kk)), m1 = w1 & (0x03030303u << (2 * kk));
+    int v = dp2a_lo_su(pr[2 * kk], m0, 0);
+    v = dp2a_hi_su(pr[2 * kk + 1], m0, v);
+    v = dp2a_lo_su(pr[8 + 2 * kk], m1, v);
+    acc[kk] = dp2a_hi_su(pr[9 + 2 * kk], m1, v);
+  }
+  return ((acc[0] * 4 + acc[1]) * 4 + acc[2]) * 4 + acc[3];
 }
 
 __host__ __device__ inline int align128(int v) { return (v + 127) & ~127; }
@@ -557,12 +615,14 @@ struct StageInfo {
   int seg;     // K segment of the stage
   int ntok;
   int nch;     // chunks in the stage
-  int flags;   // k* bits | pieces of the unit << 8 | K segments of the unit << 16
+  int flags;   // k* bits | pieces of the unit << 8 | K segments of the unit << 16 |
+               // first token slot of the unit's token group << 24
   int c0;      // first chunk of the stage
 };
 constexpr int kPieceStart = 1, kSegStart = 2, kSegEnd = 4, kPieceEnd = 8;
 __device__ __forceinline__ int info_pieces(int flags) { return (flags >> 8) & 0xFF; }
-__device__ __forceinline__ int info_nseg(int flags) { return flags >> 16; }
+__device__ __forceinline__ int info_nseg(int flags) { return (flags >> 16) & 0xFF; }
+__device__ __forceinline__ int info_tok0(int flags) { return flags >> 24; }
 
 struct RingHdr {
   uint64_t full[kRing];
@@ -572,8 +632,8 @@ struct RingHdr {
   int n_active;
   volatile int abort;
   int flag[2];
-  float wmax[2][kConsWarps][kDecodeMaxTokens];
-  float tot[2][kDecodeMaxTokens][kTileRows];  // running unit sums of an unsplit unit (thread = row)
+  float wmax[2][kConsWarps][kUnitTok];
+  float tot[2][kUnitTok][kTileRows];  // running unit sums of an unsplit unit (thread = row)
 };
 
 __host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax, int umax) {
@@ -589,7 +649,7 @@ __host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax, int uma
   p.g = so;
   if (fmt == MOE_FMT_CB35_32) so += align128(nr * cmax * kTileRows * 8);
   p.rec = so;
-  so += align128(kDecodeMaxTokens * cmax * static_cast<int>(sizeof(ActRec)));
+  so += align128(kUnitTok * cmax * static_cast<int>(sizeof(ActRec)));
   p.stage = so;
   off += ring_depth(fmt) * so;
   p.tab = off;
@@ -604,7 +664,7 @@ __host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax, int uma
 template <int FMT, int T0, int TN, int NR, int CMAX>
 __device__ __forceinline__ void chunk_tokens(const uint4 (&A)[NR], const float2 (&sc)[NR], const uint2 (&G)[NR],
                                              uint32_t rec, int c, uint32_t tab, int lane,
-                                             float (&acc)[2][kDecodeMaxTokens]) {
+                                             float (&acc)[2][kUnitTok]) {
   constexpr uint32_t kRec = sizeof(ActRec);
   float cacc[NR][TN];
 #pragma unroll
@@ -614,10 +674,12 @@ __device__ __forceinline__ void chunk_tokens(const uint4 (&A)[NR], const float2 
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
     uint32_t q[NR][8];
+    if (FMT == MOE_FMT_CB35_32) {
 #pragma unroll
-    for (int m = 0; m < NR; ++m) {
-      const uint32_t w0 = b ? A[m].z : A[m].x, w1 = b ? A[m].w : A[m].y;
-      unpack_block<FMT>(w0, w1, b ? G[m].y : G[m].x, tab, lane, q[m]);
+      for (int m = 0; m < NR; ++m) {
+        const uint32_t w0 = b ? A[m].z : A[m].x, w1 = b ? A[m].w : A[m].y;
+        unpack_block<FMT>(w0, w1, b ? G[m].y : G[m].x, tab, lane, q[m]);
+      }
     }
 #pragma unroll
     for (int t = 0; t < TN; ++t) {
@@ -629,8 +691,12 @@ __device__ __forceinline__ void chunk_tokens(const uint4 (&A)[NR], const float2 
       const int M = FMT == MOE_FMT_Q2_32 ? static_cast<int>(lds_u32(ra + offsetof(ActRec, m) + 4 * b)) : 0;
 #pragma unroll
       for (int m = 0; m < NR; ++m) {
-        const int S = block_dot(q[m], p);
-        cacc[m][t] = fmaf(block_value<FMT>(S, M), b ? sc[m].y : sc[m].x, cacc[m][t]);
+        float v;
+        if (FMT == MOE_FMT_Q2_32)  // 64 (2S - 3M); the 1/64 and 1/2 are in the factor
+          v = static_cast<float>(2 * q2_block_dot64(b ? A[m].z : A[m].x, b ? A[m].w : A[m].y, p) + M);
+        else
+          v = static_cast<float>(block_dot(q[m], p));
+        cacc[m][t] = fmaf(v, b ? sc[m].y : sc[m].x, cacc[m][t]);
       }
     }
   }
@@ -645,7 +711,7 @@ __device__ __forceinline__ void chunk_tokens(const uint4 (&A)[NR], const float2 
 // GEMV of NR matrices (1 or 2) over the nch chunks of one stage for tokens T0 .. T0+TN-1.
 template <int FMT, int T0, int TN, int NR, int CMAX>
 __device__ __forceinline__ void gemv_stage(const unsigned char *st, const RingPlan &P, int nch, uint32_t tab,
-                                           float (&acc)[2][kDecodeMaxTokens]) {
+                                           float (&acc)[2][kUnitTok]) {
   const int r = threadIdx.x, lane = r & 31;
   const uint32_t base = smem_u32(st);
   const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g, rec = base + P.rec;
@@ -666,24 +732,14 @@ __device__ __forceinline__ void gemv_stage(const unsigned char *st, const RingPl
   }
 }
 
-// Up to four tokens per pass over the stage (more tokens take a second pass, unpacking the
-// codes again), which keeps the loop's registers within three CTAs per SM.
+// One or two tokens (a unit serves at most kUnitTok tokens).
 template <int FMT, int NR, int CMAX>
 __device__ __forceinline__ void gemv_dispatch(int nt, const unsigned char *st, const RingPlan &P, int nch,
-                                              uint32_t tab, float (&acc)[2][kDecodeMaxTokens]) {
-  switch (nt < 4 ? nt : 4) {
-    case 1: gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc); break;
-    case 2: gemv_stage<FMT, 0, 2, NR, CMAX>(st, P, nch, tab, acc); break;
-    case 3: gemv_stage<FMT, 0, 3, NR, CMAX>(st, P, nch, tab, acc); break;
-    default: gemv_stage<FMT, 0, 4, NR, CMAX>(st, P, nch, tab, acc); break;
-  }
-  switch (nt) {
-    case 5: gemv_stage<FMT, 4, 1, NR, CMAX>(st, P, nch, tab, acc); break;
-    case 6: gemv_stage<FMT, 4, 2, NR, CMAX>(st, P, nch, tab, acc); break;
-    case 7: gemv_stage<FMT, 4, 3, NR, CMAX>(st, P, nch, tab, acc); break;
-    case 8: gemv_stage<FMT, 4, 4, NR, CMAX>(st, P, nch, tab, acc); break;
-    default: break;
-  }
+                                              uint32_t tab, float (&acc)[2][kUnitTok]) {
+  if (nt == 1)
+    gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc);
+  else
+    gemv_stage<FMT, 0, 2, NR, CMAX>(st, P, nch, tab, acc);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -742,10 +798,11 @@ __device__ __forceinline__ int producer_tables(const DecodeArgs &a, RingHdr *H, 
     if (!b) {
       const int F = e == E ? a.L.shared.f : a.L.routed.f;
       const int nc = (GU ? D : F) / kChunk;
-      const int pk = row[GU ? 11 : 13];
+      const int pk = row[GU ? 11 : 13], ng = row[14];
       const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
-      b = (seg != 2 && seg != 4) || nseg * seg != nc || len < 1 || len > nseg || pieces != (nseg + len - 1) / len;
-      const int cnt = GU ? (F / kTileRows) * pieces : pieces;
+      b = (seg != 2 && seg != 4) || nseg * seg != nc || len < 1 || len > nseg || pieces != (nseg + len - 1) / len ||
+          ng != tok_groups(nt);
+      const int cnt = GU ? (F / kTileRows) * ng * pieces : ng * pieces;
       const int base = row[GU ? 10 : 12];
       const int next = u + 1 < na ? row[kTabInts + (GU ? 10 : 12)] : total;
       b = b || base + cnt != next || (u == 0 && base != 0);
@@ -809,20 +866,28 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
     if (lane == 0) nxt = static_cast<int>(atomicAdd(ctr, 1u));  // fetched while this piece is issued
     int u, mt, piece;
     const int *tr = tb + kTabHead;
+    int grp;
     if (GU) {
       u = find_expert<true>(tb, na, task);
-      const int pieces = (tr[u * kTabInts + 11] >> 8) & 0xFF;
+      const int pieces = (tr[u * kTabInts + 11] >> 8) & 0xFF, ng = tr[u * kTabInts + 14];
       const int r = task - tr[u * kTabInts + 10];
-      mt = r / pieces;
-      piece = r - mt * pieces;
+      mt = r / (ng * pieces);
+      const int q = r - mt * ng * pieces;
+      grp = q / pieces;
+      piece = q - grp * pieces;
     } else {
       mt = task / per_mt;
       const int r = task - mt * per_mt;
       u = find_expert<false>(tb, na, r);
-      piece = r - tr[u * kTabInts + 12];
+      const int pieces = (tr[u * kTabInts + 13] >> 8) & 0xFF;
+      const int q = r - tr[u * kTabInts + 12];
+      grp = q / pieces;
+      piece = q - grp * pieces;
     }
     const int *row = tr + u * kTabInts;
-    const int e = row[0], ntok = row[1];
+    const int e = row[0];
+    const int gsz = tok_group_size(row[1]), tok0 = grp * gsz;
+    const int ntok = min(gsz, row[1] - tok0);  // tokens of this unit: slots tok0 .. tok0 + ntok - 1
     const int pk = row[GU ? 11 : 13];
     const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
     const bool shared = a.sh.n_shared && e == E;
@@ -847,7 +912,7 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
         in.nch = nch;
         in.flags = (c0 == cbeg ? kPieceStart : 0) | (c0 % seg == 0 ? kSegStart : 0) |
                    ((c0 + nch) % seg == 0 ? kSegEnd : 0) | (c0 + nch == cend ? kPieceEnd : 0) | (pieces << 8) |
-                   (nseg << 16);
+                   (nseg << 16) | (tok0 << 24);
         in.c0 = c0;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&H->full[slot], NR * wbytes + ntok * rbytes);
@@ -875,8 +940,8 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
       auto issue_records = [&](int sl, int cc0) {
         const int i = lane - NR * kPlanes;
         if (i >= 0 && i < ntok) {
-          const ActRec *src = GU ? a.ws.xrec + static_cast<int64_t>(row[2 + i]) * (D / kChunk) + cc0
-                                 : a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + i) * (a.ws.fmax / kChunk) + cc0;
+          const ActRec *src = GU ? a.ws.xrec + static_cast<int64_t>(row[2 + tok0 + i]) * (D / kChunk) + cc0
+                                 : a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + i) * (a.ws.fmax / kChunk) + cc0;
           bulk_g2s(smem + P.stage0 + sl * P.stage + P.rec + i * CMAX * static_cast<int>(sizeof(ActRec)), src,
                    min(sch, cend - cc0) * static_cast<uint32_t>(sizeof(ActRec)), &H->full[sl]);
         }
@@ -938,12 +1003,12 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
 // Sums of a split unit's segment partials in segment order (the last piece of the unit), row r:
 // tot[m][t] = sum_j part[j][m][t][r].  32 loads are in flight at a time.
 template <int NR>
-__device__ __forceinline__ void sum_segments(const float *part, int nseg, int ntok, float (&tot)[2][kDecodeMaxTokens]) {
+__device__ __forceinline__ void sum_segments(const float *part, int nseg, int ntok, float (&tot)[2][kUnitTok]) {
   const int r = threadIdx.x;
   constexpr int kSegStride = NR * kPartStride;
   constexpr int TPR = 2 / NR;  // tokens per round
 #pragma unroll
-  for (int t0 = 0; t0 < kDecodeMaxTokens; t0 += TPR) {
+  for (int t0 = 0; t0 < kUnitTok; t0 += TPR) {
     if (t0 < ntok) {
       float v[TPR][NR][16];
 #pragma unroll
@@ -997,29 +1062,30 @@ template <int FMT>
 __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in) {
   const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
   const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags);
-  const int nseg = info_nseg(in.flags);
-  float tot[2][kDecodeMaxTokens];
+  const int nseg = info_nseg(in.flags), tok0 = info_tok0(in.flags);
+  float tot[2][kUnitTok];
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxTokens; ++t)
+  for (int t = 0; t < kUnitTok; ++t)
     if (t < ntok) {
       tot[0][t] = H->tot[0][t][r];
       tot[1][t] = H->tot[1][t][r];
     }
   if (pieces > 1) {
-    unsigned *ticket = a.ws.gu_ticket + u * a.ws.tmax + mt;
+    unsigned *ticket = a.ws.gu_ticket + (u * a.ws.tmax + mt) * kMaxTokGroups + tok0 / kTokGroup;
     bool ok;
     const bool last = unit_ticket(a, H, cs, ticket, static_cast<unsigned>(pieces - 1), ok);
     if (!ok) return false;
     if (!last) return true;
-    sum_segments<2>(a.ws.gu_part + static_cast<int64_t>(u * a.ws.tmax + mt) * a.ws.gu_nseg * 2 * kPartStride, nseg,
+    sum_segments<2>(a.ws.gu_part + static_cast<int64_t>(u * a.ws.tmax + mt) * a.ws.gu_nseg * 2 * kPartStride +
+                        tok0 * kTileRows, nseg,
                     ntok, tot);
     if (r == 0) *ticket = 0u;
   }
   // SwiGLU, then h of each token quantised over the tile's 128 rows
   const int wb = cs.nwmax++ & 1;
-  float hv[kDecodeMaxTokens];
+  float hv[kUnitTok];
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxTokens; ++t) {
+  for (int t = 0; t < kUnitTok; ++t) {
     hv[t] = 0.f;
     if (t < ntok) {
       hv[t] = silu_f(tot[0][t]) * tot[1][t];
@@ -1032,21 +1098,21 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
   if (!cons_sync(H, cs.cph, a.spin_limit)) return false;
   const int fs = a.ws.fmax / kChunk;
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxTokens; ++t) {
+  for (int t = 0; t < kUnitTok; ++t) {
     if (t < ntok) {
       float mx = H->wmax[wb][0][t];
 #pragma unroll
       for (int w = 1; w < kConsWarps; ++w) mx = fmaxf(mx, H->wmax[wb][w][t]);
       const int e = fix16_exponent(mx);
       const int m = fix16(hv[t], pow2f(e));
-      ActRec *rec = a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + t) * fs + 2 * mt + (r >> 6);
+      ActRec *rec = a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + t) * fs + 2 * mt + (r >> 6);
       rec->x[r & 63] = static_cast<int16_t>(m);
       int sum = m;  // warp = 32 consecutive rows = one block of the down matrix's K
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) rec->m[warp & 1] = sum;
+      if (lane == 0) rec->m[warp & 1] = FMT == MOE_FMT_Q2_32 ? kQ2SumMul * sum : sum;
       if ((r & 63) == 0) {
-        rec->f = pow2f(-e) * (FMT == MOE_FMT_Q2_32 ? 0.5f : 1.0f);
+        rec->f = pow2f(-e) * (FMT == MOE_FMT_Q2_32 ? kQ2Factor : 1.0f);
         rec->pad = 0u;
       }
     }
@@ -1057,25 +1123,26 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
 __device__ __forceinline__ bool dn_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in) {
   const int r = threadIdx.x;
   const int D = a.sh.d, TD = D / kTileRows;
-  const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags);
-  float tot[2][kDecodeMaxTokens];
+  const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags), tok0 = info_tok0(in.flags);
+  float tot[2][kUnitTok];
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxTokens; ++t)
+  for (int t = 0; t < kUnitTok; ++t)
     if (t < ntok) tot[0][t] = H->tot[0][t][r];
   if (pieces > 1) {
-    unsigned *ticket = a.ws.dn_ticket + u * TD + mt;
+    unsigned *ticket = a.ws.dn_ticket + (u * TD + mt) * kMaxTokGroups + tok0 / kTokGroup;
     bool ok;
     const bool last = unit_ticket(a, H, cs, ticket, static_cast<unsigned>(pieces - 1), ok);
     if (!ok) return false;
     if (!last) return true;
     const int nseg = info_nseg(in.flags);
-    sum_segments<1>(a.ws.dn_part + static_cast<int64_t>(u * TD + mt) * a.ws.dn_nseg * kPartStride, nseg, ntok, tot);
+    sum_segments<1>(a.ws.dn_part + static_cast<int64_t>(u * TD + mt) * a.ws.dn_nseg * kPartStride + tok0 * kTileRows,
+                    nseg, ntok, tot);
     if (r == 0) *ticket = 0u;
   }
   const int row = mt * kTileRows + r;
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxTokens; ++t)
-    if (t < ntok) a.ws.o[(static_cast<int64_t>(u) * kDecodeMaxTokens + t) * D + row] = tot[0][t];
+  for (int t = 0; t < kUnitTok; ++t)
+    if (t < ntok) a.ws.o[(static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + t) * D + row] = tot[0][t];
   return true;
 }
 
@@ -1095,7 +1162,7 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
       return;
     }
   }
-  float seg[2][kDecodeMaxTokens];
+  float seg[2][kUnitTok];
   int slot = 0;
   uint32_t round = 0;
   for (;;) {
@@ -1110,13 +1177,13 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
 #pragma unroll
       for (int m = 0; m < NR; ++m)
 #pragma unroll
-        for (int t = 0; t < kDecodeMaxTokens; ++t) H->tot[m][t][r] = 0.f;
+        for (int t = 0; t < kUnitTok; ++t) H->tot[m][t][r] = 0.f;
     }
     if (in.flags & kSegStart) {
 #pragma unroll
       for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int t = 0; t < kDecodeMaxTokens; ++t) seg[m][t] = 0.f;
+        for (int t = 0; t < kUnitTok; ++t) seg[m][t] = 0.f;
     }
     gemv_dispatch<FMT, NR, CMAX>(in.ntok, smem + P.stage0 + slot * P.stage, P, in.nch, smem_u32(tab), seg);
     __syncwarp();
@@ -1130,13 +1197,13 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
 #pragma unroll
         for (int m = 0; m < NR; ++m)
 #pragma unroll
-          for (int t = 0; t < kDecodeMaxTokens; ++t)
-            if (t < in.ntok) part[m * kPartStride + t * kTileRows + r] = seg[m][t];
+          for (int t = 0; t < kUnitTok; ++t)
+            if (t < in.ntok) part[m * kPartStride + (info_tok0(in.flags) + t) * kTileRows + r] = seg[m][t];
       } else {
 #pragma unroll
         for (int m = 0; m < NR; ++m)
 #pragma unroll
-          for (int t = 0; t < kDecodeMaxTokens; ++t)
+          for (int t = 0; t < kUnitTok; ++t)
             if (t < in.ntok) H->tot[m][t][r] += seg[m][t];
       }
     }
@@ -1311,7 +1378,7 @@ cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gu, int *grid_dn, int
   if (occ_gu < 1 || occ_dn < 1) return cudaErrorInvalidConfiguration;
   *grid_gu = nsm * occ_gu;
   *grid_dn = nsm * occ_dn;
-  *min_streams = 2 * nsm;
+  *min_streams = MOE_STREAMS_PER_SM * nsm;
   return cudaSuccess;
 }
 

@@ -93,7 +93,7 @@ struct DecodeWs {
   // Task table of the GEMV kernels, written by the router kernel: a header
   // [n_active, gate/up tasks, down pieces per output tile, 0] and one 16-int row per active
   // expert u: [expert (E = shared), ntok, tokens 0..7, first gate/up task, gate/up split,
-  // first down piece, down split, 0, 0]; a split packs run length | pieces << 8 |
+  // first down piece, down split, token groups, 0]; a split packs run length | pieces << 8 |
   // chunks per segment << 16 | segments << 20.
   int *task_tab;        // [4 + umax * 16]
   ActRec *xrec;         // [8][D/64]
@@ -103,8 +103,8 @@ struct DecodeWs {
   float *o;             // [umax * 8][D] expert outputs (unweighted)
   unsigned *route_ticket;   // [1]
   unsigned *group_ticket;   // [ceil(E/32)]
-  unsigned *gu_ticket;      // [umax][tmax]
-  unsigned *dn_ticket;      // [umax][D/128]
+  unsigned *gu_ticket;      // [umax][tmax][4 token groups]
+  unsigned *dn_ticket;      // [umax][D/128][4 token groups]
   unsigned *counters;       // [2] work queues of the gate/up and down kernels
   int umax;
   int tmax;             // max(F, F_shared) / 128
