@@ -135,10 +135,33 @@ __device__ __forceinline__ void softmax_store(const DecodeArgs &a, int t, int la
   }
 }
 
-// Top-k of token t by one warp, logits in registers (lane l holds experts l + 32 q).  Each
-// round takes the largest key by a warp max-reduction and, among the lanes holding it, the
-// lowest expert index by a min-reduction: the order of repeated strict maxima, ties to the
-// lower index.
+// Largest key of a lane's VPL keys and its position (ties: the lower position), by a pairwise
+// tree over compile-time positions.
+template <int VPL>
+__device__ __forceinline__ void lane_argmax(const uint32_t (&key)[VPL], uint32_t &bk, int &bq) {
+  uint32_t k[VPL];
+  int q[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    k[i] = key[i];
+    q[i] = i;
+  }
+#pragma unroll
+  for (int s = 1; s < VPL; s <<= 1)
+#pragma unroll
+    for (int i = 0; i + s < VPL; i += 2 * s) {
+      const bool take = k[i + s] > k[i];
+      k[i] = take ? k[i + s] : k[i];
+      q[i] = take ? q[i + s] : q[i];
+    }
+  bk = k[0];
+  bq = q[0];
+}
+
+// Top-k of token t by one warp, logits in registers (lane l holds experts l + 32 q).  Each lane
+// keeps its best key; a round takes the largest by a warp max-reduction and, among the lanes
+// holding it, the lowest expert index by a min-reduction (the order of repeated strict maxima,
+// ties to the lower index); only the winning lane clears that key and rescans its own keys.
 template <int VPL>
 __device__ __forceinline__ void topk_regs(const DecodeArgs &a, int t, int lane, int *s_idx) {
   const int E = a.sh.e, K = a.sh.k;
@@ -148,29 +171,26 @@ __device__ __forceinline__ void topk_regs(const DecodeArgs &a, int t, int lane, 
   uint32_t key[VPL];
 #pragma unroll
   for (int q = 0; q < VPL; ++q) key[q] = lane + 32 * q < E ? order_key(lv[q]) : 0u;
+  uint32_t lb;
+  int lq;
+  lane_argmax<VPL>(key, lb, lq);
   float my_l = 0.f, l0 = 0.f;
   int my_i = 0;
   for (int j = 0; j < K; ++j) {
-    uint32_t lb = key[0];
-#pragma unroll
-    for (int q = 1; q < VPL; ++q) lb = max(lb, key[q]);
     const uint32_t m = __reduce_max_sync(0xffffffffu, lb);
-    int qm = 0;
-#pragma unroll
-    for (int q = VPL - 1; q >= 0; --q)
-      if (key[q] == m) qm = q;
-    int bi = __reduce_min_sync(0xffffffffu, lb == m ? lane + 32 * qm : INT_MAX);
+    int bi = __reduce_min_sync(0xffffffffu, lb == m ? lane + 32 * lq : INT_MAX);
     float bv = key_value(m);
     if (bi >= E || !(bv > -INFINITY)) {  // only non-finite logits left
       if (lane == 0) flag_error(a.err, kErrBadIndex);
       bi = j;
       bv = 0.f;
     }
-    // clear the winner by selects on every register (a conditional store with a data-dependent
-    // index would move key[] to local memory)
-    const int qb = (bi & 31) == lane ? bi >> 5 : -1;
+    if ((bi & 31) == lane) {  // the winner: clear the key (selects, not an indexed store), rescan
+      const int qb = bi >> 5;
 #pragma unroll
-    for (int q = 0; q < VPL; ++q) key[q] = q == qb ? 0u : key[q];
+      for (int q = 0; q < VPL; ++q) key[q] = q == qb ? 0u : key[q];
+      lane_argmax<VPL>(key, lb, lq);
+    }
     if (j == 0) l0 = bv;
     if (lane == j) { my_l = bv; my_i = bi; }
     if (lane == 0) s_idx[t * K + j] = bi;
@@ -221,7 +241,10 @@ __device__ __forceinline__ int piece_run(int nseg, int units_total, int min_stre
 // Token groups of an active expert: an expert serving three or more tokens is cut into groups of
 // at most two tokens, each a unit of its own over the whole K (the weights are read once per
 // group), which keeps every unit's arithmetic within about 1.6 times that of a one-token unit.
-constexpr int kTokGroup = 2;
+#ifndef MOE_TOK_GROUP
+#define MOE_TOK_GROUP 2
+#endif
+constexpr int kTokGroup = MOE_TOK_GROUP;
 constexpr int kMaxTokGroups = kDecodeMaxTokens / kTokGroup;
 constexpr int kUnitTok = kTokGroup;  // tokens of one GEMV unit (at most)
 __host__ __device__ inline int tok_groups(int ntok) { return ntok >= 3 ? (ntok + kTokGroup - 1) / kTokGroup : 1; }
@@ -393,9 +416,12 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
 
   const int K = a.sh.k;
   uint32_t *tokmask = reinterpret_cast<uint32_t *>(smem);  // [E]: bit t = token t chose the expert
-  int *rank = reinterpret_cast<int *>(tokmask + E);          // [E]
-  float *lg = reinterpret_cast<float *>(rank + E);           // [n][E] (more than 1,024 experts)
+  uint32_t *bitmap = tokmask + E;                          // [E/32]: active experts
+  int *wpre = reinterpret_cast<int *>(bitmap + kMaxExperts / 32);  // [E/32]: active experts before word w
+  float *lg = reinterpret_cast<float *>(wpre + kMaxExperts / 32);  // [n][E] (more than 1,024 experts)
+  const int nw = (E + 31) / 32;
   for (int i = tid; i < E; i += kRouteThreads) tokmask[i] = 0u;
+  for (int i = tid; i < nw; i += kRouteThreads) bitmap[i] = 0u;
   if (warp < n) {
     if (E <= 128) topk_regs<4>(a, warp, lane, s_idx);
     else if (E <= 256) topk_regs<8>(a, warp, lane, s_idx);
@@ -404,54 +430,49 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
     else topk_smem(a, warp, lane, lg + warp * E, s_idx);
   }
   __syncthreads();
-  for (int p = tid; p < n * K; p += kRouteThreads) atomicOr(tokmask + s_idx[p], 1u << (p / K));
-  __syncthreads();
-  // block-wide exclusive scan of (tokmask != 0) -> rank (ascending expert id)
-  {
-    const int per = (E + kRouteThreads - 1) / kRouteThreads;
-    const int lo = tid * per, hi = min(E, lo + per);
-    int local = 0;
-    for (int i = lo; i < hi; ++i) local += tokmask[i] != 0u;
-    int inc = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += v;
-    }
-    if (lane == 31) s_wsum[warp] = inc;
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += s_wsum[w];
-    int run = base + inc - local;
-    for (int i = lo; i < hi; ++i) {
-      rank[i] = run;
-      run += tokmask[i] != 0u;
-    }
-    __syncthreads();
+  for (int p = tid; p < n * K; p += kRouteThreads) {
+    const int ex = s_idx[p];
+    atomicOr(tokmask + ex, 1u << (p / K));
+    atomicOr(bitmap + (ex >> 5), 1u << (ex & 31));
   }
-  // active-expert rows of the task table (u = 0: the shared expert; routed experts follow in
-  // ascending id) and the token slots of the combine
-  const int ns = a.sh.n_shared;
-  int total = 0;
-#pragma unroll
-  for (int w = 0; w < kRouteWarps; ++w) total += s_wsum[w];
-  const int na = ns + total;
-  const int TD = D / kTileRows;
-  int *tt = a.ws.task_tab;
   if (tid == 0) s_units[0] = s_units[1] = 0;
   __syncthreads();
-  // pass 1: expert, tokens and token groups of each row; unit counts of the call
+  if (warp == 0) {  // active experts before each bitmap word
+    int run = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      const int c = w < nw ? __popc(bitmap[w]) : 0;
+      int inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (w < nw) wpre[w] = run + inc - c;
+      run += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) s_wsum[0] = run;
+  }
+  __syncthreads();
+  // active-expert rows of the task table (u = 0: the shared expert; routed experts follow in
+  // ascending id), written by the thread of each expert's first token, and the combine's slots
+  const int ns = a.sh.n_shared;
+  const int na = ns + s_wsum[0];
+  const int TD = D / kTileRows;
+  int *tt = a.ws.task_tab;
+  auto rank_of = [&](int e) { return wpre[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u)); };
   int ug = 0, ud = 0;
-  for (int i = tid; i < E + ns; i += kRouteThreads) {
-    const bool shared = i == E;
-    uint32_t m = shared ? (n == 32 ? 0xFFFFFFFFu : (1u << n) - 1u) : tokmask[i];
-    if (!shared && a.out_counts) a.out_counts[i] = __popc(m);
-    if (!m) continue;
-    const int u = shared ? 0 : ns + rank[i];
+  for (int p = tid; p < n * K + ns; p += kRouteThreads) {
+    const bool shared = p == n * K;
+    const int t = shared ? 0 : p / K, ex = shared ? E : s_idx[p];
+    uint32_t m = shared ? (1u << n) - 1u : tokmask[ex];
+    const int u = shared ? 0 : ns + rank_of(ex);
+    if (!shared) a.ws.slotpos[p] = u * kDecodeMaxTokens + __popc(m & ((1u << t) - 1u));
+    if (!shared && (m & ((1u << t) - 1u))) continue;  // not the expert's first token
     const int nt = __popc(m), ng = tok_groups(nt);
     const int F = shared ? a.L.shared.f : a.L.routed.f;
     int *row = tt + kTabHead + u * kTabInts;
-    row[0] = i;
+    row[0] = ex;
     row[1] = nt;
     row[14] = ng;
     int c = 0;
@@ -459,34 +480,30 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
       row[2 + c++] = __ffs(m) - 1;
       m &= m - 1u;
     }
-    s_cnt[0][u] = F;   // d_ff of the row, for pass 2
+    s_cnt[0][u] = F;   // d_ff of the row, for the split pass
     s_cnt[1][u] = ng;
     ug += (F / kTileRows) * ng;
     ud += TD * ng;
   }
   if (ug) atomicAdd(&s_units[0], ug);
   if (ud) atomicAdd(&s_units[1], ud);
+  if (a.out_counts)
+    for (int i = tid; i < E; i += kRouteThreads) a.out_counts[i] = __popc(tokmask[i]);
   __syncthreads();
-  // pass 2: K splits and task counts per row
-  for (int u = tid; u < na; u += kRouteThreads) {
-    const int F = s_cnt[0][u], ng = s_cnt[1][u];
-    int *row = tt + kTabHead + u * kTabInts;
-    int pg, pd;
-    row[11] = unit_split(D / kChunk, s_units[0], a.ws.min_streams, pg);
-    row[13] = unit_split(F / kChunk, s_units[1], a.ws.min_streams, pd);
-    s_cnt[0][u] = (F / kTileRows) * ng * pg;
-    s_cnt[1][u] = ng * pd;
-  }
-  for (int p = tid; p < n * K; p += kRouteThreads) {
-    const int t = p / K, ex = s_idx[p];
-    a.ws.slotpos[p] = (ns + rank[ex]) * kDecodeMaxTokens + __popc(tokmask[ex] & ((1u << t) - 1u));
-  }
-  __syncthreads();
-  if (warp == 0) {  // first task of each active expert: exclusive prefix over u
+  if (warp == 0) {  // K splits, task counts and first task of each active expert (prefix over u)
     int run0 = 0, run1 = 0;
     for (int u0 = 0; u0 < na; u0 += 32) {
       const int u = u0 + lane;
-      const int c0v = u < na ? s_cnt[0][u] : 0, c1v = u < na ? s_cnt[1][u] : 0;
+      int c0v = 0, c1v = 0;
+      if (u < na) {
+        const int F = s_cnt[0][u], ng = s_cnt[1][u];
+        int *row = tt + kTabHead + u * kTabInts;
+        int pg, pd;
+        row[11] = unit_split(D / kChunk, s_units[0], a.ws.min_streams, pg);
+        row[13] = unit_split(F / kChunk, s_units[1], a.ws.min_streams, pd);
+        c0v = (F / kTileRows) * ng * pg;
+        c1v = ng * pd;
+      }
       int i0 = c0v, i1 = c1v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -732,14 +749,20 @@ __device__ __forceinline__ void gemv_stage(const unsigned char *st, const RingPl
   }
 }
 
-// One or two tokens (a unit serves at most kUnitTok tokens).
+// 1 .. kUnitTok tokens (a unit serves at most kUnitTok tokens).
 template <int FMT, int NR, int CMAX>
 __device__ __forceinline__ void gemv_dispatch(int nt, const unsigned char *st, const RingPlan &P, int nch,
                                               uint32_t tab, float (&acc)[2][kUnitTok]) {
-  if (nt == 1)
-    gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc);
-  else
-    gemv_stage<FMT, 0, 2, NR, CMAX>(st, P, nch, tab, acc);
+  if (kUnitTok <= 2 || nt <= 2) {
+    if (nt == 1)
+      gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc);
+    else
+      gemv_stage<FMT, 0, (kUnitTok < 2 ? kUnitTok : 2), NR, CMAX>(st, P, nch, tab, acc);
+  } else if (nt == 3) {
+    gemv_stage<FMT, 0, (kUnitTok < 3 ? kUnitTok : 3), NR, CMAX>(st, P, nch, tab, acc);
+  } else {
+    gemv_stage<FMT, 0, (kUnitTok < 4 ? kUnitTok : 4), NR, CMAX>(st, P, nch, tab, acc);
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1288,7 +1311,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
 // host launcher
 // ------------------------------------------------------------------------------------------
 int route_smem_bytes(int n_experts) {
-  return 2 * n_experts * 4 + (n_experts > 1024 ? kDecodeMaxTokens * n_experts * 4 : 0);
+  return n_experts * 4 + 2 * (kMaxExperts / 32) * 4 + (n_experts > 1024 ? kDecodeMaxTokens * n_experts * 4 : 0);
 }
 
 // Under stream capture the records are made external, so that the CUDA graph records the

@@ -43,6 +43,7 @@ void plan_prefill_workspace(PrefillWs &w, const moe_config &g, char *base, uint6
   w.row_w = static_cast<float *>(take(w.rows_max * 4ull));
   w.tile_prefix = static_cast<int *>(take((E + 2) * 4));
   w.n_tiles = static_cast<int *>(take(4));
+  w.tile_info = static_cast<int4 *>(take((w.rows_max / kPfBN + E + 2) * 16));
   w.xs = static_cast<__nv_bfloat16 *>(take((static_cast<uint64_t>(w.rows_max) + kPfBN) * D * 2));
   w.hs = static_cast<__nv_bfloat16 *>(take((static_cast<uint64_t>(w.rows_max) + kPfBN) * fmax * 2));
   w.outs = static_cast<__nv_bfloat16 *>(take(static_cast<uint64_t>(w.rows_max) * D * 2));
@@ -195,6 +196,8 @@ __global__ void __launch_bounds__(1024) k_pf_scan(PrefillArgs a) {
     a.ws.offsets[g] = crun;
     a.ws.tile_prefix[g] = trun;
     a.ws.fill[g] = 0;
+    for (int j = 0; j * kPfBN < c; ++j)  // token tiles of the group: first row, rows, group
+      a.ws.tile_info[trun + j] = make_int4(crun + j * kPfBN, min(kPfBN, c - j * kPfBN), g, 0);
     crun += c;
     trun += (c + kPfBN - 1) / kPfBN;
   }
@@ -290,6 +293,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 consecutive TMEM columns of this warp's 32 lanes; completes at tmem_wait_ld
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of 128 bytes (64 bf16)
 // in groups of 8 (1024 bytes, the stride between groups); the tile base is 1024-byte aligned and
 // the start address steps by 32 bytes per K = 16.
@@ -325,36 +341,46 @@ __device__ __forceinline__ void cp_async_wait() {
 // ------------------------------------------------------------------------------------------
 // grouped GEMM on tcgen05, warp-specialised.  MODE 0: gate + up (two A matrices, SwiGLU
 // epilogue -> hs); MODE 1: down (one A matrix, epilogue x routing weight -> outs).
-// One CTA per SM walks its (token tile, row tile) list as one stream of 64-deep K-steps through a
-// ring of stages.  Warp roles:
+// One CTA per SM walks its (token tile, row tile) list as one stream of 64-deep K-steps.  Two
+// rings: stages of (raw A blocks + B tile), deep enough to cover the load latency, and a
+// double buffer of dequantised bf16 A tiles.  Warp roles:
 //   warp 12       producer: per stage, the raw blocks of the A matrices (bulk copies) and the B
 //                 tile (one 2-D TMA load, 128-byte swizzle) on one "full" barrier
-//   warps 4..11   dequantisation: raw blocks -> bf16 A tiles (128-byte swizzle), then "a_ready"
+//   warps 4..11   dequantisation: raw blocks -> bf16 A tiles (128-byte swizzle) in a free A
+//                 buffer, then "a_full"
 //   warp 13       MMA: tcgen05.mma kind::f16, M = 128, N <= 256, fp32 accumulators in TMEM;
-//                 the commit of a stage's MMAs frees the stage ("empty")
+//                 the commit of a stage's MMAs frees its stage ("empty") and its A buffer
+//                 ("a_empty")
 //   warps 0..3    epilogue: TMEM -> registers -> SwiGLU / weight -> global (bf16)
 // Accumulators: MODE 0 uses all 512 TMEM columns (gate + up at N = 256), MODE 1 double-buffers
 // (2 x 256 columns) so the epilogue of a tile overlaps the next tile's MMAs.  Every wait is
 // bounded; a role that gives up raises a shared abort flag that ends the others' waits.
 // ------------------------------------------------------------------------------------------
-constexpr int kPfWarps = 14;
+#ifndef MOE_PF_DEQ_WARPS
+#define MOE_PF_DEQ_WARPS 8
+#endif
+constexpr int kDeqWarps = MOE_PF_DEQ_WARPS;           // 8 or 16: 1 or 2 threads per (row, block)
+constexpr int kPfWarps = 6 + kDeqWarps;
 constexpr int kPfThreads = 32 * kPfWarps;
-constexpr int kWarpEpi0 = 0, kWarpDeq0 = 4, kWarpProd = 12, kWarpMma = 13;
-constexpr int kDeqThreads = 256;
+constexpr int kWarpEpi0 = 0, kWarpDeq0 = 4, kWarpProd = 4 + kDeqWarps, kWarpMma = 5 + kDeqWarps;
+constexpr int kDeqThreads = 32 * kDeqWarps;
+constexpr int kDeqSub = kDeqWarps / 8;                 // threads sharing one (row, block)
 
 template <int FMT, int MODE>
 struct PfPlan {
   static constexpr int NM = MODE == 0 ? 2 : 1;
-  static constexpr int kStages = MODE == 0 ? 3 : 4;
+  static constexpr int kStages = MODE == 0 ? 4 : 5;            // (raw + B) stages
+  static constexpr int kABufs = 2;                              // bf16 A buffers
   static constexpr int kAcc = MODE == 0 ? 1 : 2;               // accumulator buffers
   static constexpr int kATile = 128 * 128;                      // 128 x 64 bf16
   static constexpr int kBTile = kPfBN * 128;                    // kPfBN x 64 bf16
   static constexpr int kRawA = 128 * 16, kRawS = 128 * 4, kRawG = FMT == MOE_FMT_CB35_32 ? 128 * 8 : 0;
   static constexpr int kRawM = kRawA + kRawS + kRawG;
   static constexpr int kRaw = NM * kRawM;
-  static constexpr int kStage = NM * kATile + kBTile + ((kRaw + 1023) & ~1023);
+  static constexpr int kStage = kBTile + ((kRaw + 1023) & ~1023);  // B tile, then the raw blocks
+  static constexpr int kABuf = NM * kATile;
   static constexpr int kHead = 2048;  // barriers, flags, TMEM address [0, 1024); grid [1024, 2048)
-  static constexpr int kBytes = 1024 + kHead + kStages * kStage;
+  static constexpr int kBytes = 1024 + kHead + kABufs * kABuf + kStages * kStage;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -362,22 +388,15 @@ struct PfTile {
   int g, rows0, cnt, mt;
 };
 
+// Tile `tile` = (token tile tt, 128-row tile mt); the scan wrote each token tile's group and rows.
 __device__ __forceinline__ bool pf_tile(const PrefillArgs &a, int tile, int mtiles, PfTile &pt) {
   const int tt = tile / mtiles;
-  pt.mt = tile % mtiles;
-  const int G = a.sh.e + a.sh.n_shared;
-  int lo = 0, hi = G;  // group g with tile_prefix[g] <= tt < tile_prefix[g + 1]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldcg(a.ws.tile_prefix + mid) <= tt) lo = mid; else hi = mid;
-  }
-  while (lo + 1 < G && __ldcg(a.ws.tile_prefix + lo + 1) <= tt) ++lo;  // skip empty groups
-  pt.g = lo;
-  const int j = tt - __ldcg(a.ws.tile_prefix + lo);
-  const int c = __ldcg(a.ws.counts + lo);
-  pt.rows0 = __ldcg(a.ws.offsets + lo) + j * kPfBN;
-  pt.cnt = min(kPfBN, c - j * kPfBN);
-  return pt.cnt > 0;
+  pt.mt = tile - tt * mtiles;
+  const int4 ti = __ldcg(a.ws.tile_info + tt);
+  pt.g = ti.z;
+  pt.rows0 = ti.x;
+  pt.cnt = ti.y;
+  return pt.cnt > 0 && pt.g >= 0 && pt.g < a.sh.e + a.sh.n_shared;
 }
 
 // A tile of this CTA's list (blockIdx.x + i * gridDim.x) with its K-step count.
@@ -441,15 +460,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
   constexpr int NM = PL::NM, NS = PL::kStages, NACC = PL::kAcc;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int NA = PL::kABufs;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);   // [NS] producer -> dequant + MMA
-  uint64_t *a_ready = full + NS;                          // [NS] dequant -> MMA
-  uint64_t *empty = a_ready + NS;                         // [NS] MMA commit -> producer
-  uint64_t *acc_full = empty + NS;                        // [NACC] MMA commit -> epilogue
+  uint64_t *empty = full + NS;                            // [NS] MMA commit -> producer
+  uint64_t *a_full = empty + NS;                          // [NA] dequant -> MMA
+  uint64_t *a_empty = a_full + NA;                        // [NA] MMA commit -> dequant
+  uint64_t *acc_full = a_empty + NA;                      // [NACC] MMA commit -> epilogue
   uint64_t *acc_empty = acc_full + NACC;                  // [NACC] epilogue -> MMA
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
   int8_t *grid_s = reinterpret_cast<int8_t *>(smem + 1024);
-  unsigned char *stages = smem + PL::kHead;
+  unsigned char *abufs = smem + PL::kHead;                 // [NA][NM][128 x 64 bf16]
+  unsigned char *stages = abufs + NA * PL::kABuf;          // [NS][B tile | raw blocks]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int D = a.sh.d, fmax = a.ws.fmax;
   const int mtiles = MODE == 0 ? fmax / kTileRows : D / kTileRows;
@@ -463,8 +485,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&a_ready[s], kDeqThreads);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < NA; ++s) {
+      mbar_init(&a_full[s], kDeqThreads);
+      mbar_init(&a_empty[s], 1);
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -498,7 +523,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
           const int st = it % NS;
           if (it >= NS && !(ok = pf_wait(&empty[st], ((it / NS) - 1) & 1u, lim, abort_flag, a.err))) break;
           unsigned char *sb = stages + st * PL::kStage;
-          unsigned char *raw = sb + NM * PL::kATile + PL::kBTile;
+          unsigned char *raw = sb + PL::kBTile;
           mbar_arrive_expect_tx(&full[st], PL::kRaw + PL::kBTile);
           const int64_t slot0 = (static_cast<int64_t>(c.pt.mt) * c.nc + s) * kTileRows;
 #pragma unroll
@@ -510,7 +535,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
             if (FMT == MOE_FMT_CB35_32)
               bulk_g2s(rm + PL::kRawA + PL::kRawS, G.g + mat * G.g_mat + slot0, PL::kRawG, &full[st]);
           }
-          tma_load_2d(sb + NM * PL::kATile, bmap, s * kChunk, c.pt.rows0, &full[st]);
+          tma_load_2d(sb, bmap, s * kChunk, c.pt.rows0, &full[st]);
         }
       }
       // leave only once every copy this thread issued has landed
@@ -518,19 +543,23 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
       for (uint32_t k = (issued > NS ? issued - NS : 0); k < issued; ++k)
         mbar_wait_bounded(&full[k % NS], (k / NS) & 1u, kDrainLimit);
     }
-  } else if (warp >= kWarpDeq0 && warp < kWarpDeq0 + 8) {
-    // ---------------- dequantisation: thread -> (row r, block h) of each matrix
-    const int t = tid - 32 * kWarpDeq0, r = t & 127, h = t >> 7;
+  } else if (warp >= kWarpDeq0 && warp < kWarpDeq0 + kDeqWarps) {
+    // ---------------- dequantisation: thread -> (row r, block h, share sub) of the NM x 4 items
+    // (matrix, 8-weight group) of that block; sub takes a contiguous share of the items
+    const int t = tid - 32 * kWarpDeq0, r = t & 127, h = (t >> 7) & 1, sub = t >> 8;
+    constexpr int kItems = 4 * NM / kDeqSub;
     uint32_t it = 0;
     bool ok = true;
     for (PfCursor c = first; c.valid && ok; pf_advance<MODE>(a, mtiles, total, c)) {
       for (int s = 0; s < c.nc; ++s, ++it) {
-        const int st = it % NS;
+        const int st = it % NS, sa = it % NA;
         if (!(ok = pf_wait(&full[st], (it / NS) & 1u, lim, abort_flag, a.err))) break;
-        unsigned char *sb = stages + st * PL::kStage;
-        const unsigned char *raw = sb + NM * PL::kATile + PL::kBTile;
+        if (it >= NA && !(ok = pf_wait(&a_empty[sa], ((it / NA) - 1) & 1u, lim, abort_flag, a.err))) break;
+        const unsigned char *raw = stages + st * PL::kStage + PL::kBTile;
+        unsigned char *ab = abufs + sa * PL::kABuf;
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
+          if (kDeqSub > 1 && NM == 2 && m != sub) continue;  // gate/up: one matrix per share
           const unsigned char *rm = raw + m * PL::kRawM;
           const uint4 A = reinterpret_cast<const uint4 *>(rm)[r];
           const __half2 sc2 = reinterpret_cast<const __half2 *>(rm + PL::kRawA)[r];
@@ -541,21 +570,37 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
             const uint2 G2 = reinterpret_cast<const uint2 *>(rm + PL::kRawA + PL::kRawS)[r];
             sgn = h ? G2.y : G2.x;
           }
-          unsigned char *at = sb + m * PL::kATile;
+          unsigned char *at = ab + m * PL::kATile;
+          // Q2: the block's four bf16 values s (q - 1.5), q = 0..3, as bytes 0..7 of (T0, T1); a
+          // prmt selector built from two codes picks the bf16 pair of two consecutive weights
+          uint32_t T0 = 0, T1 = 0;
+          if (FMT == MOE_FMT_Q2_32) {
+            const __nv_bfloat162 t01 = __floats2bfloat162_rn(-1.5f * sc, -0.5f * sc);
+            const __nv_bfloat162 t23 = __floats2bfloat162_rn(0.5f * sc, 1.5f * sc);
+            T0 = *reinterpret_cast<const uint32_t *>(&t01);
+            T1 = *reinterpret_cast<const uint32_t *>(&t23);
+          }
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
-            float v[8];
+            if (kDeqSub > 1 && NM == 1 && cc / kItems != sub) continue;  // down: half the groups
             if (FMT == MOE_FMT_Q2_32) {
-              // float(2^23 + q) by exponent bias, minus 2^23: the code q exactly; then s (q - 1.5)
+              // weights 8cc .. 8cc+7 = groups kk, kk+1 of one word (weight 4kk + j in byte j)
+              const uint32_t w = cc < 2 ? w0 : w1;
+              uint32_t o[4];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int p = 8 * cc + i;
-                const uint32_t w = p < 16 ? w0 : w1;
-                const int pw = p & 15, kk = pw >> 2, jj = pw & 3;
-                const float q = __uint_as_float(((w >> (8 * jj + 2 * kk)) & 3u) | 0x4B000000u) - 8388608.0f;
-                v[i] = fmaf(sc, q, -1.5f * sc);
+              for (int g = 0; g < 2; ++g) {
+                const int kk = 2 * (cc & 1) + g;
+                const uint32_t x = (w >> (2 * kk)) & 0x03030303u;  // code of weight 4kk + j in byte j
+                // nibbles (2c, 2c+1) per code: x * 34 = 2x | (2x << 4) (no carries), + 1 on odd nibbles
+                const uint32_t sel = x * 34u + 0x10101010u;
+                o[2 * g] = __byte_perm(T0, T1, sel & 0xFFFFu);
+                o[2 * g + 1] = __byte_perm(T0, T1, sel >> 16);
               }
-            } else {
+              *reinterpret_cast<uint4 *>(at + sw128_off(r, 4 * h + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+              continue;
+            }
+            float v[8];
+            {
 #pragma unroll
               for (int gg = 0; gg < 2; ++gg) {
                 const int g = 2 * cc + gg;
@@ -580,7 +625,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
           }
         }
         fence_proxy_async_smem();  // make the generic-proxy stores visible to the tensor core
-        mbar_arrive(&a_ready[st]);
+        mbar_arrive(&a_full[sa]);
       }
     }
   } else if (warp == kWarpMma) {
@@ -588,6 +633,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
     if (lane == 0) {
       uint32_t it = 0, tl = 0;
       bool ok = true;
+      const uint64_t adesc0 = sw128_desc(smem_u32(abufs)), bdesc0 = sw128_desc(smem_u32(stages));
       for (PfCursor c = first; c.valid && ok; pf_advance<MODE>(a, mtiles, total, c), ++tl) {
         const int b = tl % NACC;
         if (tl >= NACC && !(ok = pf_wait(&acc_empty[b], ((tl / NACC) - 1) & 1u, lim, abort_flag, a.err))) break;
@@ -595,21 +641,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
         const uint32_t acc = tmem + b * (NM * kPfBN);
         const uint32_t idesc = idesc_bf16((c.pt.cnt + 15) & ~15);
         for (int s = 0; s < c.nc; ++s, ++it) {
-          const int st = it % NS;
+          const int st = it % NS, sa = it % NA;
           if (!(ok = pf_wait(&full[st], (it / NS) & 1u, lim, abort_flag, a.err))) break;
-          if (!(ok = pf_wait(&a_ready[st], (it / NS) & 1u, lim, abort_flag, a.err))) break;
+          if (!(ok = pf_wait(&a_full[sa], (it / NA) & 1u, lim, abort_flag, a.err))) break;
           tc_fence_after();
-          unsigned char *sb = stages + st * PL::kStage;
-          const uint32_t bt = smem_u32(sb + NM * PL::kATile);
+          // descriptor start fields advance by (byte offset >> 4); K = 16 is 32 bytes
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>((st * PL::kStage) >> 4);
 #pragma unroll
           for (int m = 0; m < NM; ++m) {
-            const uint32_t at = smem_u32(sb + m * PL::kATile);
+            const uint64_t ad = adesc0 + static_cast<uint64_t>((sa * PL::kABuf + m * PL::kATile) >> 4);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              tc_mma(acc + m * kPfBN, sw128_desc(at + 32 * kk), sw128_desc(bt + 32 * kk), idesc,
-                     (s > 0 || kk > 0) ? 1u : 0u);
+              tc_mma(acc + m * kPfBN, ad + 2 * kk, bd + 2 * kk, idesc, (s > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&empty[st]);
+          tc_commit(&a_empty[sa]);
         }
         if (ok) tc_commit(&acc_full[b]);
       }
@@ -628,24 +674,31 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
       const PfTile &pt = c.pt;
       const int row = pt.mt * kTileRows + 32 * q + lane;
       const uint32_t acc = tmem + b * (NM * kPfBN) + (static_cast<uint32_t>(32 * q) << 16);
-      for (int c0 = 0; c0 < pt.cnt; c0 += 16) {
-        float g[16];
-        tmem_ld16(acc + c0, g);
+      for (int c0 = 0; c0 < pt.cnt; c0 += 32) {
+        uint32_t g[32];
+        tmem_ld32_nowait(acc + c0, g);
         if (MODE == 0) {
-          float u[16];
-          tmem_ld16(acc + kPfBN + c0, u);
+          uint32_t u[32];
+          tmem_ld32_nowait(acc + kPfBN + c0, u);
+          tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < pt.cnt)
-              a.ws.hs[static_cast<int64_t>(pt.rows0 + c0 + i) * fmax + row] = __float2bfloat16_rn(silu_f(g[i]) * u[i]);
+          for (int i = 0; i < 32; ++i) {
+            if (c0 + i < pt.cnt) {
+              const float z = __uint_as_float(g[i]);
+              const float h = __fdividef(z, 1.0f + __expf(-z)) * __uint_as_float(u[i]);
+              a.ws.hs[static_cast<int64_t>(pt.rows0 + c0 + i) * fmax + row] = __float2bfloat16_rn(h);
+            }
+          }
         } else {
-          float wr[16];
+          // routing weights of the 32 rows: lane i loads row c0 + i, shuffled to every lane
+          const float wl = c0 + lane < pt.cnt ? __ldcg(a.ws.row_w + pt.rows0 + c0 + lane) : 0.f;
+          tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) wr[i] = c0 + i < pt.cnt ? __ldcg(a.ws.row_w + pt.rows0 + c0 + i) : 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < 32; ++i) {
+            const float wr = __shfl_sync(0xffffffffu, wl, i);
             if (c0 + i < pt.cnt)
-              a.ws.outs[static_cast<int64_t>(pt.rows0 + c0 + i) * D + row] = __float2bfloat16_rn(g[i] * wr[i]);
+              a.ws.outs[static_cast<int64_t>(pt.rows0 + c0 + i) * D + row] = __float2bfloat16_rn(__uint_as_float(g[i]) * wr);
+          }
         }
       }
       tc_fence_before();

@@ -31,6 +31,7 @@ struct PrefillWs {
   float *row_w;          // [rows_max] routing weight of each grouped row (1 for the shared expert)
   int *tile_prefix;      // [E + 2]   prefix over groups of kPfBN-row token tiles
   int *n_tiles;          // [1]       token tiles of the call
+  int4 *tile_info;       // [token tiles] first grouped row, rows, group (written by the scan)
   __nv_bfloat16 *xs;     // [rows_max + kPfBN][D]   gathered bf16 activations
   __nv_bfloat16 *hs;     // [rows_max + kPfBN][Fmax] SwiGLU outputs (bf16)
   __nv_bfloat16 *outs;   // [rows_max][D]   weighted expert outputs (bf16)
