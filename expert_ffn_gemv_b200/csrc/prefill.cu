@@ -360,9 +360,13 @@ __device__ __forceinline__ void cp_async_wait() {
 #define MOE_PF_DEQ_WARPS 8
 #endif
 constexpr int kDeqWarps = MOE_PF_DEQ_WARPS;           // 8 or 16: 1 or 2 threads per (row, block)
-constexpr int kPfWarps = 6 + kDeqWarps;
+// epilogue: warps 0..3 and kWarpEpi1..+3 (warp w reads TMEM lanes 32 (w % 4) ..; the two sets
+// take alternate 32-column groups)
+constexpr int kPfWarps = 10 + kDeqWarps;
 constexpr int kPfThreads = 32 * kPfWarps;
-constexpr int kWarpEpi0 = 0, kWarpDeq0 = 4, kWarpProd = 4 + kDeqWarps, kWarpMma = 5 + kDeqWarps;
+constexpr int kWarpEpi0 = 0, kWarpDeq0 = 4, kWarpProd = 4 + kDeqWarps, kWarpMma = 5 + kDeqWarps,
+              kWarpEpi1 = 6 + kDeqWarps;
+constexpr int kEpiThreads = 256;
 constexpr int kDeqThreads = 32 * kDeqWarps;
 constexpr int kDeqSub = kDeqWarps / 8;                 // threads sharing one (row, block)
 
@@ -493,7 +497,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], kEpiThreads);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -662,9 +666,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
       // every committed MMA must be complete before the TMEM is released
       if (it > 0) mbar_wait_bounded(&empty[(it - 1) % NS], ((it - 1) / NS) & 1u, kDrainLimit);
     }
-  } else if (warp < kWarpEpi0 + 4) {
-    // ---------------- epilogue: warp q reads TMEM lanes 32q .. 32q+31 (= rows of the tile)
-    const int q = warp - kWarpEpi0;
+  } else if (warp < kWarpEpi0 + 4 || warp >= kWarpEpi1) {
+    // ---------------- epilogue: warp q reads TMEM lanes 32q .. 32q+31 (= rows of the tile);
+    // set e (0: warps 0..3, 1: the second four) takes column groups e, e + 2, ...
+    const int q = warp & 3, e = warp >= kWarpEpi1 ? 1 : 0;
     uint32_t tl = 0;
     bool ok = true;
     for (PfCursor c = first; c.valid && ok; pf_advance<MODE>(a, mtiles, total, c), ++tl) {
@@ -674,7 +679,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
       const PfTile &pt = c.pt;
       const int row = pt.mt * kTileRows + 32 * q + lane;
       const uint32_t acc = tmem + b * (NM * kPfBN) + (static_cast<uint32_t>(32 * q) << 16);
-      for (int c0 = 0; c0 < pt.cnt; c0 += 32) {
+      for (int c0 = 32 * e; c0 < pt.cnt; c0 += 64) {
         uint32_t g[32];
         tmem_ld32_nowait(acc + c0, g);
         if (MODE == 0) {
