@@ -289,8 +289,8 @@ def bench_verify(args, rank, world, local):
     barrier(world)
     ms_local = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms_local, world)
-    # roofline kernel: a second graph of the same pass with event pairs around each gate/up
-    # launch, replayed Kr times over the same inputs; durations of its last replay
+    # roofline kernel: a second graph of the same pass with event pairs around each expert-GEMV
+    # launch (gate/up + down), replayed Kr times over the same inputs; durations of its last replay
     P.moe_profile_enable(moe.h, 1 << P.PROF_GATEUP)
     Kr = min(K, 32)
     with torch.cuda.stream(stream):
@@ -312,7 +312,7 @@ def bench_verify(args, rank, world, local):
         moe.forward_stack(0, L, x_in, out)
     stream.synchronize()
     kern = {}
-    for kind, name in ((P.PROF_ROUTE, "k_route"), (P.PROF_GATEUP, "k_gemv<gate/up>"), (P.PROF_DOWN, "k_gemv<down>+combine")):
+    for kind, name in ((P.PROF_ROUTE, "k_route"), (P.PROF_GATEUP, "k_gemv"), (P.PROF_DOWN, "k_combine")):
         _, tot, cnt = P.moe_profile_read(moe.h, kind)
         kern[name] = (tot, cnt)
     P.moe_profile_enable(moe.h, False)
@@ -331,17 +331,16 @@ def bench_verify(args, rank, world, local):
     # algorithmic bytes: every active expert's blocks (gate + up + down) + shared, + router
     router_bytes = wl.n_experts * wl.d_model * 2
     step_bytes = ((u_all + wl.n_shared) * expert_bytes).sum(axis=1) + L * router_bytes  # per pass
-    gateup_bytes_last = float(((u_all[Kr - 1] + wl.n_shared) * 2 * mat_bytes).sum())  # input of g2's last replay
-    down_bytes_last = float(((u_all[-1] + wl.n_shared) * mat_bytes).sum())
+    gemv_bytes_last = float(((u_all[Kr - 1] + wl.n_shared) * expert_bytes).sum())  # input of g2's last replay
 
     tokens = K * n
     total_tokens = sum_over_ranks(tokens, world)
     value = total_tokens / (ms / 1e3)
     pk, pk_kind = peaks()
     hbm_peak = pk["hbm_gbs"]
-    achieved = gateup_bytes_last / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
+    achieved = gemv_bytes_last / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
     src = source_hash("expert_ffn_gemv_b200/csrc/decode.cu", "expert_ffn_gemv_b200/csrc/moe_internal.cuh")
-    traffic = profiled_traffic("k_gemv_gateup", "verify", src)
+    traffic = profiled_traffic("k_gemv", "verify", src)
     res = {
         "metric": METRIC,
         "value": value,
@@ -361,20 +360,18 @@ def bench_verify(args, rank, world, local):
                    "resident_weight_gb": round(moe.device_bytes() / 1e9, 2),
                    "l2": "inputs larger than L2: each pass reads ~%.1f GB of distinct expert blocks"
                          % (step_bytes.mean() / 1e9),
-                   "parallelism": f"replicas x{world}", "cuda_graph": "one pass (48 x 4 kernels, programmatic launches) per replay"},
+                   "parallelism": f"replicas x{world}", "cuda_graph": "one pass (48 x 3 kernels, programmatic launches) per replay"},
         "hbm": {"active_expert_and_router_bytes_per_step": float(step_bytes.mean()),
                 "gbs": float(step_bytes.sum() / (ms_local / 1e3) / 1e9),
                 "frac_of_measured_peak": float(step_bytes.sum() / (ms_local / 1e3) / 1e9 / hbm_peak),
                 "mean_active_experts_per_layer": float(u_all.mean() + wl.n_shared)},
-        "roofline": {"kernel": "k_gemv<gate/up>", "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+        "roofline": {"kernel": "k_gemv (gate/up + down)", "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
                      "peak_kind": pk_kind, "unit": "GB/s",
                      "frac": achieved / hbm_peak if achieved else None, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": gateup_bytes_last / max(gu_cnt, 1),
+                     "algorithmic_bytes_per_launch": gemv_bytes_last / max(gu_cnt, 1),
                      "avg_launch_us": gu_ms / max(gu_cnt, 1) * 1e3},
         "kernels_eager_pass_us": {k: round(v[0] * 1e3, 2) for k, v in kern.items()},
-        "down_roofline": {"achieved": down_bytes_last / (kern["k_gemv<down>+combine"][0] / 1e3) / 1e9
-                          if kern["k_gemv<down>+combine"][0] else None, "unit": "GB/s"},
-        "gpu_launches": K * L * 4,
+        "gpu_launches": K * L * 3,
         "clocks": clk.summary(),
         "load_seconds": round(load_s, 1),
     }
@@ -478,7 +475,6 @@ def bench_decode_layers(args, rank, world, local):
     u = np.array([int((c > 0).sum()) for c in counts]) + wl.n_shared
     eb = wl.expert_bytes()
     step_bytes = float((u * eb).sum())
-    gu_bytes = float((u * 2 * eb // 3).sum())
     pk, kind = peaks()
     gbs = step_bytes * K / (ms / 1e3) / 1e9
     res = _base_result(wl, world, K, W, ms, "GB/s", sum_over_ranks(gbs, world))
@@ -488,12 +484,12 @@ def bench_decode_layers(args, rank, world, local):
                            "l2": "16 distinct layers per step"},
                 "tokens_per_s_one_layer": K * nl / (ms / 1e3),
                 "us_per_layer": ms * 1e3 / (K * nl),
-                "roofline": {"kernel": "k_gemv<gate/up>", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                "roofline": {"kernel": "k_gemv (gate/up + down)", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
                              "peak_kind": kind,
-                             "achieved": gu_bytes / (kms / 1e3) / 1e9 if kms else None,
-                             "frac": gu_bytes / (kms / 1e3) / 1e9 / pk["hbm_gbs"] if kms else None,
+                             "achieved": step_bytes / (kms / 1e3) / 1e9 if kms else None,
+                             "frac": step_bytes / (kms / 1e3) / 1e9 / pk["hbm_gbs"] if kms else None,
                              "avg_launch_us": kms / max(kcnt, 1) * 1e3},
-                "hbm_frac_whole_layer": gbs / pk["hbm_gbs"], "clocks": clocks, "gpu_launches": K * nl * 4})
+                "hbm_frac_whole_layer": gbs / pk["hbm_gbs"], "clocks": clocks, "gpu_launches": K * nl * 3})
     moe.close()
     return res
 
@@ -528,17 +524,17 @@ def bench_codebook(args, rank, world, local):
         u = np.array([int((c > 0).sum()) for c in counts]) + wl.n_shared
         eb = wl.expert_bytes()
         gbs = float((u * eb).sum()) * K / (ms / 1e3) / 1e9
-        gu = float((u * 2 * eb // 3).sum())
+        gb = float((u * eb).sum())
         out[n] = {"tokens_per_s": sum_over_ranks(n * K / (ms / 1e3), world), "ms_per_step": ms / K, "gbs": gbs,
-                  "frac": gbs / pk["hbm_gbs"], "gateup_gbs": gu / (kms / 1e3) / 1e9 if kms else None,
+                  "frac": gbs / pk["hbm_gbs"], "gemv_gbs": gb / (kms / 1e3) / 1e9 if kms else None,
                   "clocks": clocks}
     res = _base_result(wl, world, K, W, out[8]["ms_per_step"] * K, "tokens/s", out[8]["tokens_per_s"])
     res.update({"dtype": "cb35 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
                 "config": {"workload": wl.name, "layers": nl, "tokens": [1, 8], "chain": "independent layers"},
-                "by_tokens": out, "gpu_launches": K * nl * 4,
-                "roofline": {"kernel": "k_gemv<gate/up>", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
-                             "peak_kind": kind, "achieved": out[8]["gateup_gbs"],
-                             "frac": out[8]["gateup_gbs"] / pk["hbm_gbs"] if out[8]["gateup_gbs"] else None}})
+                "by_tokens": out, "gpu_launches": K * nl * 3,
+                "roofline": {"kernel": "k_gemv (gate/up + down)", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                             "peak_kind": kind, "achieved": out[8]["gemv_gbs"],
+                             "frac": out[8]["gemv_gbs"] / pk["hbm_gbs"] if out[8]["gemv_gbs"] else None}})
     moe.close()
     return res
 

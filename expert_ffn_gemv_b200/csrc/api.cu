@@ -144,6 +144,7 @@ void plan_workspace(moe_handle *h, Carve &c) {
   w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * 4);  // x token groups of a unit
   w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td * 4);
   w.counters = c.take<unsigned>(2);
+  w.h_done = c.take<unsigned>(static_cast<uint64_t>(umax) * 4);
   const uint64_t nt = static_cast<uint64_t>(g.max_tokens) * D;
   h->res[0] = c.take<float>(nt);
   h->res[1] = c.take<float>(nt);
@@ -165,6 +166,7 @@ moe_status check_device_error(moe_handle *h, cudaStream_t st) {
   cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax * 4, st);
   cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td * 4, st);
   cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * 2, st);
+  cudaMemsetAsync(w.h_done, 0, sizeof(unsigned) * w.umax * 4, st);
   if (e & kErrTimeout) return fail(h, MOE_ERR_TIMEOUT, "a device-side bounded wait ran out");
   return fail(h, MOE_ERR_DEVICE_FAULT, "a device-side check found an invalid routing index");
 }
@@ -336,7 +338,7 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
         goto fail_out;
       }
     }
-    cudaError_t ge = decode_grid_sizes(g.fmt, h->dws.umax, &h->dws.grid_gu, &h->dws.grid_dn, &h->dws.min_streams);
+    cudaError_t ge = decode_grid_sizes(g.fmt, h->dws.umax, &h->dws.grid_gemv, &h->dws.min_streams);
     if (ge != cudaSuccess) {
       s = cuda_fail(h, ge, "grid sizing");
       goto fail_out;

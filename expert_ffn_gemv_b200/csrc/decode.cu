@@ -40,7 +40,7 @@ constexpr int kConsWarps = kTileRows / 32;      // consumer warps: thread = row 
 constexpr int kGemvThreads = kTileRows + 32;    // + one producer warp
 constexpr int kRing = 4;                        // most stages of the bulk-copy ring
 #ifndef MOE_GEMV_MIN_BLOCKS
-#define MOE_GEMV_MIN_BLOCKS 4                   // resident CTAs per SM the register budget allows
+#define MOE_GEMV_MIN_BLOCKS 3                   // resident CTAs per SM the register budget allows
 #endif
 #ifndef MOE_GEMV_UNROLL
 #define MOE_GEMV_UNROLL 1                       // chunks of a stage in flight per iteration
@@ -54,6 +54,8 @@ constexpr int kGemvUnroll = MOE_GEMV_UNROLL;
 __host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_CB35_32 ? 3 : 4; }
 constexpr int kGuStageChunks = 2;               // gate/up: chunks per stage
 constexpr int kDnStageChunks = 4;               // down: chunks per stage (one K segment)
+constexpr int kStageSlots = 2 * kGuStageChunks;   // (matrix, chunk) slots of a stage: 4 either way
+static_assert(kStageSlots == kDnStageChunks, "gate/up and down stages share one layout");
 constexpr int kPartStride = kDecodeMaxTokens * kTileRows;  // floats per (segment, matrix)
 
 // Q2 block arithmetic.  A block's value is sum_i (q_i - 1.5) m_i = (2S - 3M) / 2 with S = sum q_i m_i
@@ -290,10 +292,11 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
   }
   griddep_wait();
   griddep_launch();
-  // the work queues of this layer's GEMV kernels start empty (the previous layer is done)
-  if (blockIdx.x == 0 && tid == 0) {
-    a.ws.counters[0] = 0u;
-    a.ws.counters[1] = 0u;
+  // the work queue and the h counters of this layer's GEMV kernel start empty (the previous
+  // layer is done)
+  if (blockIdx.x == 0) {
+    if (tid < 2) a.ws.counters[tid] = 0u;
+    for (int i = tid; i < a.ws.umax * kMaxTokGroups; i += kRouteThreads) a.ws.h_done[i] = 0u;
   }
 
   // ---- the K slice of the n tokens, as fp32
@@ -647,6 +650,7 @@ struct RingHdr {
   uint64_t cbar;  // barrier of the consumer warps (kConsWarps arrivals)
   StageInfo info[kRing];
   int n_active;
+  int n_gu;        // tasks below n_gu are gate/up pieces, the rest down pieces
   volatile int abort;
   int flag[2];
   float wmax[2][kConsWarps][kUnitTok];
@@ -800,10 +804,9 @@ __device__ __forceinline__ void cons_fail(const DecodeArgs &a, RingHdr *H) {
 }
 
 
-// Load the task table (one round of independent loads) and check it.  Returns the task count,
-// or -1 (uniform over the warp) when an entry is out of range.
-template <bool GU>
-__device__ __forceinline__ int producer_tables(const DecodeArgs &a, RingHdr *H, int *tb) {
+// Load the task table (one round of independent loads) and check it for both GEMVs.  Returns
+// false (uniform over the warp) when an entry is out of range; n_gu / n_dn: the task counts.
+__device__ bool producer_tables(const DecodeArgs &a, RingHdr *H, int *tb, int &n_gu, int &n_dn) {
   const int lane = threadIdx.x & 31;
   const int umax = a.ws.umax, E = a.sh.e, D = a.sh.d;
   const int4 *src = reinterpret_cast<const int4 *>(a.ws.task_tab);
@@ -811,32 +814,38 @@ __device__ __forceinline__ int producer_tables(const DecodeArgs &a, RingHdr *H, 
   for (int i = lane; i < (kTabHead + kTabInts * umax) / 4; i += 32) dst[i] = __ldcg(src + i);
   __syncwarp();
   const int na = tb[0];
-  const int total = GU ? tb[1] : tb[2];
-  bool bad = na < 1 || na > umax || total < 1;
+  n_gu = tb[1];
+  n_dn = tb[2] * (D / kTileRows);
+  bool bad = na < 1 || na > umax || tb[1] < 1 || tb[2] < 1;
   for (int u = lane; !bad && u < na; u += 32) {
     const int *row = tb + kTabHead + u * kTabInts;
-    const int e = row[0], nt = row[1];
-    bool b = e < 0 || e > E || (e == E) != (a.sh.n_shared && u == 0) || nt < 1 || nt > kDecodeMaxTokens;
+    const int e = row[0], nt = row[1], ng = row[14];
+    bool b = e < 0 || e > E || (e == E) != (a.sh.n_shared && u == 0) || nt < 1 || nt > kDecodeMaxTokens ||
+             ng != tok_groups(nt);
     for (int i = 0; !b && i < nt; ++i) b = row[2 + i] < 0 || row[2 + i] >= a.n;
-    if (!b) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {  // k = 0: gate/up (K = d_model), k = 1: down (K = d_ff)
+      if (b) break;
       const int F = e == E ? a.L.shared.f : a.L.routed.f;
-      const int nc = (GU ? D : F) / kChunk;
-      const int pk = row[GU ? 11 : 13], ng = row[14];
+      const int nc = (k == 0 ? D : F) / kChunk;
+      const int pk = row[k == 0 ? 11 : 13];
       const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
-      b = (seg != 2 && seg != 4) || nseg * seg != nc || len < 1 || len > nseg || pieces != (nseg + len - 1) / len ||
-          ng != tok_groups(nt);
-      const int cnt = GU ? (F / kTileRows) * ng * pieces : ng * pieces;
-      const int base = row[GU ? 10 : 12];
-      const int next = u + 1 < na ? row[kTabInts + (GU ? 10 : 12)] : total;
+      b = (seg != 2 && seg != 4) || nseg * seg != nc || len < 1 || len > nseg || pieces != (nseg + len - 1) / len;
+      const int cnt = k == 0 ? (F / kTileRows) * ng * pieces : ng * pieces;
+      const int base = row[k == 0 ? 10 : 12];
+      const int next = u + 1 < na ? row[kTabInts + (k == 0 ? 10 : 12)] : tb[1 + k];
       b = b || base + cnt != next || (u == 0 && base != 0);
     }
     bad = b;
   }
   bad = __any_sync(0xffffffffu, bad);
-  if (bad) return -1;
-  if (lane == 0) H->n_active = na;
+  if (bad) return false;
+  if (lane == 0) {
+    H->n_active = na;
+    H->n_gu = n_gu;
+  }
   __syncwarp();
-  return GU ? total : total * (D / kTileRows);
+  return true;
 }
 
 // largest u with first-task(u) <= r (first tasks increase with u, first-task(0) = 0)
@@ -851,32 +860,34 @@ __device__ __forceinline__ int find_expert(const int *tb, int na, int r) {
   return lo;
 }
 
-// The producer warp: work queue -> bulk copies into the ring.  Every stage it arms is waited
-// for (bounded) before the warp leaves, so no copy is in flight when the CTA exits.
-template <int FMT, bool GU>
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// The producer warp: one work queue of gate/up pieces (tasks < n_gu) then down pieces ->
+// bulk copies into the ring.  A down piece issues its weight copies at once and its h records
+// once every gate/up tile of its expert and token group has written h (a counter the gate/up
+// epilogue raises); gate/up pieces wait for nothing but their own copies, and all CTAs of the
+// grid are resident, so that wait always ends.  Every stage the warp arms is waited for
+// (bounded) before it leaves, so no copy is in flight when the CTA exits.
+template <int FMT>
 __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H) {
-  constexpr int NR = GU ? 2 : 1;
-  constexpr int CMAX = GU ? kGuStageChunks : kDnStageChunks;
   constexpr int RING = ring_depth(FMT);
+  constexpr int kPlanes = FMT == MOE_FMT_CB35_32 ? 3 : 2;
   const int lane = threadIdx.x & 31;
-  const int D = a.sh.d, E = a.sh.e;
+  const int D = a.sh.d, E = a.sh.e, TD = D / kTileRows;
   int *tb = reinterpret_cast<int *>(smem + P.table);
-  unsigned *ctr = a.ws.counters + (GU ? 0 : 1);
-  // gate/up reads the router kernel's tables, so it waits for that kernel first.  The down
-  // kernel's tables and work queue come from the router kernel too (complete before gate/up,
-  // the kernel before down, could start), so down loads them and issues the weight copies of
-  // its first task while gate/up finishes; the h records wait for gate/up.
-  if (GU) griddep_wait();
-  bool waited = GU;
-  int npend = 0, pend_slot[RING], pend_c0[RING];
+  unsigned *ctr = a.ws.counters;
+  griddep_wait();  // the router kernel's tables
   int task = 0;
   if (lane == 0) task = static_cast<int>(atomicAdd(ctr, 1u));  // in flight while the table loads
-  const int n_tasks = producer_tables<GU>(a, H, tb);
-  bool ok = n_tasks >= 0;
+  int n_gu = 0, n_dn = 0;
+  bool ok = producer_tables(a, H, tb, n_gu, n_dn);
   if (!ok && lane == 0) flag_error(a.err, kErrBadIndex);
+  const int n_tasks = ok ? n_gu + n_dn : 0;
   const int na = ok ? H->n_active : 0;
-  const int TD = D / kTileRows;
-  const int per_mt = GU ? 0 : (ok ? n_tasks / TD : 0);
   const uint64_t pol = l2_evict_first_policy();
   int slot = 0;
   uint32_t round = 0;
@@ -887,10 +898,10 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
   while (ok && task < n_tasks) {
     int nxt = 0;
     if (lane == 0) nxt = static_cast<int>(atomicAdd(ctr, 1u));  // fetched while this piece is issued
-    int u, mt, piece;
+    const bool gu = task < n_gu;
+    int u, mt, grp, piece;
     const int *tr = tb + kTabHead;
-    int grp;
-    if (GU) {
+    if (gu) {
       u = find_expert<true>(tb, na, task);
       const int pieces = (tr[u * kTabInts + 11] >> 8) & 0xFF, ng = tr[u * kTabInts + 14];
       const int r = task - tr[u * kTabInts + 10];
@@ -898,12 +909,13 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
       const int q = r - mt * ng * pieces;
       grp = q / pieces;
       piece = q - grp * pieces;
-    } else {
-      mt = task / per_mt;
-      const int r = task - mt * per_mt;
-      u = find_expert<false>(tb, na, r);
-      const int pieces = (tr[u * kTabInts + 13] >> 8) & 0xFF;
-      const int q = r - tr[u * kTabInts + 12];
+    } else {  // expert-major, like the gate/up pieces, so that the first down pieces find h early
+      const int t2 = task - n_gu;
+      u = find_expert<false>(tb, na, t2 / TD);
+      const int pieces = (tr[u * kTabInts + 13] >> 8) & 0xFF, ng = tr[u * kTabInts + 14];
+      const int r = t2 - tr[u * kTabInts + 12] * TD;
+      mt = r / (ng * pieces);
+      const int q = r - mt * ng * pieces;
       grp = q / pieces;
       piece = q - grp * pieces;
     }
@@ -911,14 +923,16 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
     const int e = row[0];
     const int gsz = tok_group_size(row[1]), tok0 = grp * gsz;
     const int ntok = min(gsz, row[1] - tok0);  // tokens of this unit: slots tok0 .. tok0 + ntok - 1
-    const int pk = row[GU ? 11 : 13];
+    const int pk = row[gu ? 11 : 13];
     const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
     const bool shared = a.sh.n_shared && e == E;
     const ExpertGroup &G = shared ? a.L.shared : a.L.routed;
     const int eidx = shared ? 0 : e;
-    const int nc = GU ? D / kChunk : G.f / kChunk;
+    const int nr = gu ? 2 : 1, cmax = gu ? kGuStageChunks : kDnStageChunks;
+    const int nc = gu ? D / kChunk : G.f / kChunk;
     const int cbeg = piece * len * seg, cend = min(nseg, (piece + 1) * len) * seg;
-    const int sch = GU ? kGuStageChunks : seg;
+    const int sch = gu ? kGuStageChunks : seg;
+    bool h_ready = gu;
     for (int c0 = cbeg; c0 < cend; c0 += sch) {
       if (round > 0) ok = ring_wait(H, &H->empty[slot], (round - 1) & 1u, a.spin_limit);
       if (!ok) break;
@@ -938,46 +952,51 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
                    (nseg << 16) | (tok0 << 24);
         in.c0 = c0;
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&H->full[slot], NR * wbytes + ntok * rbytes);
+        mbar_arrive_expect_tx(&H->full[slot], nr * wbytes + ntok * rbytes);
       }
       __syncwarp();
       unsigned char *st = smem + P.stage0 + slot * P.stage;
-      // copy l of the stage, issued by lane l: NR x (A, S[, G]) weight planes, then one run of
-      // records per token
-      constexpr int kPlanes = FMT == MOE_FMT_CB35_32 ? 3 : 2;
-      if (lane < NR * kPlanes) {
+      // copy l of the stage, issued by lane l: nr x (A, S[, G]) weight planes, then one run of
+      // records per token (chunk slot of matrix m, chunk c: m * cmax + c)
+      if (lane < nr * kPlanes) {
         const int m = lane / kPlanes, pl = lane - m * kPlanes;
-        const int64_t mat = static_cast<int64_t>(eidx) * 3 + (GU ? m : 2);
+        const int64_t mat = static_cast<int64_t>(eidx) * 3 + (gu ? m : 2);
         const int64_t slot0 = (static_cast<int64_t>(mt) * nc + c0) * kTileRows;
         if (pl == 0)
-          bulk_g2s_hint(st + P.a + m * CMAX * kTileRows * 16, G.a + mat * G.a_mat + slot0 * 16,
+          bulk_g2s_hint(st + P.a + m * cmax * kTileRows * 16, G.a + mat * G.a_mat + slot0 * 16,
                         nch * kTileRows * 16, &H->full[slot], pol);
         else if (pl == 1)
-          bulk_g2s_hint(st + P.s + m * CMAX * kTileRows * 4, G.s + mat * G.s_mat + slot0, nch * kTileRows * 4,
+          bulk_g2s_hint(st + P.s + m * cmax * kTileRows * 4, G.s + mat * G.s_mat + slot0, nch * kTileRows * 4,
                         &H->full[slot], pol);
         else
-          bulk_g2s_hint(st + P.g + m * CMAX * kTileRows * 8, G.g + mat * G.g_mat + slot0, nch * kTileRows * 8,
+          bulk_g2s_hint(st + P.g + m * cmax * kTileRows * 8, G.g + mat * G.g_mat + slot0, nch * kTileRows * 8,
                         &H->full[slot], pol);
       }
-      // records of the tokens: one copy per token, lanes NR * kPlanes ..
-      auto issue_records = [&](int sl, int cc0) {
-        const int i = lane - NR * kPlanes;
-        if (i >= 0 && i < ntok) {
-          const ActRec *src = GU ? a.ws.xrec + static_cast<int64_t>(row[2 + tok0 + i]) * (D / kChunk) + cc0
-                                 : a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + i) * (a.ws.fmax / kChunk) + cc0;
-          bulk_g2s(smem + P.stage0 + sl * P.stage + P.rec + i * CMAX * static_cast<int>(sizeof(ActRec)), src,
-                   min(sch, cend - cc0) * static_cast<uint32_t>(sizeof(ActRec)), &H->full[sl]);
+      if (!h_ready) {  // down: the expert's h (this token group, all tiles) must be complete
+        bool hok = true;
+        if (lane == 0) {
+          const unsigned *cnt = a.ws.h_done + u * kMaxTokGroups + grp;
+          const unsigned target = static_cast<unsigned>(G.f / kTileRows * kConsWarps);  // every warp of every tile
+          const long long t0 = clock64();
+          while (ld_acquire_u32(cnt) < target) {
+            if (H->abort || static_cast<uint64_t>(clock64() - t0) > a.spin_limit) {
+              hok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
         }
-      };
-      if (waited) {
-        issue_records(slot, c0);
-      } else {
-#pragma unroll
-        for (int q = 0; q < RING; ++q) {
-          pend_slot[q] = q == npend ? slot : pend_slot[q];
-          pend_c0[q] = q == npend ? c0 : pend_c0[q];
-        }
-        ++npend;
+        ok = __shfl_sync(0xffffffffu, hok, 0);
+        __syncwarp();
+        asm volatile("fence.proxy.async.global;" ::: "memory");  // h was written by generic stores
+        h_ready = true;
+      }
+      const int i = lane - nr * kPlanes;
+      if (i >= 0 && i < ntok) {
+        const ActRec *srcr = gu ? a.ws.xrec + static_cast<int64_t>(row[2 + tok0 + i]) * (D / kChunk) + c0
+                                : a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + i) * (a.ws.fmax / kChunk) + c0;
+        // (after a failed h wait the copy still goes out, so that the stage completes and drains)
+        bulk_g2s(st + P.rec + i * cmax * static_cast<int>(sizeof(ActRec)), srcr, rbytes, &H->full[slot]);
       }
 #pragma unroll
       for (int s = 0; s < RING; ++s) last_round[s] = s == slot ? static_cast<int>(round) : last_round[s];
@@ -985,22 +1004,9 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
         slot = 0;
         ++round;
       }
-      if (!waited && (npend == RING || c0 + sch >= cend)) {
-        griddep_wait();  // the previous kernel's records are complete
-        waited = true;
-#pragma unroll
-        for (int q = 0; q < RING; ++q)
-          if (q < npend) issue_records(pend_slot[q], pend_c0[q]);
-        npend = 0;
-      }
+      if (!ok) break;
     }
     task = __shfl_sync(0xffffffffu, nxt, 0);
-  }
-  if (!waited) {  // no work taken before the wait (or a bad table)
-    griddep_wait();
-#pragma unroll
-    for (int q = 0; q < RING; ++q)
-      if (q < npend) ok = false;  // cannot happen: a task's stages flush before the next task
   }
   // end of work: one more stage, with no copies, tells the consumers to leave
   if (ok && round > 0) ok = ring_wait(H, &H->empty[slot], (round - 1) & 1u, a.spin_limit);
@@ -1013,7 +1019,7 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
       H->info[slot].task = -1;
       mbar_arrive(&H->full[slot]);
     } else {
-      if (n_tasks >= 0) flag_error(a.err, kErrTimeout);
+      if (n_tasks > 0) flag_error(a.err, kErrTimeout);
       H->abort = 1;
     }
     // drain: the last phase armed on each stage has completed before the warp leaves
@@ -1140,6 +1146,12 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
       }
     }
   }
+  // this warp's rows of h are written: count them for the down pieces waiting on the group
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence();
+    atomicAdd(a.ws.h_done + u * kMaxTokGroups + tok0 / kTokGroup, 1u);
+  }
   return true;
 }
 
@@ -1169,10 +1181,10 @@ __device__ __forceinline__ bool dn_finish(const DecodeArgs &a, RingHdr *H, ConsS
   return true;
 }
 
-template <int FMT, bool GU>
+// The consumer warps: stages in ring order; gate/up stages (task below n_gu) take two matrices
+// of two chunks, down stages one matrix of up to four chunks (one K segment).
+template <int FMT>
 __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H) {
-  constexpr int NR = GU ? 2 : 1;
-  constexpr int CMAX = GU ? kGuStageChunks : kDnStageChunks;
   constexpr int RING = ring_depth(FMT);
   const int r = threadIdx.x, lane = r & 31;
   const int D = a.sh.d, TD = D / kTileRows;
@@ -1195,10 +1207,11 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
     }
     const StageInfo in = H->info[slot];
     if (in.task < 0) return;
-    const int pieces = info_pieces(in.flags);
+    const bool gu = in.task < H->n_gu;
+    const int pieces = info_pieces(in.flags), tok0 = info_tok0(in.flags);
     if ((in.flags & kPieceStart) && pieces == 1) {
 #pragma unroll
-      for (int m = 0; m < NR; ++m)
+      for (int m = 0; m < 2; ++m)
 #pragma unroll
         for (int t = 0; t < kUnitTok; ++t) H->tot[m][t][r] = 0.f;
     }
@@ -1208,30 +1221,35 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
 #pragma unroll
         for (int t = 0; t < kUnitTok; ++t) seg[m][t] = 0.f;
     }
-    gemv_dispatch<FMT, NR, CMAX>(in.ntok, smem + P.stage0 + slot * P.stage, P, in.nch, smem_u32(tab), seg);
+    const unsigned char *st = smem + P.stage0 + slot * P.stage;
+    if (gu)
+      gemv_dispatch<FMT, 2, kGuStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), seg);
+    else
+      gemv_dispatch<FMT, 1, kDnStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), seg);
     __syncwarp();
     if (lane == 0) mbar_arrive(&H->empty[slot]);
     if (in.flags & kSegEnd) {
+      const int nr = gu ? 2 : 1;
       if (pieces > 1) {
         // segment sum of a split unit -> partial buffer [segment][matrix][token][row]
-        float *part = GU ? a.ws.gu_part + (static_cast<int64_t>(in.u * a.ws.tmax + in.mt) * a.ws.gu_nseg + in.seg) *
+        float *part = gu ? a.ws.gu_part + (static_cast<int64_t>(in.u * a.ws.tmax + in.mt) * a.ws.gu_nseg + in.seg) *
                                               2 * kPartStride
                          : a.ws.dn_part + (static_cast<int64_t>(in.u * TD + in.mt) * a.ws.dn_nseg + in.seg) * kPartStride;
 #pragma unroll
-        for (int m = 0; m < NR; ++m)
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
           for (int t = 0; t < kUnitTok; ++t)
-            if (t < in.ntok) part[m * kPartStride + (info_tok0(in.flags) + t) * kTileRows + r] = seg[m][t];
+            if (m < nr && t < in.ntok) part[m * kPartStride + (tok0 + t) * kTileRows + r] = seg[m][t];
       } else {
 #pragma unroll
-        for (int m = 0; m < NR; ++m)
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
           for (int t = 0; t < kUnitTok; ++t)
-            if (t < in.ntok) H->tot[m][t][r] += seg[m][t];
+            if (m < nr && t < in.ntok) H->tot[m][t][r] += seg[m][t];
       }
     }
     if (in.flags & kPieceEnd) {
-      const bool ok = GU ? gu_finish<FMT>(a, H, cs, in) : dn_finish(a, H, cs, in);
+      const bool ok = gu ? gu_finish<FMT>(a, H, cs, in) : dn_finish(a, H, cs, in);
       if (!ok) {
         cons_fail(a, H);
         return;
@@ -1244,10 +1262,13 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
   }
 }
 
-template <int FMT, bool GU>
+// One persistent kernel for the expert GEMVs of a layer: gate/up + SwiGLU (h quantised into
+// records), then down.  Thread block = 4 consumer warps (thread = row of a 128-row tile) + one
+// producer warp; the grid is every resident CTA of the device.
+template <int FMT>
 __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const RingPlan P = ring_plan(FMT, GU ? 2 : 1, GU ? kGuStageChunks : kDnStageChunks, a.ws.umax);
+  const RingPlan P = ring_plan(FMT, 1, kStageSlots, a.ws.umax);
   RingHdr *H = reinterpret_cast<RingHdr *>(smem);
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -1261,11 +1282,11 @@ __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(Deco
   }
   __syncthreads();
   if (threadIdx.x >= kTileRows) {
-    producer<FMT, GU>(a, smem, P, H);
+    producer<FMT>(a, smem, P, H);
   } else {
     griddep_wait();
     if (threadIdx.x == 0) griddep_launch();
-    consumer<FMT, GU>(a, smem, P, H);
+    consumer<FMT>(a, smem, P, H);
   }
 }
 
@@ -1361,10 +1382,8 @@ cudaError_t configure_decode_kernels() {
   if (e != cudaSuccess) return e;
   const void *ks[] = {(const void *)k_route<true>,
                       (const void *)k_route<false>,
-                      (const void *)k_gemv<MOE_FMT_Q2_32, true>,
-                      (const void *)k_gemv<MOE_FMT_CB35_32, true>,
-                      (const void *)k_gemv<MOE_FMT_Q2_32, false>,
-                      (const void *)k_gemv<MOE_FMT_CB35_32, false>};
+                      (const void *)k_gemv<MOE_FMT_Q2_32>,
+                      (const void *)k_gemv<MOE_FMT_CB35_32>};
   for (const void *k : ks) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, k);
@@ -1376,31 +1395,22 @@ cudaError_t configure_decode_kernels() {
   return cudaSuccess;
 }
 
-static int gemv_smem(int fmt, bool gu, int umax) {
-  return ring_plan(fmt, gu ? 2 : 1, gu ? kGuStageChunks : kDnStageChunks, umax).total;
-}
+static int gemv_smem(int fmt, int umax) { return ring_plan(fmt, 1, kStageSlots, umax).total; }
 
-// Persistent grids: SMs x resident CTAs of each GEMV kernel; min_streams = 2 x SMs.
-cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gu, int *grid_dn, int *min_streams) {
+// Persistent grid: SMs x resident CTAs of the GEMV kernel; min_streams = MOE_STREAMS_PER_SM x SMs.
+cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_streams) {
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  int occ_gu = 0, occ_dn = 0;
-  const int sg = gemv_smem(fmt, true, umax), sd = gemv_smem(fmt, false, umax);
-  if (fmt == MOE_FMT_Q2_32) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_gu, k_gemv<MOE_FMT_Q2_32, true>, kGemvThreads, sg);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_dn, k_gemv<MOE_FMT_Q2_32, false>, kGemvThreads, sd);
-  } else {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_gu, k_gemv<MOE_FMT_CB35_32, true>, kGemvThreads, sg);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_dn, k_gemv<MOE_FMT_CB35_32, false>, kGemvThreads, sd);
-  }
+  int occ = 0;
+  const int sm = gemv_smem(fmt, umax);
+  e = fmt == MOE_FMT_Q2_32
+          ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<MOE_FMT_Q2_32>, kGemvThreads, sm)
+          : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<MOE_FMT_CB35_32>, kGemvThreads, sm);
   if (e != cudaSuccess) return e;
-  if (occ_gu < 1 || occ_dn < 1) return cudaErrorInvalidConfiguration;
-  *grid_gu = nsm * occ_gu;
-  *grid_dn = nsm * occ_dn;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  *grid_gemv = nsm * occ;
   *min_streams = MOE_STREAMS_PER_SM * nsm;
   return cudaSuccess;
 }
@@ -1418,22 +1428,18 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     rec(a, kProfRoute, 1, st);
   }
-  // 2. gate/up + SwiGLU (persistent)
+  // 2. gate/up + SwiGLU, then down (one persistent kernel)
   {
-    const int sm = gemv_smem(a.sh.fmt, true, a.ws.umax);
+    const int sm = gemv_smem(a.sh.fmt, a.ws.umax);
     rec(a, kProfGateUp, 0, st);
-    err = a.sh.fmt == MOE_FMT_Q2_32 ? launch_pdl(k_gemv<MOE_FMT_Q2_32, true>, a.ws.grid_gu, kGemvThreads, sm, st, a)
-                                    : launch_pdl(k_gemv<MOE_FMT_CB35_32, true>, a.ws.grid_gu, kGemvThreads, sm, st, a);
+    err = a.sh.fmt == MOE_FMT_Q2_32 ? launch_pdl(k_gemv<MOE_FMT_Q2_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a)
+                                    : launch_pdl(k_gemv<MOE_FMT_CB35_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a);
     if (err != cudaSuccess) return err;
     rec(a, kProfGateUp, 1, st);
   }
-  // 3. down + combine (persistent)
+  // 3. weighted combine
   {
-    const int sm = gemv_smem(a.sh.fmt, false, a.ws.umax);
     rec(a, kProfDown, 0, st);
-    err = a.sh.fmt == MOE_FMT_Q2_32 ? launch_pdl(k_gemv<MOE_FMT_Q2_32, false>, a.ws.grid_dn, kGemvThreads, sm, st, a)
-                                    : launch_pdl(k_gemv<MOE_FMT_CB35_32, false>, a.ws.grid_dn, kGemvThreads, sm, st, a);
-    if (err != cudaSuccess) return err;
     err = launch_pdl(k_combine, a.n * (a.sh.d / kCombineThreads), kCombineThreads, 0, st, a);
     if (err != cudaSuccess) return err;
     rec(a, kProfDown, 1, st);

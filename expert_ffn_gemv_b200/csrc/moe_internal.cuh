@@ -105,7 +105,8 @@ struct DecodeWs {
   unsigned *group_ticket;   // [ceil(E/32)]
   unsigned *gu_ticket;      // [umax][tmax][4 token groups]
   unsigned *dn_ticket;      // [umax][D/128][4 token groups]
-  unsigned *counters;       // [2] work queues of the gate/up and down kernels
+  unsigned *counters;       // [2] work queue of the GEMV kernel (gate/up pieces, then down pieces)
+  unsigned *h_done;         // [umax][4 token groups] (tile, consumer warp) pairs that wrote h
   int umax;
   int tmax;             // max(F, F_shared) / 128
   int fmax;
@@ -113,8 +114,7 @@ struct DecodeWs {
   int gu_seg;           // gate/up: chunks per K segment (2 or 4)
   int gu_nseg;          // gate/up: K segments (d_model / 64 / gu_seg)
   int dn_nseg;          // down: most K segments of any expert
-  int grid_gu;          // persistent grids of the GEMV kernels
-  int grid_dn;
+  int grid_gemv;        // persistent grid of the GEMV kernel
   int min_streams;      // pieces wanted in flight (about two per SM)
 };
 
@@ -271,12 +271,12 @@ struct DecodeArgs {
 
 // kernel classes of the per-kernel event timing
 constexpr int kProfRoute = 0;     // router + top-k (+ routing tables / grouping)
-constexpr int kProfGateUp = 1;    // gate/up GEMV or GEMM + SwiGLU
-constexpr int kProfDown = 2;      // down GEMV or GEMM + combine
+constexpr int kProfGateUp = 1;    // the GEMV kernel (gate/up + SwiGLU + down) or the gate/up GEMM + SwiGLU
+constexpr int kProfDown = 2;      // the combine kernel or the down GEMM + combine
 constexpr int kProfKinds = 3;
 
 cudaError_t configure_decode_kernels();
-cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gu, int *grid_dn, int *min_streams);
+cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_streams);
 int route_smem_bytes(int n_experts);
 cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_wait_test(unsigned *never_set, uint32_t *err, uint64_t spin_limit, cudaStream_t st);

@@ -140,7 +140,9 @@ uint64_t moe_device_bytes(const moe_handle *h);
  * (bit k of `on` selects class k; such events are captured into a CUDA graph like the kernels).
  * moe_profile_read sums, over the layers run since profiling was (re-)enabled, the durations
  * recorded by the latest call that ran each layer, for one kernel class -- 0: router + top-k
- * (+ grouping), 1: gate/up + SwiGLU, 2: down + combine -- and returns how many layers
+ * (+ grouping); 1: the expert matrices (1-8 tokens: the one GEMV kernel that runs gate/up +
+ * SwiGLU and down; more tokens: the gate/up GEMM + SwiGLU); 2: what follows (1-8 tokens: the
+ * weighted combine; more tokens: the down GEMM + combine) -- and returns how many layers
  * contributed.  It waits for those events to complete. */
 moe_status moe_profile_enable(moe_handle *h, int32_t on);
 moe_status moe_profile_read(moe_handle *h, int32_t kind, float *total_ms, int32_t *launches);
