@@ -117,7 +117,6 @@ void plan_workspace(moe_handle *h, Carve &c) {
   w.fmax = fmax;
   w.tmax = tmax;
   // router: 256 (else 128) d_model columns per CTA; K segments of 4 (else 2) chunks
-  w.rk_cols = D % 256 == 0 ? 256 : 128;
   const int ncd = D / kChunk;
   w.gu_seg = ncd % 4 == 0 ? 4 : 2;
   w.gu_nseg = ncd / w.gu_seg;
@@ -126,21 +125,19 @@ void plan_workspace(moe_handle *h, Carve &c) {
     w.dn_nseg = nseg(g.d_ff);
     if (g.n_shared && nseg(g.shared_d_ff) > w.dn_nseg) w.dn_nseg = nseg(g.shared_d_ff);
   }
-  const int ks = D / w.rk_cols, ngrp = (E + 31) / 32, td = D / kTileRows;
-  w.logit_part = c.take<float>(static_cast<uint64_t>(ks) * kDecodeMaxTokens * E);
+  const int td = D / kTileRows;
   w.logits = c.take<float>(static_cast<uint64_t>(kDecodeMaxTokens) * E);
+  w.sel = c.take<int>(kDecodeMaxTokens * K);
+  w.route_sync = c.take<unsigned>(2);
   w.route_idx = c.take<int>(kDecodeMaxTokens * K);
   w.route_w = c.take<float>(kDecodeMaxTokens * K);
   w.slotpos = c.take<int>(kDecodeMaxTokens * K);
-  w.task_tab = c.take<int>(4 + static_cast<uint64_t>(umax) * 16);
   w.xrec = c.take<ActRec>(static_cast<uint64_t>(kDecodeMaxTokens) * ncd);
   const uint64_t hrows = static_cast<uint64_t>(umax) * kDecodeMaxTokens;
   w.hrec = c.take<ActRec>(hrows * (fmax / kChunk));
   w.gu_part = c.take<float>(static_cast<uint64_t>(umax) * tmax * w.gu_nseg * 2 * kDecodeMaxTokens * kTileRows);
   w.dn_part = c.take<float>(static_cast<uint64_t>(umax) * td * w.dn_nseg * kDecodeMaxTokens * kTileRows);
   w.o = c.take<float>(hrows * D);
-  w.route_ticket = c.take<unsigned>(1);
-  w.group_ticket = c.take<unsigned>(ngrp);
   w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * 4);  // x token groups of a unit
   w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td * 4);
   w.counters = c.take<unsigned>(2);
@@ -161,11 +158,10 @@ moe_status check_device_error(moe_handle *h, cudaStream_t st) {
   // a kernel that gave up may have left arrival counters set: clear them
   const DecodeWs &w = h->dws;
   const int td = h->cfg.d_model / kTileRows;
-  cudaMemsetAsync(w.route_ticket, 0, sizeof(unsigned), st);
-  cudaMemsetAsync(w.group_ticket, 0, sizeof(unsigned) * ((h->cfg.n_experts + 31) / 32), st);
   cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax * 4, st);
   cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td * 4, st);
   cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * 2, st);
+  cudaMemsetAsync(w.route_sync, 0, sizeof(unsigned) * 2, st);
   cudaMemsetAsync(w.h_done, 0, sizeof(unsigned) * w.umax * 4, st);
   if (e & kErrTimeout) return fail(h, MOE_ERR_TIMEOUT, "a device-side bounded wait ran out");
   return fail(h, MOE_ERR_DEVICE_FAULT, "a device-side check found an invalid routing index");

@@ -1,25 +1,28 @@
 // decode.cu -- the dequant-fused GEMV path for 1..8 tokens (decode steps and 1 + 7 token
 // verify batches of the routed-MoE pages: strata-mlx README, "Draft and verify").
 //
-// Three kernels per layer, all on CUDA cores:
-//   k_route   router GEMV over all experts: lane = expert, the tokens' activations broadcast
-//             from shared memory, fp32 accumulation; each CTA takes 32 experts x one K slice,
-//             the last CTA of a 32-expert group adds the slices in slice order.  The CTAs of
-//             group 0 also quantise the layer input into activation records (int16 + block
-//             sums + a power-of-two factor per 128 columns).  The last group to finish takes
-//             the top-k (warp per token, argmax by warp reductions over order-preserving keys),
-//             the fp32 softmax over the selected logits and builds the active-expert tables.
-//   k_gateup  persistent.  A producer warp takes pieces (active expert, 128-row tile, run of K
-//             segments) from a work queue and bulk-copies (cp.async.bulk) the gate and up rows
-//             of the piece straight from their low-bit planes, with the activation records of
-//             the expert's tokens, into a ring of shared-memory stages; four consumer warps
-//             (thread = row) unpack the codes with two ALU ops per four weights and multiply
-//             them with the int16 activations by dp2a (int16 x int8 -> int32).  The exact
-//             integer block sums are scaled by the fp16 block scale into fp32 sums, one per K
-//             segment; the segment sums are added in segment order.  The unit's last piece
-//             applies SwiGLU and quantises h per (token, 128-row tile) into records.
-//   k_down    the same over h -> o rows; the last expert to finish a 128-column tile of the
-//             output sums y = sum_j w_j o_j + o_shared (+ x) over it, slots in a fixed order.
+// Three kernels per layer, all on CUDA cores, chained by programmatic dependent launches:
+//   k_route    router GEMV: CTA = 4 experts, warp = (expert, half of d_model), fp32 sums over
+//              the whole d_model (no cross-CTA reduction), logits + bias to global memory.  The
+//              CTAs also quantise the layer input into activation records (int16 + block sums +
+//              a power-of-two factor per 128 columns).
+//   k_gemv     persistent, one CTA per resident slot.  Every CTA first takes the top-k of each
+//              token from the logits (warp per token, argmax by warp reductions over
+//              order-preserving keys), the fp32 softmax over the selected logits, and builds the
+//              active-expert task table in its own shared memory (all CTAs build the same
+//              table; CTA 0 also writes the routing outputs).  Then a producer warp takes
+//              pieces (active expert, 128-row tile, token group, run of K segments) from one
+//              work queue -- gate/up pieces first, then down pieces -- and bulk-copies
+//              (cp.async.bulk) the rows of the piece straight from their low-bit planes, with
+//              the activation records of the unit's tokens, into a ring of shared-memory
+//              stages; four consumer warps (thread = row) unpack the codes with one ALU op per
+//              four weights and multiply them with the int16 activations by dp2a (int16 x int8
+//              -> int32).  The exact integer block sums are scaled by the fp16 block scale into
+//              fp32 sums, one per K segment; segment sums are added in segment order.  A gate/up
+//              unit's last piece applies SwiGLU and quantises h per (token, 128-row tile) into
+//              records and counts the tile on its (expert, token group); a down piece issues
+//              its weight copies at once and its h copies once that count is complete.
+//   k_combine  y = sum_j w_j o_j + o_shared (+ x), slots in descending-logit order.
 // No fp32 atomics, and the K segments are fixed by the matrix shapes: results are
 // bit-reproducible and independent of which tokens share a call and of how the work queue
 // split the units among CTAs.
@@ -33,8 +36,8 @@ namespace moe {
 
 constexpr int kRouteWarps = 8;
 constexpr int kRouteThreads = 32 * kRouteWarps;
-constexpr int kRouteExperts = 32;               // experts per router CTA: lane = expert
-constexpr int kRouteMaxCols = 256;              // d_model columns per router CTA (at most)
+constexpr int kRouteExperts = kRouteWarps / 2;   // experts per router CTA: two warps (K halves) each
+constexpr int kRouteMaxG = kDecodeMaxD / 16 / 32;  // 8-column groups of a router lane (at most)
 constexpr int kQGroup = 128;                    // columns sharing one activation factor
 constexpr int kConsWarps = kTileRows / 32;      // consumer warps: thread = row of the tile
 constexpr int kGemvThreads = kTileRows + 32;    // + one producer warp
@@ -122,13 +125,14 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 }
 
 // fp32 softmax over the K selected logits (lane j holds the j-th), results to the tables
-__device__ __forceinline__ void softmax_store(const DecodeArgs &a, int t, int lane, float my_l, float l0, int my_i) {
+__device__ __forceinline__ void softmax_store(const DecodeArgs &a, int t, int lane, float my_l, float l0, int my_i,
+                                              bool wr) {
   const int K = a.sh.k;
   float w = lane < K ? __expf(my_l - l0) : 0.f;
   float sum = w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane < K) {
+  if (wr && lane < K) {
     w = w / sum;
     a.ws.route_idx[t * K + lane] = my_i;
     a.ws.route_w[t * K + lane] = w;
@@ -160,48 +164,154 @@ __device__ __forceinline__ void lane_argmax(const uint32_t (&key)[VPL], uint32_t
   bq = q[0];
 }
 
-// Top-k of token t by one warp, logits in registers (lane l holds experts l + 32 q).  Each lane
-// keeps its best key; a round takes the largest by a warp max-reduction and, among the lanes
-// holding it, the lowest expert index by a min-reduction (the order of repeated strict maxima,
-// ties to the lower index); only the winning lane clears that key and rescans its own keys.
-template <int VPL>
-__device__ __forceinline__ void topk_regs(const DecodeArgs &a, int t, int lane, int *s_idx) {
+// Top-k of NT tokens by one warp, logits in registers (lane l holds experts l + 32 q); the NT
+// tokens' rounds interleave.  Each lane keeps its best key; a round takes the largest by a warp
+// max-reduction and, among the lanes holding it, the lowest expert index by a min-reduction (the
+// order of repeated strict maxima, ties to the lower index); the winning lane clears that key
+// and every lane rescans its keys (selects only, so a round has no divergent branch).
+template <int VPL, int NT>
+__device__ __forceinline__ void topk_regs(const DecodeArgs &a, const int (&t)[NT], int lane, int *s_idx, bool wr) {
   const int E = a.sh.e, K = a.sh.k;
-  float lv[VPL];  // all loads first (in-range index), then the keys
+  uint32_t key[NT][VPL];
+  {
+    float lv[NT][VPL];  // all loads first (in-range index), then the keys
 #pragma unroll
-  for (int q = 0; q < VPL; ++q) lv[q] = __ldcg(a.ws.logits + t * E + min(lane + 32 * q, E - 1));
-  uint32_t key[VPL];
+    for (int i = 0; i < NT; ++i)
 #pragma unroll
-  for (int q = 0; q < VPL; ++q) key[q] = lane + 32 * q < E ? order_key(lv[q]) : 0u;
-  uint32_t lb;
-  int lq;
-  lane_argmax<VPL>(key, lb, lq);
-  float my_l = 0.f, l0 = 0.f;
-  int my_i = 0;
+      for (int q = 0; q < VPL; ++q) lv[i][q] = __ldcg(a.ws.logits + t[i] * E + min(lane + 32 * q, E - 1));
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) key[i][q] = lane + 32 * q < E ? order_key(lv[i][q]) : 0u;
+  }
+  uint32_t lb[NT];
+  int lq[NT];
+  float my_l[NT], l0[NT];
+  int my_i[NT];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    lane_argmax<VPL>(key[i], lb[i], lq[i]);
+    my_l[i] = l0[i] = 0.f;
+    my_i[i] = 0;
+  }
   for (int j = 0; j < K; ++j) {
-    const uint32_t m = __reduce_max_sync(0xffffffffu, lb);
-    int bi = __reduce_min_sync(0xffffffffu, lb == m ? lane + 32 * lq : INT_MAX);
-    float bv = key_value(m);
-    if (bi >= E || !(bv > -INFINITY)) {  // only non-finite logits left
-      if (lane == 0) flag_error(a.err, kErrBadIndex);
-      bi = j;
-      bv = 0.f;
-    }
-    if ((bi & 31) == lane) {  // the winner: clear the key (selects, not an indexed store), rescan
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const uint32_t m = __reduce_max_sync(0xffffffffu, lb[i]);
+      int bi = __reduce_min_sync(0xffffffffu, lb[i] == m ? lane + 32 * lq[i] : INT_MAX);
+      float bv = key_value(m);
+      if (bi >= E || !(bv > -INFINITY)) {  // only non-finite logits left
+        if (lane == 0) flag_error(a.err, kErrBadIndex);
+        bi = j;
+        bv = 0.f;
+      }
+      const bool win = (bi & 31) == lane;
       const int qb = bi >> 5;
 #pragma unroll
-      for (int q = 0; q < VPL; ++q) key[q] = q == qb ? 0u : key[q];
-      lane_argmax<VPL>(key, lb, lq);
+      for (int q = 0; q < VPL; ++q) key[i][q] = (win && q == qb) ? 0u : key[i][q];
+      lane_argmax<VPL>(key[i], lb[i], lq[i]);
+      if (j == 0) l0[i] = bv;
+      if (lane == j) {
+        my_l[i] = bv;
+        my_i[i] = bi;
+      }
+      if (lane == 0) s_idx[t[i] * K + j] = bi;
     }
-    if (j == 0) l0 = bv;
-    if (lane == j) { my_l = bv; my_i = bi; }
-    if (lane == 0) s_idx[t * K + j] = bi;
   }
-  softmax_store(a, t, lane, my_l, l0, my_i);
+#pragma unroll
+  for (int i = 0; i < NT; ++i) softmax_store(a, t[i], lane, my_l[i], l0[i], my_i[i], wr);
+}
+
+// Top-k of token t by one warp from a rank count (no per-selection rounds): with lane l holding
+// experts l + 32 q, T = the K-th largest of the 32 lane maxima bounds the K-th largest key from
+// below (K lane maxima are >= T), so the top K are among the keys >= T.  Those candidates are
+// compacted into the warp's scratch and each one's rank is counted against all of them
+// (descending key, ties to the lower expert index: the order of the round-based pass).
+// Returns false (uniform over the warp) when there are more than kTopkCand candidates or fewer
+// than K valid ones (equal or non-finite logits); the caller then runs the round-based pass.
+constexpr int kTopkCand = 64;
+constexpr int kTopkScratch = 32 + 2 * kTopkCand + 2 * kMaxTopK;  // 32-bit words per warp
+
+template <int VPL>
+__device__ __forceinline__ bool topk_rank(const DecodeArgs &a, int t, int lane, int *s_idx, bool wr, uint32_t *ws) {
+  const int E = a.sh.e, K = a.sh.k;
+  uint32_t key[VPL];
+  {
+    float lv[VPL];
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) lv[q] = __ldcg(a.ws.logits + t * E + min(lane + 32 * q, E - 1));
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) key[q] = lane + 32 * q < E ? order_key(lv[q]) : 0u;
+  }
+  uint32_t mk = key[0];
+#pragma unroll
+  for (int q = 1; q < VPL; ++q) mk = max(mk, key[q]);
+  ws[lane] = mk;
+  __syncwarp();
+  int r = 0;
+#pragma unroll 8
+  for (int l = 0; l < 32; ++l) {
+    const uint32_t o = ws[l];
+    r += (o > mk) || (o == mk && l < lane);
+  }
+  const uint32_t T = __shfl_sync(0xffffffffu, mk, __ffs(__ballot_sync(0xffffffffu, r == K - 1)) - 1);
+  int c = 0;
+#pragma unroll
+  for (int q = 0; q < VPL; ++q) c += (key[q] >= T && lane + 32 * q < E) ? 1 : 0;
+  int inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  const int C = __shfl_sync(0xffffffffu, inc, 31);
+  if (C > kTopkCand || C < K) return false;
+  uint32_t *ck = ws + 32, *ci = ck + kTopkCand;
+  float *sv = reinterpret_cast<float *>(ci + kTopkCand);
+  int *si = reinterpret_cast<int *>(sv + kMaxTopK);
+  int o = inc - c;
+#pragma unroll
+  for (int q = 0; q < VPL; ++q)
+    if (key[q] >= T && lane + 32 * q < E) {
+      ck[o] = key[q];
+      ci[o] = lane + 32 * q;
+      ++o;
+    }
+  __syncwarp();
+  for (int i = lane; i < C; i += 32) {
+    const uint32_t ki = ck[i];
+    const int ei = static_cast<int>(ci[i]);
+    int rk = 0;
+    for (int j = 0; j < C; ++j) {
+      const uint32_t kj = ck[j];
+      rk += (kj > ki) || (kj == ki && static_cast<int>(ci[j]) < ei);
+    }
+    if (rk < K) {
+      sv[rk] = key_value(ki);
+      si[rk] = ei;
+    }
+  }
+  __syncwarp();
+  float my_l = 0.f;
+  int my_i = 0;
+  if (lane < K) {
+    my_l = sv[lane];
+    my_i = si[lane];
+    if (!(my_l > -INFINITY)) {  // a non-finite logit was selected
+      flag_error(a.err, kErrBadIndex);
+      my_l = 0.f;
+      my_i = lane;
+    }
+    s_idx[t * K + lane] = my_i;
+  }
+  const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
+  softmax_store(a, t, lane, my_l, l0, my_i, wr);
+  __syncwarp();  // the scratch is reused by the warp's next token
+  return true;
 }
 
 // Top-k of token t by one warp over logits in shared memory (more than 1,024 experts).
-__device__ __forceinline__ void topk_smem(const DecodeArgs &a, int t, int lane, float *row, int *s_idx) {
+__device__ __forceinline__ void topk_smem(const DecodeArgs &a, int t, int lane, float *row, int *s_idx, bool wr) {
   const int E = a.sh.e, K = a.sh.k;
   for (int i = lane; i < E; i += 32) row[i] = __ldcg(a.ws.logits + t * E + i);
   __syncwarp();
@@ -229,15 +339,25 @@ __device__ __forceinline__ void topk_smem(const DecodeArgs &a, int t, int lane, 
     if (lane == 0) { row[bi] = -INFINITY; s_idx[t * K + j] = bi; }
     __syncwarp();
   }
-  softmax_store(a, t, lane, my_l, l0, my_i);
+  softmax_store(a, t, lane, my_l, l0, my_i, wr);
+}
+
+// floor(a / b) for 0 <= a < 2^24, 1 <= b < 2^24: the fast float quotient is within one of the
+// exact one, and the remainder corrects it.
+__device__ __forceinline__ int udiv_small(int a, int b) {
+  int q = static_cast<int>(__fdividef(static_cast<float>(a), static_cast<float>(b)));
+  const int r = a - q * b;
+  q += r >= b ? 1 : 0;
+  q -= r < 0 ? 1 : 0;
+  return q;
 }
 
 // Pieces per unit: K is cut only when there are fewer units than about min_streams (e.g. one
 // token's ~11 experts), so that enough pieces are in flight.  Returns the run length in segments.
 __device__ __forceinline__ int piece_run(int nseg, int units_total, int min_streams) {
-  int p = (min_streams + units_total - 1) / units_total;
+  int p = udiv_small(min_streams + units_total - 1, units_total);
   p = min(max(p, 1), nseg);
-  return (nseg + p - 1) / p;
+  return udiv_small(nseg + p - 1, p);
 }
 
 // Token groups of an active expert: an expert serving three or more tokens is cut into groups of
@@ -256,9 +376,9 @@ __host__ __device__ inline int tok_group_size(int ntok) { return ntok >= 3 ? kTo
 // pieces of `len` segments.  Returns the packed split; `pieces` the number of pieces.
 __device__ __forceinline__ int unit_split(int nc, int units_total, int min_streams, int &pieces) {
   const int seg = nc % 4 == 0 ? 4 : 2;
-  const int nseg = nc / seg;
+  const int nseg = seg == 4 ? nc >> 2 : nc >> 1;
   const int len = piece_run(nseg, units_total, min_streams);
-  pieces = (nseg + len - 1) / len;
+  pieces = udiv_small(nseg + len - 1, len);
   return len | (pieces << 8) | (seg << 16) | (nseg << 20);
 }
 
@@ -266,30 +386,39 @@ constexpr int kTabHead = 4;    // ints before the first row of the task table
 constexpr int kTabInts = 16;   // ints per active expert
 constexpr int kMaxActive = kDecodeMaxTokens * kMaxTopK + 1;
 
-template <bool RBF16>
-__global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ __align__(16) float xs[kDecodeMaxTokens][kRouteMaxCols];
-  __shared__ float red[kRouteWarps][kDecodeMaxTokens][32];
-  __shared__ int s_idx[kDecodeMaxTokens * kMaxTopK];
-  __shared__ int s_wsum[kRouteWarps];
-  __shared__ int s_cnt[2][kMaxActive];
-  __shared__ int s_units[2];
-  __shared__ int s_last;
-  const int D = a.sh.d, E = a.sh.e, n = a.n;
-  const int CK = a.ws.rk_cols, KS = D / CK;
-  const int grp = blockIdx.x / KS, ks = blockIdx.x - grp * KS, ngrp = gridDim.x / KS;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c0 = ks * CK;
-  // this CTA's router weights (written by no kernel) load while the previous kernel finishes
-  const int re0 = grp * kRouteExperts + lane;  // lane = expert
-  const int cw = CK / kRouteWarps, cb = warp * cw;  // warp = CK/8 columns of the slice
-  float w[4][8];
-  if (re0 < E) {
+template <bool XBF16>
+__device__ __forceinline__ void load_x8(const void *x, int64_t off, float (&v)[8]) {
+  if (XBF16) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + off));
+    const uint32_t p[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (8 * i < cw) load_row8<RBF16>(a.L.router_w, static_cast<int64_t>(re0) * D + c0 + cb + 8 * i, w[i]);
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(p[i] << 16);
+      v[2 * i + 1] = __uint_as_float(p[i] & 0xFFFF0000u);
+    }
+  } else {
+    const float4 *f = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + off);
+    const float4 a = __ldg(f), b = __ldg(f + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
+}
+
+// Router logits l = W_r x + b for kRouteExperts experts per CTA (fp32 sums over the whole
+// d_model: lane = 8-column groups of one half, then the two halves in order), and the
+// activation records of the n tokens (warp per (token, 128-column group)).
+template <bool RBF16, bool XBF16>
+__global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
+  __shared__ float red[kRouteWarps][kDecodeMaxTokens];
+  const int D = a.sh.d, E = a.sh.e, n = a.n;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int e = blockIdx.x * kRouteExperts + (warp >> 1), c0 = (warp & 1) * (D / 2);
+  const int G = D / 16;  // 8-column groups per half
+  // this warp's half router row (written by no kernel) loads while the previous kernel finishes
+  float w[kRouteMaxG][8];
+#pragma unroll
+  for (int i = 0; i < kRouteMaxG; ++i)
+    if (e < E && lane + 32 * i < G) load_row8<RBF16>(a.L.router_w, static_cast<int64_t>(e) * D + c0 + 8 * (lane + 32 * i), w[i]);
   griddep_wait();
   griddep_launch();
   // the work queue and the h counters of this layer's GEMV kernel start empty (the previous
@@ -299,146 +428,174 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
     for (int i = tid; i < a.ws.umax * kMaxTokGroups; i += kRouteThreads) a.ws.h_done[i] = 0u;
   }
 
-  // ---- the K slice of the n tokens, as fp32
-  if (a.x_bf16) {
-    const int per = CK / 8;
-    for (int v = tid; v < n * per; v += kRouteThreads) {
-      const int t = v / per, j = v - t * per;
-      const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) +
-                                                            static_cast<int64_t>(t) * D + c0) + j);
-      float4 lo, hi;
-      lo.x = __uint_as_float(q.x << 16); lo.y = __uint_as_float(q.x & 0xFFFF0000u);
-      lo.z = __uint_as_float(q.y << 16); lo.w = __uint_as_float(q.y & 0xFFFF0000u);
-      hi.x = __uint_as_float(q.z << 16); hi.y = __uint_as_float(q.z & 0xFFFF0000u);
-      hi.z = __uint_as_float(q.w << 16); hi.w = __uint_as_float(q.w & 0xFFFF0000u);
-      *reinterpret_cast<float4 *>(&xs[t][8 * j]) = lo;
-      *reinterpret_cast<float4 *>(&xs[t][8 * j + 4]) = hi;
-    }
-  } else {
-    const int per = CK / 4;
-    for (int v = tid; v < n * per; v += kRouteThreads) {
-      const int t = v / per, j = v - t * per;
-      *reinterpret_cast<float4 *>(&xs[t][4 * j]) =
-          __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + static_cast<int64_t>(t) * D + c0) + j);
-    }
-  }
-  __syncthreads();
-
-  // ---- input quantisation (group 0): warp per (token, 128-column group), lane = 4 columns
-  if (grp == 0) {
-    const int qpt = CK / kQGroup;
-    for (int p = warp; p < n * qpt; p += kRouteWarps) {
+  // ---- activation records: warp per (token, 128-column group), lane = 4 columns
+  {
+    const int qpt = D / kQGroup;
+    for (int p = blockIdx.x * kRouteWarps + warp; p < n * qpt; p += gridDim.x * kRouteWarps) {
       const int t = p / qpt, qg = p - t * qpt;
-      const float4 v = *reinterpret_cast<const float4 *>(&xs[t][qg * kQGroup + 4 * lane]);
+      const int64_t i0 = static_cast<int64_t>(t) * D + qg * kQGroup + 4 * lane;
+      float4 v;
+      if (XBF16) {
+        const uint2 q = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(a.x) + i0));
+        v = make_float4(__uint_as_float(q.x << 16), __uint_as_float(q.x & 0xFFFF0000u), __uint_as_float(q.y << 16),
+                        __uint_as_float(q.y & 0xFFFF0000u));
+      } else {
+        v = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + i0));
+      }
       float mx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const int e = fix16_exponent(mx);
-      const float sc = pow2f(e);
+      const int ex = fix16_exponent(mx);
+      const float sc = pow2f(ex);
       const int q0 = fix16(v.x, sc), q1 = fix16(v.y, sc), q2 = fix16(v.z, sc), q3 = fix16(v.w, sc);
-      ActRec *rec = a.ws.xrec + static_cast<int64_t>(t) * (D / kChunk) + (c0 + qg * kQGroup) / kChunk + (lane >> 4);
+      ActRec *rec = a.ws.xrec + static_cast<int64_t>(t) * (D / kChunk) + (qg * kQGroup) / kChunk + (lane >> 4);
       *reinterpret_cast<uint2 *>(&rec->x[(4 * lane) & 63]) =
           make_uint2((static_cast<uint32_t>(q0) & 0xFFFFu) | (static_cast<uint32_t>(q1) << 16),
                      (static_cast<uint32_t>(q2) & 0xFFFFu) | (static_cast<uint32_t>(q3) << 16));
-      int s = q0 + q1 + q2 + q3;  // eight lanes = one 32-column block
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s += __shfl_xor_sync(0xffffffffu, s, 4);
-      if ((lane & 7) == 0) rec->m[(lane >> 3) & 1] = a.sh.fmt == MOE_FMT_Q2_32 ? kQ2SumMul * s : s;
+      int sm = q0 + q1 + q2 + q3;  // eight lanes = one 32-column block
+      sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+      if ((lane & 7) == 0) rec->m[(lane >> 3) & 1] = a.sh.fmt == MOE_FMT_Q2_32 ? kQ2SumMul * sm : sm;
       if ((lane & 15) == 0) {
-        rec->f = pow2f(-e) * (a.sh.fmt == MOE_FMT_Q2_32 ? kQ2Factor : 1.0f);
+        rec->f = pow2f(-ex) * (a.sh.fmt == MOE_FMT_Q2_32 ? kQ2Factor : 1.0f);
         rec->pad = 0u;
       }
     }
   }
 
-  // ---- router GEMV: lane = expert, warp = CK/8 columns of the slice
-  {
-    float acc[kDecodeMaxTokens];
+  // ---- router GEMV: every token's x loads are issued before its sums
+  float acc[kDecodeMaxTokens];
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxTokens; ++t) acc[t] = 0.f;
-    if (re0 < E) {
+  for (int t = 0; t < kDecodeMaxTokens; ++t) {
+    acc[t] = 0.f;
+    if (e < E && t < n) {
+      float xv[kRouteMaxG][8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (8 * i < cw) {
+      for (int i = 0; i < kRouteMaxG; ++i)
+        if (lane + 32 * i < G) load_x8<XBF16>(a.x, static_cast<int64_t>(t) * D + c0 + 8 * (lane + 32 * i), xv[i]);
+      float sacc = 0.f;
 #pragma unroll
-          for (int t = 0; t < kDecodeMaxTokens; ++t) {
-            if (t < n) {
-              const float4 x0 = *reinterpret_cast<const float4 *>(&xs[t][cb + 8 * i]);
-              const float4 x1 = *reinterpret_cast<const float4 *>(&xs[t][cb + 8 * i + 4]);
-              float v = acc[t];
-              v = fmaf(w[i][0], x0.x, v); v = fmaf(w[i][1], x0.y, v); v = fmaf(w[i][2], x0.z, v);
-              v = fmaf(w[i][3], x0.w, v); v = fmaf(w[i][4], x1.x, v); v = fmaf(w[i][5], x1.y, v);
-              v = fmaf(w[i][6], x1.z, v); v = fmaf(w[i][7], x1.w, v);
-              acc[t] = v;
-            }
-          }
+      for (int i = 0; i < kRouteMaxG; ++i)
+        if (lane + 32 * i < G) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sacc = fmaf(w[i][j], xv[i][j], sacc);
         }
+      acc[t] = sacc;
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kDecodeMaxTokens; ++t) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int t = 0; t < kDecodeMaxTokens; ++t) red[warp][t] = acc[t];
+  }
+  __syncthreads();
+  if (tid < kRouteExperts * kDecodeMaxTokens) {
+    const int j = tid / kDecodeMaxTokens, t = tid - j * kDecodeMaxTokens, ej = blockIdx.x * kRouteExperts + j;
+    if (t < n && ej < E) a.ws.logits[t * E + ej] = (red[2 * j][t] + red[2 * j + 1][t]) + a.L.bias[ej];
+  }
+
+  // ---- the last m = min(n, CTAs) CTAs to finish take the top-k (warp per token) once every
+  // CTA's logits are written: a CTA holding one of the last tickets waits only for CTAs that took
+  // a ticket after it, which are running, so the bounded wait ends.
+  __shared__ int s_tk;
+  __shared__ __align__(16) uint32_t s_topk[kRouteWarps][kTopkScratch];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_tk = static_cast<int>(atomicAdd(a.ws.route_sync, 1u));
+  __syncthreads();
+  const int m = min(n, static_cast<int>(gridDim.x));
+  const int j = s_tk - (static_cast<int>(gridDim.x) - m);
+  if (j < 0) return;
+  if (tid == 0) {
+    const long long t0 = clock64();
+    while (ld_acquire_u32(a.ws.route_sync) < gridDim.x) {
+      if (static_cast<uint64_t>(clock64() - t0) > a.spin_limit) {
+        flag_error(a.err, kErrTimeout);
+        break;
+      }
+      __nanosleep(32);
+    }
+  }
+  __syncthreads();
+  if (E <= 1024) {
+    for (int t = j + m * warp; t < n; t += m * kRouteWarps) {
+      const int tt[1] = {t};
+      bool done;
+      if (E <= 128) {
+        done = topk_rank<4>(a, t, lane, a.ws.sel, true, s_topk[warp]);
+        if (!done) topk_regs<4, 1>(a, tt, lane, a.ws.sel, true);
+      } else if (E <= 256) {
+        done = topk_rank<8>(a, t, lane, a.ws.sel, true, s_topk[warp]);
+        if (!done) topk_regs<8, 1>(a, tt, lane, a.ws.sel, true);
+      } else if (E <= 512) {
+        done = topk_rank<16>(a, t, lane, a.ws.sel, true, s_topk[warp]);
+        if (!done) topk_regs<16, 1>(a, tt, lane, a.ws.sel, true);
+      } else {
+        done = topk_rank<32>(a, t, lane, a.ws.sel, true, s_topk[warp]);
+        if (!done) topk_regs<32, 1>(a, tt, lane, a.ws.sel, true);
       }
     }
-#pragma unroll
-    for (int t = 0; t < kDecodeMaxTokens; ++t)
-      if (t < n) red[warp][t][lane] = acc[t];
+  } else if (warp == 0) {  // one logit row in dynamic shared memory
+    extern __shared__ __align__(16) unsigned char route_dyn[];
+    for (int t = j; t < n; t += m) topk_smem(a, t, lane, reinterpret_cast<float *>(route_dyn), a.ws.sel, true);
   }
   __syncthreads();
-  const int rt = tid >> 5, re = grp * kRouteExperts + lane;  // thread = (token, expert of the group)
-  if (rt < n && re < E) {
-    float s = red[0][rt][lane];
-#pragma unroll
-    for (int w = 1; w < kRouteWarps; ++w) s += red[w][rt][lane];
-    a.ws.logit_part[(static_cast<int64_t>(ks) * kDecodeMaxTokens + rt) * E + re] = s;
+  if (tid == 0) {  // the last top-k CTA to finish clears the counters for the next layer
+    __threadfence();
+    if (atomicAdd(a.ws.route_sync + 1, 1u) == static_cast<unsigned>(m - 1)) {
+      a.ws.route_sync[0] = 0u;
+      a.ws.route_sync[1] = 0u;
+    }
   }
+}
 
-  // ---- the last CTA of the group adds the K slices in slice order
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(a.ws.group_ticket + grp, 1u) == static_cast<unsigned>(KS - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  if (rt < n && re < E) {
-    float pv[kDecodeMaxD / 128];
-#pragma unroll
-    for (int q = 0; q < kDecodeMaxD / 128; ++q)
-      if (q < KS) pv[q] = __ldcg(a.ws.logit_part + (static_cast<int64_t>(q) * kDecodeMaxTokens + rt) * E + re);
-    float s = 0.f;
-#pragma unroll
-    for (int q = 0; q < kDecodeMaxD / 128; ++q)
-      if (q < KS) s += pv[q];
-    a.ws.logits[rt * E + re] = s + a.L.bias[re];
-  }
-  if (tid == 0) a.ws.group_ticket[grp] = 0u;
+// ------------------------------------------------------------------------------------------
+// routing tables, built by every GEMV CTA in its own shared memory
+// ------------------------------------------------------------------------------------------
+// Scratch (the ring's stage area, unused until the tables exist): tokmask [E] (bit t = token t
+// chose the expert), bitmap and wpre [kMaxExperts / 32] (active experts; active experts before
+// word w), s_idx [8][kMaxTopK], s_cnt [2][kMaxActive], s_misc [4], then one logit row per
+// top-k warp when there are more than 1,024 experts.
+__host__ __device__ constexpr int table_scratch_bytes() {
+  return kMaxExperts * 4 + 2 * (kMaxExperts / 32) * 4 + kDecodeMaxTokens * kMaxTopK * 4 + 2 * kMaxActive * 4 + 16;
+}
 
-  // ---- the last group continues with top-k and the routing tables
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(a.ws.route_ticket, 1u) == static_cast<unsigned>(ngrp - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  const int K = a.sh.k;
-  uint32_t *tokmask = reinterpret_cast<uint32_t *>(smem);  // [E]: bit t = token t chose the expert
-  uint32_t *bitmap = tokmask + E;                          // [E/32]: active experts
-  int *wpre = reinterpret_cast<int *>(bitmap + kMaxExperts / 32);  // [E/32]: active experts before word w
-  float *lg = reinterpret_cast<float *>(wpre + kMaxExperts / 32);  // [n][E] (more than 1,024 experts)
+// Top-k + softmax per token, the active-expert rows (u = 0: the shared expert; routed experts
+// follow in ascending id), K splits and first tasks of each active expert.  Every thread of the
+// CTA calls it; wr: also write the routing outputs (one CTA does).
+__device__ void build_tables(const DecodeArgs &a, unsigned char *scratch, int *tb, bool wr) {
+  constexpr int kThreads = kGemvThreads, kWarps = kGemvThreads / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int D = a.sh.d, E = a.sh.e, K = a.sh.k, n = a.n;
+  uint32_t *tokmask = reinterpret_cast<uint32_t *>(scratch);
+  uint32_t *bitmap = tokmask + E;
+  int *wpre = reinterpret_cast<int *>(bitmap + kMaxExperts / 32);
+  int *s_idx = wpre + kMaxExperts / 32;
+  int *s_cnt = s_idx + kDecodeMaxTokens * kMaxTopK;
+  int *s_misc = s_cnt + 2 * kMaxActive;  // units of gate/up, units of down, routed active
   const int nw = (E + 31) / 32;
-  for (int i = tid; i < E; i += kRouteThreads) tokmask[i] = 0u;
-  for (int i = tid; i < nw; i += kRouteThreads) bitmap[i] = 0u;
-  if (warp < n) {
-    if (E <= 128) topk_regs<4>(a, warp, lane, s_idx);
-    else if (E <= 256) topk_regs<8>(a, warp, lane, s_idx);
-    else if (E <= 512) topk_regs<16>(a, warp, lane, s_idx);
-    else if (E <= 1024) topk_regs<32>(a, warp, lane, s_idx);
-    else topk_smem(a, warp, lane, lg + warp * E, s_idx);
+  for (int i = tid; i < E; i += kThreads) tokmask[i] = 0u;
+  for (int i = tid; i < nw; i += kThreads) bitmap[i] = 0u;
+  if (tid < 4) s_misc[tid] = 0;
+  for (int p = tid; p < n * K; p += kThreads) {  // the router's selections
+    int ex = __ldcg(a.ws.sel + p);
+    if (ex < 0 || ex >= E) {
+      flag_error(a.err, kErrBadIndex);
+      ex = 0;
+    }
+    s_idx[p] = ex;
   }
   __syncthreads();
-  for (int p = tid; p < n * K; p += kRouteThreads) {
+  for (int p = tid; p < n * K; p += kThreads) {
     const int ex = s_idx[p];
     atomicOr(tokmask + ex, 1u << (p / K));
     atomicOr(bitmap + (ex >> 5), 1u << (ex & 31));
   }
-  if (tid == 0) s_units[0] = s_units[1] = 0;
   __syncthreads();
   if (warp == 0) {  // active experts before each bitmap word
     int run = 0;
@@ -454,27 +611,25 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
       if (w < nw) wpre[w] = run + inc - c;
       run += __shfl_sync(0xffffffffu, inc, 31);
     }
-    if (lane == 0) s_wsum[0] = run;
+    if (lane == 0) s_misc[2] = run;
   }
   __syncthreads();
-  // active-expert rows of the task table (u = 0: the shared expert; routed experts follow in
-  // ascending id), written by the thread of each expert's first token, and the combine's slots
+  // rows written by the thread of each expert's first token, and the combine's slots
   const int ns = a.sh.n_shared;
-  const int na = ns + s_wsum[0];
+  const int na = ns + s_misc[2];
   const int TD = D / kTileRows;
-  int *tt = a.ws.task_tab;
   auto rank_of = [&](int e) { return wpre[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u)); };
   int ug = 0, ud = 0;
-  for (int p = tid; p < n * K + ns; p += kRouteThreads) {
+  for (int p = tid; p < n * K + ns; p += kThreads) {
     const bool shared = p == n * K;
     const int t = shared ? 0 : p / K, ex = shared ? E : s_idx[p];
     uint32_t m = shared ? (1u << n) - 1u : tokmask[ex];
     const int u = shared ? 0 : ns + rank_of(ex);
-    if (!shared) a.ws.slotpos[p] = u * kDecodeMaxTokens + __popc(m & ((1u << t) - 1u));
+    if (wr && !shared) a.ws.slotpos[p] = u * kDecodeMaxTokens + __popc(m & ((1u << t) - 1u));
     if (!shared && (m & ((1u << t) - 1u))) continue;  // not the expert's first token
     const int nt = __popc(m), ng = tok_groups(nt);
     const int F = shared ? a.L.shared.f : a.L.routed.f;
-    int *row = tt + kTabHead + u * kTabInts;
+    int *row = tb + kTabHead + u * kTabInts;
     row[0] = ex;
     row[1] = nt;
     row[14] = ng;
@@ -483,29 +638,35 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
       row[2 + c++] = __ffs(m) - 1;
       m &= m - 1u;
     }
-    s_cnt[0][u] = F;   // d_ff of the row, for the split pass
-    s_cnt[1][u] = ng;
+    s_cnt[kMaxActive + u] = ng;
     ug += (F / kTileRows) * ng;
     ud += TD * ng;
   }
-  if (ug) atomicAdd(&s_units[0], ug);
-  if (ud) atomicAdd(&s_units[1], ud);
-  if (a.out_counts)
-    for (int i = tid; i < E; i += kRouteThreads) a.out_counts[i] = __popc(tokmask[i]);
+  if (ug) atomicAdd(&s_misc[0], ug);
+  if (ud) atomicAdd(&s_misc[1], ud);
+  if (wr && a.out_counts)
+    for (int i = tid; i < E; i += kThreads) a.out_counts[i] = __popc(tokmask[i]);
   __syncthreads();
   if (warp == 0) {  // K splits, task counts and first task of each active expert (prefix over u)
+    // a split depends on the unit totals and the matrix's K only: one gate/up split, one down
+    // split per d_ff (routed, shared)
+    int pg, pdr, pds = 0;
+    const int sg = unit_split(D / kChunk, s_misc[0], a.ws.min_streams, pg);
+    const int sdr = unit_split(a.L.routed.f / kChunk, s_misc[1], a.ws.min_streams, pdr);
+    const int sds = ns ? unit_split(a.L.shared.f / kChunk, s_misc[1], a.ws.min_streams, pds) : 0;
+    const int tgr = (a.L.routed.f / kTileRows) * pg, tgs = ns ? (a.L.shared.f / kTileRows) * pg : 0;
     int run0 = 0, run1 = 0;
     for (int u0 = 0; u0 < na; u0 += 32) {
       const int u = u0 + lane;
       int c0v = 0, c1v = 0;
       if (u < na) {
-        const int F = s_cnt[0][u], ng = s_cnt[1][u];
-        int *row = tt + kTabHead + u * kTabInts;
-        int pg, pd;
-        row[11] = unit_split(D / kChunk, s_units[0], a.ws.min_streams, pg);
-        row[13] = unit_split(F / kChunk, s_units[1], a.ws.min_streams, pd);
-        c0v = (F / kTileRows) * ng * pg;
-        c1v = ng * pd;
+        const bool sh = ns && u == 0;
+        const int ng = s_cnt[kMaxActive + u];
+        int *row = tb + kTabHead + u * kTabInts;
+        row[11] = sg;
+        row[13] = sh ? sds : sdr;
+        c0v = (sh ? tgs : tgr) * ng;
+        c1v = ng * (sh ? pds : pdr);
       }
       int i0 = c0v, i1 = c1v;
 #pragma unroll
@@ -517,20 +678,20 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
         }
       }
       if (u < na) {
-        tt[kTabHead + u * kTabInts + 10] = run0 + i0 - c0v;
-        tt[kTabHead + u * kTabInts + 12] = run1 + i1 - c1v;
+        tb[kTabHead + u * kTabInts + 10] = run0 + i0 - c0v;
+        tb[kTabHead + u * kTabInts + 12] = run1 + i1 - c1v;
       }
       run0 += __shfl_sync(0xffffffffu, i0, 31);
       run1 += __shfl_sync(0xffffffffu, i1, 31);
     }
     if (lane == 0) {
-      tt[0] = na;
-      tt[1] = run0;
-      tt[2] = run1;
-      tt[3] = 0;
+      tb[0] = na;
+      tb[1] = run0;
+      tb[2] = run1;
+      tb[3] = 0;
     }
   }
-  if (tid == 0) *a.ws.route_ticket = 0u;
+  __syncthreads();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -649,8 +810,6 @@ struct RingHdr {
   uint64_t empty[kRing];
   uint64_t cbar;  // barrier of the consumer warps (kConsWarps arrivals)
   StageInfo info[kRing];
-  int n_active;
-  int n_gu;        // tasks below n_gu are gate/up pieces, the rest down pieces
   volatile int abort;
   int flag[2];
   float wmax[2][kConsWarps][kUnitTok];
@@ -804,50 +963,6 @@ __device__ __forceinline__ void cons_fail(const DecodeArgs &a, RingHdr *H) {
 }
 
 
-// Load the task table (one round of independent loads) and check it for both GEMVs.  Returns
-// false (uniform over the warp) when an entry is out of range; n_gu / n_dn: the task counts.
-__device__ bool producer_tables(const DecodeArgs &a, RingHdr *H, int *tb, int &n_gu, int &n_dn) {
-  const int lane = threadIdx.x & 31;
-  const int umax = a.ws.umax, E = a.sh.e, D = a.sh.d;
-  const int4 *src = reinterpret_cast<const int4 *>(a.ws.task_tab);
-  int4 *dst = reinterpret_cast<int4 *>(tb);
-  for (int i = lane; i < (kTabHead + kTabInts * umax) / 4; i += 32) dst[i] = __ldcg(src + i);
-  __syncwarp();
-  const int na = tb[0];
-  n_gu = tb[1];
-  n_dn = tb[2] * (D / kTileRows);
-  bool bad = na < 1 || na > umax || tb[1] < 1 || tb[2] < 1;
-  for (int u = lane; !bad && u < na; u += 32) {
-    const int *row = tb + kTabHead + u * kTabInts;
-    const int e = row[0], nt = row[1], ng = row[14];
-    bool b = e < 0 || e > E || (e == E) != (a.sh.n_shared && u == 0) || nt < 1 || nt > kDecodeMaxTokens ||
-             ng != tok_groups(nt);
-    for (int i = 0; !b && i < nt; ++i) b = row[2 + i] < 0 || row[2 + i] >= a.n;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {  // k = 0: gate/up (K = d_model), k = 1: down (K = d_ff)
-      if (b) break;
-      const int F = e == E ? a.L.shared.f : a.L.routed.f;
-      const int nc = (k == 0 ? D : F) / kChunk;
-      const int pk = row[k == 0 ? 11 : 13];
-      const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
-      b = (seg != 2 && seg != 4) || nseg * seg != nc || len < 1 || len > nseg || pieces != (nseg + len - 1) / len;
-      const int cnt = k == 0 ? (F / kTileRows) * ng * pieces : ng * pieces;
-      const int base = row[k == 0 ? 10 : 12];
-      const int next = u + 1 < na ? row[kTabInts + (k == 0 ? 10 : 12)] : tb[1 + k];
-      b = b || base + cnt != next || (u == 0 && base != 0);
-    }
-    bad = b;
-  }
-  bad = __any_sync(0xffffffffu, bad);
-  if (bad) return false;
-  if (lane == 0) {
-    H->n_active = na;
-    H->n_gu = n_gu;
-  }
-  __syncwarp();
-  return true;
-}
-
 // largest u with first-task(u) <= r (first tasks increase with u, first-task(0) = 0)
 template <bool GU>
 __device__ __forceinline__ int find_expert(const int *tb, int na, int r) {
@@ -860,12 +975,6 @@ __device__ __forceinline__ int find_expert(const int *tb, int na, int r) {
   return lo;
 }
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // The producer warp: one work queue of gate/up pieces (tasks < n_gu) then down pieces ->
 // bulk copies into the ring.  A down piece issues its weight copies at once and its h records
 // once every gate/up tile of its expert and token group has written h (a counter the gate/up
@@ -873,28 +982,25 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
 // grid are resident, so that wait always ends.  Every stage the warp arms is waited for
 // (bounded) before it leaves, so no copy is in flight when the CTA exits.
 template <int FMT>
-__device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H) {
+__device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H,
+                                         int first_task) {
   constexpr int RING = ring_depth(FMT);
   constexpr int kPlanes = FMT == MOE_FMT_CB35_32 ? 3 : 2;
   const int lane = threadIdx.x & 31;
   const int D = a.sh.d, E = a.sh.e, TD = D / kTileRows;
-  int *tb = reinterpret_cast<int *>(smem + P.table);
+  const int *tb = reinterpret_cast<const int *>(smem + P.table);
   unsigned *ctr = a.ws.counters;
-  griddep_wait();  // the router kernel's tables
-  int task = 0;
-  if (lane == 0) task = static_cast<int>(atomicAdd(ctr, 1u));  // in flight while the table loads
-  int n_gu = 0, n_dn = 0;
-  bool ok = producer_tables(a, H, tb, n_gu, n_dn);
-  if (!ok && lane == 0) flag_error(a.err, kErrBadIndex);
-  const int n_tasks = ok ? n_gu + n_dn : 0;
-  const int na = ok ? H->n_active : 0;
+  int task = first_task;
+  const int na = tb[0], n_gu = tb[1], n_dn = tb[2] * TD;
+  fence_proxy_async_smem();  // the tables' scratch (generic stores) becomes ring stages (bulk copies)
+  const int n_tasks = n_gu + n_dn;
+  bool ok = true;
   const uint64_t pol = l2_evict_first_policy();
   int slot = 0;
   uint32_t round = 0;
   int last_round[RING];
 #pragma unroll
   for (int s = 0; s < RING; ++s) last_round[s] = -1;
-  task = __shfl_sync(0xffffffffu, task, 0);
   while (ok && task < n_tasks) {
     int nxt = 0;
     if (lane == 0) nxt = static_cast<int>(atomicAdd(ctr, 1u));  // fetched while this piece is issued
@@ -1189,6 +1295,7 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
   const int r = threadIdx.x, lane = r & 31;
   const int D = a.sh.d, TD = D / kTileRows;
   uint32_t *tab = reinterpret_cast<uint32_t *>(smem + P.tab);
+  const int n_gu = reinterpret_cast<const int *>(smem + P.table)[1];
   ConsState cs{0u, 0, 0};
   if (FMT == MOE_FMT_CB35_32) {
     load_grid_table(a.grid, tab, kTileRows);
@@ -1207,7 +1314,7 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
     }
     const StageInfo in = H->info[slot];
     if (in.task < 0) return;
-    const bool gu = in.task < H->n_gu;
+    const bool gu = in.task < n_gu;
     const int pieces = info_pieces(in.flags), tok0 = info_tok0(in.flags);
     if ((in.flags & kPieceStart) && pieces == 1) {
 #pragma unroll
@@ -1262,6 +1369,13 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
   }
 }
 
+// L2 prefetch of this CTA's share (part of parts) of `bytes` at `base` (multiples of 16 bytes).
+__device__ __forceinline__ void prefetch_share(const void *base, int64_t bytes, int part, int parts) {
+  const int64_t per = ((bytes + parts - 1) / parts + 15) & ~static_cast<int64_t>(15);
+  const int64_t b0 = per * part;
+  if (b0 < bytes) bulk_prefetch_l2(static_cast<const unsigned char *>(base) + b0, static_cast<uint32_t>(min(per, bytes - b0)));
+}
+
 // One persistent kernel for the expert GEMVs of a layer: gate/up + SwiGLU (h quantised into
 // records), then down.  Thread block = 4 consumer warps (thread = row of a 128-row tile) + one
 // producer warp; the grid is every resident CTA of the device.
@@ -1280,12 +1394,20 @@ __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(Deco
     H->abort = 0;
     fence_barrier_init();
   }
-  __syncthreads();
+  if (threadIdx.x == kTileRows && a.sh.n_shared) {  // the shared expert's planes (written by no kernel)
+    const ExpertGroup &G = a.L.shared;
+    prefetch_share(G.a, 3 * G.a_mat, blockIdx.x, gridDim.x);
+    prefetch_share(G.s, 3 * G.s_mat * 4, blockIdx.x, gridDim.x);
+    if (G.g) prefetch_share(G.g, 3 * G.g_mat * 8, blockIdx.x, gridDim.x);
+  }
+  griddep_wait();  // the router kernel's logits and records
+  if (threadIdx.x == 0) griddep_launch();
+  int first = 0;
+  if (threadIdx.x == kTileRows) first = static_cast<int>(atomicAdd(a.ws.counters, 1u));  // in flight meanwhile
+  build_tables(a, smem + P.stage0, reinterpret_cast<int *>(smem + P.table), blockIdx.x == 0);
   if (threadIdx.x >= kTileRows) {
-    producer<FMT>(a, smem, P, H);
+    producer<FMT>(a, smem, P, H, __shfl_sync(0xffffffffu, first, 0));
   } else {
-    griddep_wait();
-    if (threadIdx.x == 0) griddep_launch();
     consumer<FMT>(a, smem, P, H);
   }
 }
@@ -1331,10 +1453,6 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
 // ------------------------------------------------------------------------------------------
 // host launcher
 // ------------------------------------------------------------------------------------------
-int route_smem_bytes(int n_experts) {
-  return n_experts * 4 + 2 * (kMaxExperts / 32) * 4 + (n_experts > 1024 ? kDecodeMaxTokens * n_experts * 4 : 0);
-}
-
 // Under stream capture the records are made external, so that the CUDA graph records the
 // events too (a plain record under capture only orders the captured work).
 static inline void rec(const DecodeArgs &a, int kind, int end, cudaStream_t st) {
@@ -1380,8 +1498,10 @@ cudaError_t configure_decode_kernels() {
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  const void *ks[] = {(const void *)k_route<true>,
-                      (const void *)k_route<false>,
+  const void *ks[] = {(const void *)k_route<true, true>,
+                      (const void *)k_route<true, false>,
+                      (const void *)k_route<false, true>,
+                      (const void *)k_route<false, false>,
                       (const void *)k_gemv<MOE_FMT_Q2_32>,
                       (const void *)k_gemv<MOE_FMT_CB35_32>};
   for (const void *k : ks) {
@@ -1397,12 +1517,16 @@ cudaError_t configure_decode_kernels() {
 
 static int gemv_smem(int fmt, int umax) { return ring_plan(fmt, 1, kStageSlots, umax).total; }
 
+
 // Persistent grid: SMs x resident CTAs of the GEMV kernel; min_streams = MOE_STREAMS_PER_SM x SMs.
 cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_streams) {
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  // the routing scratch lives in the ring
+  const RingPlan P = ring_plan(fmt, 1, kStageSlots, umax);
+  if (ring_depth(fmt) * P.stage < table_scratch_bytes()) return cudaErrorInvalidConfiguration;
   int occ = 0;
   const int sm = gemv_smem(fmt, umax);
   e = fmt == MOE_FMT_Q2_32
@@ -1417,18 +1541,21 @@ cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_stream
 
 cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
   cudaError_t err;
-  // 1. router + input quantisation + top-k + tables
+  // 1. router logits + input quantisation
   {
-    const int ngrp = (a.sh.e + kRouteExperts - 1) / kRouteExperts;
-    const int grid = ngrp * (a.sh.d / a.ws.rk_cols);
-    const int sm = route_smem_bytes(a.sh.e);
+    const int grid = (a.sh.e + kRouteExperts - 1) / kRouteExperts;
+    const int sm = a.sh.e > 1024 ? a.sh.e * 4 : 0;  // one logit row for the shared-memory top-k
     rec(a, kProfRoute, 0, st);
-    err = a.sh.router_bf16 ? launch_pdl(k_route<true>, grid, kRouteThreads, sm, st, a)
-                           : launch_pdl(k_route<false>, grid, kRouteThreads, sm, st, a);
+    if (a.sh.router_bf16)
+      err = a.x_bf16 ? launch_pdl(k_route<true, true>, grid, kRouteThreads, sm, st, a)
+                     : launch_pdl(k_route<true, false>, grid, kRouteThreads, sm, st, a);
+    else
+      err = a.x_bf16 ? launch_pdl(k_route<false, true>, grid, kRouteThreads, sm, st, a)
+                     : launch_pdl(k_route<false, false>, grid, kRouteThreads, sm, st, a);
     if (err != cudaSuccess) return err;
     rec(a, kProfRoute, 1, st);
   }
-  // 2. gate/up + SwiGLU, then down (one persistent kernel)
+  // 2. top-k + tables (per CTA), gate/up + SwiGLU, then down (one persistent kernel)
   {
     const int sm = gemv_smem(a.sh.fmt, a.ws.umax);
     rec(a, kProfGateUp, 0, st);

@@ -85,24 +85,22 @@ static_assert(sizeof(ActRec) == 144, "ActRec is 9 x 16 bytes");
 // unit or several CTAs each take a run of segments (then the segment sums pass through the
 // partial buffers), so results do not depend on how the work was split.
 struct DecodeWs {
-  float *logit_part;    // [ks][8][E] router sums per K slice
   float *logits;        // [8][E]
+  int *sel;             // [8][k] selected experts per token, descending logit (the router's top-k)
+  unsigned *route_sync; // [2] router CTAs done, top-k CTAs done
   int *route_idx;       // [8][k]
   float *route_w;       // [8][k]
   int *slotpos;         // [8][k]: u * 8 + i (i = position of the token in expert u's list)
-  // Task table of the GEMV kernels, written by the router kernel: a header
-  // [n_active, gate/up tasks, down pieces per output tile, 0] and one 16-int row per active
-  // expert u: [expert (E = shared), ntok, tokens 0..7, first gate/up task, gate/up split,
-  // first down piece, down split, token groups, 0]; a split packs run length | pieces << 8 |
-  // chunks per segment << 16 | segments << 20.
-  int *task_tab;        // [4 + umax * 16]
+  // (The GEMV kernel's task table lives in each CTA's shared memory: a header [n_active,
+  // gate/up tasks, down pieces per output tile, 0] and one 16-int row per active expert u:
+  // [expert (E = shared), ntok, tokens 0..7, first gate/up task, gate/up split, first down
+  // piece, down split, token groups, 0]; a split packs run length | pieces << 8 | chunks per
+  // segment << 16 | segments << 20.)
   ActRec *xrec;         // [8][D/64]
   ActRec *hrec;         // [umax][8][fmax/64]
   float *gu_part;       // [umax][tmax][gu_nseg][2][8][128] gate/up segment sums
   float *dn_part;       // [umax][D/128][dn_nseg][8][128]  down segment sums
   float *o;             // [umax * 8][D] expert outputs (unweighted)
-  unsigned *route_ticket;   // [1]
-  unsigned *group_ticket;   // [ceil(E/32)]
   unsigned *gu_ticket;      // [umax][tmax][4 token groups]
   unsigned *dn_ticket;      // [umax][D/128][4 token groups]
   unsigned *counters;       // [2] work queue of the GEMV kernel (gate/up pieces, then down pieces)
@@ -110,7 +108,6 @@ struct DecodeWs {
   int umax;
   int tmax;             // max(F, F_shared) / 128
   int fmax;
-  int rk_cols;          // router: d_model columns per CTA (128 or 256)
   int gu_seg;           // gate/up: chunks per K segment (2 or 4)
   int gu_nseg;          // gate/up: K segments (d_model / 64 / gu_seg)
   int dn_nseg;          // down: most K segments of any expert
@@ -184,6 +181,17 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bulk prefetch of global memory into L2 (16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // L2 policy for data read once (the weight blocks): evict first, so that a pass over the
@@ -277,7 +285,6 @@ constexpr int kProfKinds = 3;
 
 cudaError_t configure_decode_kernels();
 cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_streams);
-int route_smem_bytes(int n_experts);
 cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_wait_test(unsigned *never_set, uint32_t *err, uint64_t spin_limit, cudaStream_t st);
 
