@@ -138,10 +138,10 @@ void plan_workspace(moe_handle *h, Carve &c) {
   w.gu_part = c.take<float>(static_cast<uint64_t>(umax) * tmax * w.gu_nseg * 2 * kDecodeMaxTokens * kTileRows);
   w.dn_part = c.take<float>(static_cast<uint64_t>(umax) * td * w.dn_nseg * kDecodeMaxTokens * kTileRows);
   w.o = c.take<float>(hrows * D);
-  w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * 4);  // x token groups of a unit
-  w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td * 4);
+  w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * kDecodeMaxTokens);  // x token groups of a unit (at most one per token)
+  w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td * kDecodeMaxTokens);
   w.counters = c.take<unsigned>(2);
-  w.h_done = c.take<unsigned>(static_cast<uint64_t>(umax) * 4);
+  w.h_done = c.take<unsigned>(static_cast<uint64_t>(umax) * kDecodeMaxTokens);
   const uint64_t nt = static_cast<uint64_t>(g.max_tokens) * D;
   h->res[0] = c.take<float>(nt);
   h->res[1] = c.take<float>(nt);
@@ -158,11 +158,11 @@ moe_status check_device_error(moe_handle *h, cudaStream_t st) {
   // a kernel that gave up may have left arrival counters set: clear them
   const DecodeWs &w = h->dws;
   const int td = h->cfg.d_model / kTileRows;
-  cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax * 4, st);
-  cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td * 4, st);
+  cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax * kDecodeMaxTokens, st);
+  cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td * kDecodeMaxTokens, st);
   cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * 2, st);
   cudaMemsetAsync(w.route_sync, 0, sizeof(unsigned) * 2, st);
-  cudaMemsetAsync(w.h_done, 0, sizeof(unsigned) * w.umax * 4, st);
+  cudaMemsetAsync(w.h_done, 0, sizeof(unsigned) * w.umax * kDecodeMaxTokens, st);
   if (e & kErrTimeout) return fail(h, MOE_ERR_TIMEOUT, "a device-side bounded wait ran out");
   return fail(h, MOE_ERR_DEVICE_FAULT, "a device-side check found an invalid routing index");
 }

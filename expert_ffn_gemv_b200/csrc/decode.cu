@@ -43,7 +43,7 @@ constexpr int kConsWarps = kTileRows / 32;      // consumer warps: thread = row 
 constexpr int kGemvThreads = kTileRows + 32;    // + one producer warp
 constexpr int kRing = 4;                        // most stages of the bulk-copy ring
 #ifndef MOE_GEMV_MIN_BLOCKS
-#define MOE_GEMV_MIN_BLOCKS 3                   // resident CTAs per SM the register budget allows
+#define MOE_GEMV_MIN_BLOCKS 4                   // resident CTAs per SM the register budget allows
 #endif
 #ifndef MOE_GEMV_UNROLL
 #define MOE_GEMV_UNROLL 1                       // chunks of a stage in flight per iteration
@@ -52,9 +52,11 @@ constexpr int kGemvUnroll = MOE_GEMV_UNROLL;
 #ifndef MOE_STREAMS_PER_SM
 #define MOE_STREAMS_PER_SM 6                    // GEMV pieces wanted in flight per SM (K split when fewer)
 #endif
-// ring depth: 4 stages for Q2; 3 for CB35, whose stages and grid table are larger, so that two
-// CTAs fit on an SM
-__host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_CB35_32 ? 3 : 4; }
+// ring depth: 4 stages for Q2; 3 for CB35, whose stages and grid table are larger
+#ifndef MOE_Q2_RING
+#define MOE_Q2_RING 4
+#endif
+__host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_CB35_32 ? 3 : MOE_Q2_RING; }
 constexpr int kGuStageChunks = 2;               // gate/up: chunks per stage
 constexpr int kDnStageChunks = 4;               // down: chunks per stage (one K segment)
 constexpr int kStageSlots = 2 * kGuStageChunks;   // (matrix, chunk) slots of a stage: 4 either way
@@ -360,17 +362,18 @@ __device__ __forceinline__ int piece_run(int nseg, int units_total, int min_stre
   return udiv_small(nseg + p - 1, p);
 }
 
-// Token groups of an active expert: an expert serving three or more tokens is cut into groups of
-// at most two tokens, each a unit of its own over the whole K (the weights are read once per
-// group), which keeps every unit's arithmetic within about 1.6 times that of a one-token unit.
+// Token groups of an active expert: each group of at most kTokGroup of its tokens is a unit of
+// its own over the whole K, so the expert's rows stream once per group (the repeats mostly from
+// L2).  Groups of one token keep every unit's arithmetic equal and the one-token GEMV's registers
+// low enough for four CTAs per SM; MOE_TOK_GROUP=2 (or 4) builds the grouped variant.
 #ifndef MOE_TOK_GROUP
-#define MOE_TOK_GROUP 2
+#define MOE_TOK_GROUP 1
 #endif
 constexpr int kTokGroup = MOE_TOK_GROUP;
 constexpr int kMaxTokGroups = kDecodeMaxTokens / kTokGroup;
 constexpr int kUnitTok = kTokGroup;  // tokens of one GEMV unit (at most)
-__host__ __device__ inline int tok_groups(int ntok) { return ntok >= 3 ? (ntok + kTokGroup - 1) / kTokGroup : 1; }
-__host__ __device__ inline int tok_group_size(int ntok) { return ntok >= 3 ? kTokGroup : ntok; }
+__host__ __device__ inline int tok_groups(int ntok) { return (ntok + kTokGroup - 1) / kTokGroup; }
+__host__ __device__ inline int tok_group_size(int ntok) { return ntok < kTokGroup ? ntok : kTokGroup; }
 
 // Split of one GEMV unit whose K has nc chunks: K segments of 4 (else 2) chunks, cut into
 // pieces of `len` segments.  Returns the packed split; `pieces` the number of pieces.

@@ -101,10 +101,10 @@ struct DecodeWs {
   float *gu_part;       // [umax][tmax][gu_nseg][2][8][128] gate/up segment sums
   float *dn_part;       // [umax][D/128][dn_nseg][8][128]  down segment sums
   float *o;             // [umax * 8][D] expert outputs (unweighted)
-  unsigned *gu_ticket;      // [umax][tmax][4 token groups]
-  unsigned *dn_ticket;      // [umax][D/128][4 token groups]
+  unsigned *gu_ticket;      // [umax][tmax][8] (token groups)
+  unsigned *dn_ticket;      // [umax][D/128][8] (token groups)
   unsigned *counters;       // [2] work queue of the GEMV kernel (gate/up pieces, then down pieces)
-  unsigned *h_done;         // [umax][4 token groups] (tile, consumer warp) pairs that wrote h
+  unsigned *h_done;         // [umax][8] (token groups): (tile, consumer warp) pairs that wrote h
   int umax;
   int tmax;             // max(F, F_shared) / 128
   int fmax;
