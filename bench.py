@@ -112,18 +112,19 @@ def source_hash(*files) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str, src_hash: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+def profiled_traffic(kernel: str, workload: str, src_hash: str, algorithmic_bytes: float):
+    """DRAM bytes per launch of `kernel`: the committed ncu summary's measured ratio of DRAM bytes
+    (read + write) to the captured launch's algorithmic bytes, times this run's algorithmic bytes
+    per launch -- if the summary was taken on the current kernel source (else None)."""
     p = ROOT / "profiles" / f"{kernel}_{workload}.md"
     if not p.exists():
         return None
     t = p.read_text()
     m = re.search(r"source_hash:\s*([0-9a-f]+)", t)
-    b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", t)
-    if not m or not b or m.group(1) != src_hash:
+    r = re.search(r"dram_over_algorithmic:\s*([0-9.eE+]+)", t)
+    if not m or not r or m.group(1) != src_hash:
         return None
-    return float(b.group(1))
+    return float(r.group(1)) * algorithmic_bytes
 
 
 # ------------------------------------------------------------------------------------ distributed
@@ -340,7 +341,7 @@ def bench_verify(args, rank, world, local):
     hbm_peak = pk["hbm_gbs"]
     achieved = gemv_bytes_last / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
     src = source_hash("expert_ffn_gemv_b200/csrc/decode.cu", "expert_ffn_gemv_b200/csrc/moe_internal.cuh")
-    traffic = profiled_traffic("k_gemv", "verify", src)
+    traffic = profiled_traffic("k_gemv", "verify", src, gemv_bytes_last / max(gu_cnt, 1))
     res = {
         "metric": METRIC,
         "value": value,
