@@ -241,12 +241,29 @@ __global__ void __launch_bounds__(256) k_pf_scatter(PrefillArgs a) {
     a.ws.row_w[pos] = w;
     a.ws.pos[static_cast<int64_t>(t) * (K + 1) + j] = pos;
   }
-  // gather the activations as bf16 (round to nearest even)
-  __nv_bfloat162 *dst = reinterpret_cast<__nv_bfloat162 *>(a.ws.xs + static_cast<int64_t>(pos) * D);
-  for (int c = lane; c < D / 2; c += 32) {
-    const float v0 = pf_load_act(a.x, static_cast<int64_t>(t) * D + 2 * c, a.x_bf16);
-    const float v1 = pf_load_act(a.x, static_cast<int64_t>(t) * D + 2 * c + 1, a.x_bf16);
-    dst[c] = __floats2bfloat162_rn(v0, v1);
+  // gather the activations as bf16 (round to nearest even), 8 columns per lane and step
+  uint4 *dst = reinterpret_cast<uint4 *>(a.ws.xs + static_cast<int64_t>(pos) * D);
+  const int64_t x0 = static_cast<int64_t>(t) * D;
+  const bool vec = (reinterpret_cast<uintptr_t>(a.x) & 15) == 0;  // rows are multiples of 16 bytes
+  for (int c = lane; c < D / 8; c += 32) {
+    float v[8];
+    if (vec && a.x_bf16) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + x0) + c);
+      dst[c] = q;  // already bf16
+      continue;
+    }
+    if (vec) {
+      const float4 *f = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + x0) + 2 * c;
+      const float4 f0 = __ldg(f), f1 = __ldg(f + 1);
+      v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w; v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = pf_load_act(a.x, x0 + 8 * c + i, a.x_bf16);
+    }
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    dst[c] = *reinterpret_cast<const uint4 *>(h);
   }
 }
 
@@ -718,28 +735,67 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
 // ------------------------------------------------------------------------------------------
 // combine: y[t] = sum_j outs[pos(t, j)] + outs[pos(t, shared)] (+ x[t]), slot order
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_pf_combine(PrefillArgs a) {
-  const int D = a.sh.d, K = a.sh.k;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= static_cast<int64_t>(a.n) * D) return;
-  const int t = static_cast<int>(i / D), d = static_cast<int>(i % D);
-  const int *pos = a.ws.pos + static_cast<int64_t>(t) * (K + 1);
-  float v[kMaxTopK];
+// CTA per token, thread = 8 consecutive columns: 16-byte loads of the token's K + 1 weighted
+// rows (runs of eight loads ahead of their sums), y in slot order, then + shared (+ x).
+constexpr int kPfCombineCols = 8;
+__global__ void __launch_bounds__(512) k_pf_combine(PrefillArgs a) {
+  __shared__ int s_pos[kMaxTopK + 1];
+  const int D = a.sh.d, K = a.sh.k, t = blockIdx.x;
+  if (threadIdx.x <= K) s_pos[threadIdx.x] = a.ws.pos[static_cast<int64_t>(t) * (K + 1) + threadIdx.x];
+  __syncthreads();
+  const int c = threadIdx.x;  // columns 8c .. 8c+7
+  if (c >= D / kPfCombineCols) return;
+  const int64_t i0 = static_cast<int64_t>(t) * D + kPfCombineCols * c;
+  float y[8];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
-    v[j] = j < K ? __bfloat162float(a.ws.outs[static_cast<int64_t>(pos[j]) * D + d]) : 0.f;
-  const float sh = a.sh.n_shared ? __bfloat162float(a.ws.outs[static_cast<int64_t>(pos[K]) * D + d]) : 0.f;
-  float y = 0.f;
+  for (int q = 0; q < 8; ++q) y[q] = 0.f;
+  auto add_row = [&](const uint4 &r, float (&acc)[8]) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
-    if (j < K) y += v[j];
-  y += sh;
-  if (a.residual) y = pf_load_act(a.x, i, a.x_bf16) + y;
-  if (a.y_bf16)
-    static_cast<__nv_bfloat16 *>(a.y)[i] = __float2bfloat16_rn(y);
-  else
-    static_cast<float *>(a.y)[i] = y;
-  if (a.y_copy) a.y_copy[i] = y;
+    for (int q = 0; q < 4; ++q) {
+      acc[2 * q] += __uint_as_float(w[q] << 16);
+      acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+  };
+  for (int j0 = 0; j0 < K; j0 += 8) {
+    uint4 r[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j0 + j < K) r[j] = __ldcg(reinterpret_cast<const uint4 *>(a.ws.outs + static_cast<int64_t>(s_pos[j0 + j]) * D) + c);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j0 + j < K) add_row(r[j], y);
+  }
+  if (a.sh.n_shared) {
+    float sh[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sh[q] = 0.f;
+    add_row(__ldcg(reinterpret_cast<const uint4 *>(a.ws.outs + static_cast<int64_t>(s_pos[K]) * D) + c), sh);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) y[q] += sh[q];
+  }
+  if (a.residual) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) y[q] = pf_load_act(a.x, i0 + q, a.x_bf16) + y[q];
+  }
+  if (a.y_bf16) {
+    __nv_bfloat16 *yo = static_cast<__nv_bfloat16 *>(a.y) + i0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) yo[q] = __float2bfloat16_rn(y[q]);
+  } else {
+    float *yo = static_cast<float *>(a.y) + i0;
+    if ((reinterpret_cast<uintptr_t>(yo) & 15) == 0) {
+      reinterpret_cast<float4 *>(yo)[0] = make_float4(y[0], y[1], y[2], y[3]);
+      reinterpret_cast<float4 *>(yo)[1] = make_float4(y[4], y[5], y[6], y[7]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) yo[q] = y[q];
+    }
+  }
+  if (a.y_copy) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) a.y_copy[i0 + q] = y[q];
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -847,8 +903,8 @@ cudaError_t launch_prefill_layer(const PrefillArgs &a, cudaStream_t st) {
     k_pf_gemm<MOE_FMT_CB35_32, 1><<<grid, kPfThreads, PfPlan<MOE_FMT_CB35_32, 1>::kBytes, st>>>(a);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   {
-    const int64_t outs = static_cast<int64_t>(n) * a.sh.d;
-    k_pf_combine<<<static_cast<unsigned>((outs + 255) / 256), 256, 0, st>>>(a);
+    const int threads = max(64, a.sh.d / kPfCombineCols);  // d_model <= 4096: at most 512; >= k + 1
+    k_pf_combine<<<static_cast<unsigned>(n), threads, 0, st>>>(a);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   pf_rec(a, kProfDown, 1, st);
