@@ -128,21 +128,39 @@ def profiled_traffic(kernel: str, workload: str, src_hash: str, algorithmic_byte
 
 
 # ------------------------------------------------------------------------------------ distributed
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU: RANK / LOCAL_RANK / WORLD_SIZE come from the launcher, and WORLD_SIZE
+    must equal --gpus (a mismatch is an error, not a silent 1-GPU run)."""
     import torch
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"bench.py: --gpus {n_gpus} but WORLD_SIZE={world}")
     if world > 1:
         import datetime
 
         import torch.distributed as dist
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
-    torch.cuda.set_device(local)
+        kw = dict(device_id=torch.device("cuda", local)) if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600), **kw)
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     return rank, world, local
+
+
+def relaunch(n_gpus) -> int:
+    """--gpus N > 1 without a launcher: run this command again under torch.distributed.run with
+    N processes on this node (rendezvous on 127.0.0.1); rank 0 prints the JSON line."""
+    import socket
+
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n_gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), str(Path(__file__).resolve()), *sys.argv[1:]]
+    return subprocess.run(cmd).returncode
 
 
 def barrier(world):
@@ -242,6 +260,32 @@ def oracle_sample_stack(wl, seed, n_tokens, n_layers_sample, pass_idx=0, threads
 
 
 # ------------------------------------------------------------------------------------ verify stack
+def verify_config(wl, L):
+    """The workload description both arms print (static: identical in the reference arm)."""
+    return {"workload": wl.name, "d_model": wl.d_model, "d_ff": wl.d_ff, "n_experts": wl.n_experts,
+            "top_k": wl.top_k, "n_shared": wl.n_shared, "layers": L, "tokens_per_pass": wl.n_tokens,
+            "weights": "Q2 2-bit blocks, 10 B / 32 weights", "router_bias": "Zipf(1.1), beta 0.5",
+            "l2": "inputs larger than L2: each pass reads ~4 GB of distinct expert blocks (126 MB L2)",
+            "parallelism": "replicas (one process per GPU, no data-path collective)"}
+
+
+def near_ties(wl, seed, trace):
+    """Near ties of one pass, counted as the parity rule counts them: for each layer, the oracle's
+    router margin l_(k) - l_(k+1) on the GPU's own input of that layer (teacher-forced); a token
+    whose margin is below 1e-4 would be excluded from index parity."""
+    sys.path.insert(0, str(ROOT / "tests"))
+    from helpers import TIE_EPS, oracle_layer
+
+    per_layer = []
+    for l in range(trace.shape[0]):
+        _, _, m = oracle_layer(wl, seed, l, full=False).route(trace[l])
+        per_layer.append(int((m < TIE_EPS).sum()))
+    return {"excluded_token_layers": int(sum(per_layer)), "token_layers": int(trace.shape[0] * trace.shape[1]),
+            "layers_with_ties": [l for l, c in enumerate(per_layer) if c],
+            "rule": "oracle margin l_(k) - l_(k+1) < 1e-4 on the GPU's per-layer input (teacher-forced), "
+                    "last timed pass"}
+
+
 def bench_verify(args, rank, world, local):
     import torch
 
@@ -355,13 +399,10 @@ def bench_verify(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "q2 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
         "data": "synthetic (seeded integer-hash generator, random-init weights)",
-        "config": {"workload": wl.name, "d_model": wl.d_model, "d_ff": wl.d_ff, "n_experts": wl.n_experts,
-                   "top_k": wl.top_k, "n_shared": wl.n_shared, "layers": L, "tokens_per_pass": n,
-                   "weights": "Q2 2-bit blocks, 10 B / 32 weights", "router_bias": "Zipf(1.1), beta 0.5",
-                   "resident_weight_gb": round(moe.device_bytes() / 1e9, 2),
-                   "l2": "inputs larger than L2: each pass reads ~%.1f GB of distinct expert blocks"
-                         % (step_bytes.mean() / 1e9),
-                   "parallelism": f"replicas x{world}", "cuda_graph": "one pass (48 x 3 kernels, programmatic launches) per replay"},
+        "config": verify_config(wl, L),
+        "resident_weight_gb": round(moe.device_bytes() / 1e9, 2),
+        "distinct_block_gb_per_pass": round(float(step_bytes.mean()) / 1e9, 2),
+        "launch": "one CUDA graph per pass (48 x 3 kernels, programmatic dependent launches)",
         "hbm": {"active_expert_and_router_bytes_per_step": float(step_bytes.mean()),
                 "gbs": float(step_bytes.sum() / (ms_local / 1e3) / 1e9),
                 "frac_of_measured_peak": float(step_bytes.sum() / (ms_local / 1e3) / 1e9 / hbm_peak),
@@ -394,6 +435,12 @@ def bench_verify(args, rank, world, local):
                       "steps": Ke, "api": "moe_forward_stack(host x, host x_out)"}
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        trace = torch.empty((L, n, wl.d_model), dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            x_in.copy_(xs[W + K - 1])
+            moe.forward_stack(0, L, x_in, out, x_trace=trace)
+        stream.synchronize()
+        res["near_ties"] = near_ties(wl, seed, trace.cpu().numpy().astype(np.float64))
         nl = args.cpu_layers
         sec, used = oracle_sample_stack(wl, seed, n, nl, pass_idx=0)
         res["cpu_baseline"] = {"value": n * nl / sec / L, "unit": "tokens/s", "cores": used, "kind": "oracle",
@@ -565,20 +612,43 @@ def bench_prefill(args, rank, world, local):
     rows = n * (wl.top_k + wl.n_shared)
     flop_gu = 2.0 * rows * 2 * wl.d_ff * wl.d_model        # per layer, gate + up
     flop_layer = 2.0 * rows * 3 * wl.d_ff * wl.d_model + 2.0 * n * wl.n_experts * wl.d_model
+    # active experts of each layer (one eager pass of the last input, untimed)
+    counts = [torch.empty(wl.n_experts, dtype=torch.int32, device=dev) for _ in range(nl)]
+    x_in.copy_(xs[(W + K - 1) % 2])
+    moe.forward_stack(0, nl, x_in, out, routes=[dict(counts=c) for c in counts])
+    u = np.array([int((c > 0).sum()) for c in counts]) + wl.n_shared
+    eb = wl.expert_bytes()
+    # gate/up GEMM bytes per layer: the active experts' gate and up blocks, the grouped bf16 rows
+    # in and the bf16 h rows out
+    bytes_gu = float(((u * eb * 2) // 3).mean()) + rows * wl.d_model * 2 + rows * wl.d_ff * 2
     pk, kind = peaks()
-    peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    peak_burst = pk["bf16_tflops"]
+    peak_sus = pk.get("bf16_tflops_sustained", peak_burst)
     tfl = flop_layer * nl * K / (ms / 1e3) / 1e12
     gu_tf = flop_gu * kcnt / (kms / 1e3) / 1e12 if kms else None
+    gu_gbs = bytes_gu * kcnt / (kms / 1e3) / 1e9 if kms else None
+    # arithmetic intensity of the gate/up GEMM against the ridge of the measured peaks: the
+    # 8,192-token chunk is tensor-bound, the 1,180-token chunk HBM-bound
+    intensity = flop_gu / bytes_gu
+    ridge = peak_burst * 1e12 / (pk["hbm_gbs"] * 1e9)
+    if intensity >= ridge:
+        roof = {"kernel": "k_pf_gemm<gate/up>", "bound": "tensor", "unit": "TFLOP/s", "peak": peak_burst,
+                "peak_kind": kind + " burst bf16", "achieved": gu_tf, "frac": gu_tf / peak_burst if gu_tf else None,
+                "frac_of_sustained": gu_tf / peak_sus if gu_tf else None}
+    else:
+        roof = {"kernel": "k_pf_gemm<gate/up>", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                "peak_kind": kind, "achieved": gu_gbs, "frac": gu_gbs / pk["hbm_gbs"] if gu_gbs else None,
+                "tflops": gu_tf}
+    roof.update({"avg_launch_us": kms / max(kcnt, 1) * 1e3, "traffic": None,
+                 "algorithmic_bytes_per_launch": bytes_gu, "flop_per_launch": flop_gu,
+                 "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge})
     res = _base_result(wl, world, K, W, ms, "tokens/s", sum_over_ranks(n * K / (ms / 1e3), world))
     res.update({"dtype": "bf16 operands (dequantised q2), f32 accumulate (tcgen05)",
                 "config": {"workload": wl.name, "layers": nl, "chunk_tokens": n,
                            "l2": "each chunk reads the whole 36 GB stack"},
-                "tflops_whole_step": tfl, "frac_of_sustained_peak": tfl / peak_tf,
-                "roofline": {"kernel": "k_pf_gemm<gate/up>", "bound": "tensor", "unit": "TFLOP/s",
-                             "peak": peak_tf, "peak_kind": kind + " sustained bf16", "achieved": gu_tf,
-                             "frac": gu_tf / peak_tf if gu_tf else None,
-                             "avg_launch_us": kms / max(kcnt, 1) * 1e3, "traffic": None},
-                "clocks": clocks, "gpu_launches": K * nl * 8})
+                "tflops_whole_step": tfl, "frac_of_burst_peak_whole_step": tfl / peak_burst,
+                "mean_active_experts_per_layer": float(u.mean()),
+                "roofline": roof, "clocks": clocks, "gpu_launches": K * nl * 8})
     moe.close()
     return res
 
@@ -622,12 +692,31 @@ def bench_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / len(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded integer-hash generator)",
-        "config": {"workload": wl.name, "layers": L, "tokens_per_pass": n,
-                   "step": "8 tokens through one layer (layer = step mod 48), scaled to the 48-layer stack"},
+        "config": verify_config(wl, L),
+        "step": "8 tokens through one layer (layer = step mod 48), scaled to the 48-layer stack",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
                          "sample": f"{len(times)} steps of 8 tokens x 1 layer"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+# ------------------------------------------------------------------------------------ replica plumbing
+def bench_plumbing(args, rank, world, local):
+    """No GPU (gloo): the replica launch, the barriers and the max / sum over ranks, with a fixed
+    host loop standing in for a step.  It checks the multi-process plumbing on a CPU machine and
+    reports no GPU figure."""
+    barrier(world)
+    t0 = time.perf_counter()
+    acc = 0
+    for _ in range(args.steps):
+        acc += sum(range(20000 * (rank + 1)))
+    el_ms = (time.perf_counter() - t0) * 1e3
+    barrier(world)
+    ms = max_over_ranks(el_ms, world)
+    tokens = sum_over_ranks(args.steps * 8, world)
+    return {"metric": "replica plumbing check (host loop, no GPU)", "value": tokens / (ms / 1e3), "unit": "steps*8/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "rank_ms": el_ms, "total_tokens": tokens}
 
 
 # ------------------------------------------------------------------------------------ main
@@ -645,6 +734,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=12)
+    ap.add_argument("--plumbing-check", action="store_true",
+                    help="no GPU: run only the replica launch / barrier / max-over-ranks logic (gloo)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -654,9 +745,13 @@ def main():
             return 0
         print(json.dumps(bench_reference(args)), flush=True)
         return 0
-    rank, world, local = dist_setup(args.gpus)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(args.gpus)
+    rank, world, local = dist_setup(args.gpus, "gloo" if args.plumbing_check else "nccl")
     fn = {"verify": bench_verify, "decode": bench_decode_layers, "codebook": bench_codebook,
           "prefill": bench_prefill}[args.workload]
+    if args.plumbing_check:
+        fn = bench_plumbing
     res = fn(args, rank, world, local)
     if world > 1:
         import torch.distributed as dist

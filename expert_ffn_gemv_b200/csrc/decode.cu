@@ -114,22 +114,28 @@ __device__ __forceinline__ void load_row8(const void *w, int64_t off, float (&v)
   }
 }
 
-// Order-preserving unsigned key of a float (larger float -> larger key); NaN maps to 0, the
-// key that never wins, and 0 also marks an expert already taken.
+// Order-preserving unsigned key of a float (larger float -> larger key); NaN maps to 1, below
+// every number (-inf is 0x007FFFFF), so a NaN logit is taken only after every numeric one; 0
+// marks an expert already taken (and lanes beyond E).
 __device__ __forceinline__ uint32_t order_key(float f) {
-  if (f != f) return 0u;
+  if (f != f) return 1u;
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The logit a key stands for (the NaN key counts as -inf: weight 0 in the softmax).
 __device__ __forceinline__ float key_value(uint32_t k) {
+  if (k <= 1u) return -INFINITY;
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// fp32 softmax over the K selected logits (lane j holds the j-th), results to the tables
+// fp32 softmax over the K selected logits (lane j holds the j-th), results to the tables.  A
+// token whose largest logit is not finite has no defined weights: the call reports a device
+// fault.
 __device__ __forceinline__ void softmax_store(const DecodeArgs &a, int t, int lane, float my_l, float l0, int my_i,
                                               bool wr) {
   const int K = a.sh.k;
+  if (lane == 0 && !(l0 > -INFINITY && l0 < INFINITY)) flag_error(a.err, kErrBadIndex);
   float w = lane < K ? __expf(my_l - l0) : 0.f;
   float sum = w;
 #pragma unroll
@@ -202,7 +208,7 @@ __device__ __forceinline__ void topk_regs(const DecodeArgs &a, const int (&t)[NT
       const uint32_t m = __reduce_max_sync(0xffffffffu, lb[i]);
       int bi = __reduce_min_sync(0xffffffffu, lb[i] == m ? lane + 32 * lq[i] : INT_MAX);
       float bv = key_value(m);
-      if (bi >= E || !(bv > -INFINITY)) {  // only non-finite logits left
+      if (bi >= E) {  // cannot happen (k <= E numeric or NaN keys >= 1): keep the index in range
         if (lane == 0) flag_error(a.err, kErrBadIndex);
         bi = j;
         bv = 0.f;
@@ -299,11 +305,6 @@ __device__ __forceinline__ bool topk_rank(const DecodeArgs &a, int t, int lane, 
   if (lane < K) {
     my_l = sv[lane];
     my_i = si[lane];
-    if (!(my_l > -INFINITY)) {  // a non-finite logit was selected
-      flag_error(a.err, kErrBadIndex);
-      my_l = 0.f;
-      my_i = lane;
-    }
     s_idx[t * K + lane] = my_i;
   }
   const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
@@ -312,33 +313,32 @@ __device__ __forceinline__ bool topk_rank(const DecodeArgs &a, int t, int lane, 
   return true;
 }
 
-// Top-k of token t by one warp over logits in shared memory (more than 1,024 experts).
-__device__ __forceinline__ void topk_smem(const DecodeArgs &a, int t, int lane, float *row, int *s_idx, bool wr) {
+// Top-k of token t by one warp over keys in shared memory (more than 1,024 experts): rounds of
+// a warp argmax over the order keys (equal keys: the lower index), the winner's key cleared.
+__device__ __forceinline__ void topk_smem(const DecodeArgs &a, int t, int lane, float *row_f, int *s_idx, bool wr) {
   const int E = a.sh.e, K = a.sh.k;
-  for (int i = lane; i < E; i += 32) row[i] = __ldcg(a.ws.logits + t * E + i);
+  uint32_t *row = reinterpret_cast<uint32_t *>(row_f);
+  for (int i = lane; i < E; i += 32) row[i] = order_key(__ldcg(a.ws.logits + t * E + i));
   __syncwarp();
   float my_l = 0.f, l0 = 0.f;
   int my_i = 0;
   for (int j = 0; j < K; ++j) {
-    float bv = -INFINITY;
+    uint32_t bk = 0u;
     int bi = 0x7fffffff;
     for (int i = lane; i < E; i += 32) {
-      const float v = row[i];
-      if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+      const uint32_t v = row[i];
+      if (v > bk) { bk = v; bi = i; }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    if (bi >= E) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    bi = __reduce_min_sync(0xffffffffu, bk == m ? bi : 0x7fffffff);
+    if (bi >= E) {  // cannot happen (k <= E keys >= 1)
       if (lane == 0) flag_error(a.err, kErrBadIndex);
       bi = j;
     }
+    const float bv = key_value(m);
     if (j == 0) l0 = bv;
     if (lane == j) { my_l = bv; my_i = bi; }
-    if (lane == 0) { row[bi] = -INFINITY; s_idx[t * K + j] = bi; }
+    if (lane == 0) { row[bi] = 0u; s_idx[t * K + j] = bi; }
     __syncwarp();
   }
   softmax_store(a, t, lane, my_l, l0, my_i, wr);

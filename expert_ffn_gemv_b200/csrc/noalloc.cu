@@ -2,17 +2,17 @@
 //
 // moe_route_noalloc computes, for up to 8 tokens, the router logits (fp32 accumulation), the
 // top-k experts and their fp32 softmax weights, like the routing step of moe_forward.  It is
-// meant for callers that cannot allocate device memory at the point where they route: code
-// inside CUDA stream capture (allocation is not allowed there), runtimes that hand every byte of
-// device memory to their own planner, and latency-critical loops that must not take the
-// implicit synchronisation of cudaMalloc/cudaFree.  Its only scratch -- the logits of the call
-// and an arrival counter -- lives in the file-scope device array below, which every GPU that
-// loads this library holds until the process exits.
+// meant for callers that cannot allocate device memory at the point where they route: runtimes
+// that plan every byte of device memory up front and hand kernels only the buffers they planned,
+// and loops that must not take the device-wide synchronisation that cudaMalloc / cudaFree can
+// imply.  Its only scratch -- the logits of the call and an arrival counter -- lives in the
+// file-scope device array below, which every GPU that loads this library holds until the process
+// exits.
 //
 // Sharing rules: all calls in the process use the same array and it keeps the contents of the
-// last call.  Calls whose kernels may overlap on one device (for example on two streams) race on
-// it, so keep them in one stream order; calls on different devices do not, each device having
-// its own copy of the array.
+// last call (the arrival counter is cleared on the stream before every launch).  Calls whose
+// kernels may overlap on one device (for example on two streams) race on it, so keep them in one
+// stream order; calls on different devices do not, each device having its own copy of the array.
 #include <float.h>
 
 #include <mutex>
@@ -54,6 +54,20 @@ __device__ __forceinline__ void na_load_row8(const void *w, int bf16, int64_t of
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
+}
+
+// Order-preserving selection key of a logit: larger logit -> larger key, NaN -> 1 (below -inf,
+// whose key is 0x007FFFFF); 0 is reserved for "taken".
+__device__ __forceinline__ uint32_t na_order_key(float f) {
+  if (f != f) return 1u;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The logit a key stands for in the softmax (the NaN key counts as -inf).
+__device__ __forceinline__ float na_key_value(uint32_t k) {
+  if (k <= 1u) return -INFINITY;
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 struct NaArgs {
@@ -129,34 +143,38 @@ __global__ void __launch_bounds__(kNaThreads) k_route_noalloc(NaArgs a) {
   if (!s_last) return;
   __threadfence();
   if (warp < n) {
+    // Selection over order-preserving keys (larger logit -> larger key; NaN -> 1, below every
+    // number; 0 marks an expert already taken or a lane beyond E).  Lane l holds experts
+    // l + 32 q.  A round takes the largest key over the warp and, among equal keys, the lowest
+    // expert index; the winner's key is cleared.  E >= K valid keys exist, so every round finds
+    // a key >= 1 and the K experts are distinct.
     const int t = warp;
-    float v[kNaMaxExperts / 32];
+    constexpr int VPL = kNaMaxExperts / 32;
+    uint32_t key[VPL];
 #pragma unroll
-    for (int j = 0; j < kNaMaxExperts / 32; ++j) {
-      const int i = lane + 32 * j;
-      v[j] = i < E ? __ldcg(a.logits + t * E + i) : -INFINITY;
+    for (int q = 0; q < VPL; ++q) {
+      const int i = lane + 32 * q;
+      key[q] = i < E ? na_order_key(__ldcg(a.logits + t * E + i)) : 0u;
     }
-    float my_l = -FLT_MAX, l0 = 0.f;
+    float my_l = 0.f, l0 = 0.f;
     int my_i = 0;
     for (int j = 0; j < K; ++j) {
-      float bv = v[0];
-      int bi = lane;
+      uint32_t bk = key[0];
+      int bq = 0;
 #pragma unroll
-      for (int q = 1; q < kNaMaxExperts / 32; ++q)
-        if (v[q] > bv) { bv = v[q]; bi = lane + 32 * q; }
+      for (int q = 1; q < VPL; ++q)
+        if (key[q] > bk) { bk = key[q]; bq = q; }
+      const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+      const int bi = __reduce_min_sync(0xffffffffu, bk == m ? lane + 32 * bq : 0x7fffffff);
+      const float bv = na_key_value(m);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-      }
-      if (bi >= E) bi = j;  // only non-finite logits left: keep the index in range
-#pragma unroll
-      for (int q = 0; q < kNaMaxExperts / 32; ++q)
-        if (bi == lane + 32 * q) v[q] = -INFINITY;
+      for (int q = 0; q < VPL; ++q)
+        if (bi == lane + 32 * q) key[q] = 0u;
       if (j == 0) l0 = bv;
       if (lane == j) { my_l = bv; my_i = bi; }
     }
+    // fp32 softmax over the selected logits (a -inf or NaN logit gets weight 0; a token whose
+    // largest selected logit is not finite gets NaN weights, 0/0)
     float w = lane < K ? __expf(my_l - l0) : 0.f;
     float sum = w;
 #pragma unroll
@@ -198,6 +216,8 @@ extern "C" moe_status moe_route_noalloc(const void *router_w, int32_t router_dty
       top_k > n_experts || d_model < 128 || d_model % 128 ||
       (router_dtype != MOE_F32 && router_dtype != MOE_BF16) || (x_dtype != MOE_F32 && x_dtype != MOE_BF16))
     return MOE_ERR_INVALID_ARGUMENT;
+  // the router rows are read with 16-byte vector loads
+  if (reinterpret_cast<uintptr_t>(router_w) % 16 != 0) return MOE_ERR_INVALID_ARGUMENT;
   if (n_tokens > kNaMaxTokens || n_experts > kNaMaxExperts || d_model > kNaMaxD || top_k > kNaMaxTopK)
     return MOE_ERR_UNSUPPORTED;  // beyond the static scratch / kernel limits
   int dev = 0;

@@ -116,39 +116,52 @@ __global__ void __launch_bounds__(256) k_pf_router(PrefillArgs a) {
 // ------------------------------------------------------------------------------------------
 // top-k + softmax per token (warp per token, the token's logits in shared memory)
 // ------------------------------------------------------------------------------------------
+// Order-preserving selection key: larger logit -> larger key; NaN -> 1, below every number; 0
+// marks an expert already taken.
+__device__ __forceinline__ uint32_t pf_order_key(float f) {
+  if (f != f) return 1u;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float pf_key_value(uint32_t k) {
+  if (k <= 1u) return -INFINITY;
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 __global__ void __launch_bounds__(256) k_pf_topk(PrefillArgs a) {
   extern __shared__ __align__(16) float lgs[];
   const int E = a.sh.e, K = a.sh.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + warp;
   if (t >= a.n) return;
-  float *row = lgs + warp * E;
-  for (int i = lane; i < E; i += 32) row[i] = a.ws.logits[static_cast<int64_t>(t) * E + i];
+  uint32_t *row = reinterpret_cast<uint32_t *>(lgs) + warp * E;
+  for (int i = lane; i < E; i += 32) row[i] = pf_order_key(a.ws.logits[static_cast<int64_t>(t) * E + i]);
   __syncwarp();
-  float l0 = 0.f, my_l = -FLT_MAX;
+  float l0 = 0.f, my_l = 0.f;
   int my_i = 0;
   for (int j = 0; j < K; ++j) {
-    float bv = -INFINITY;
+    uint32_t bk = 0u;
     int bi = 0x7fffffff;
     for (int i = lane; i < E; i += 32) {
-      const float v = row[i];
-      if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+      const uint32_t v = row[i];
+      if (v > bk) { bk = v; bi = i; }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    if (bi >= E) {  // only non-finite logits left
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    bi = __reduce_min_sync(0xffffffffu, bk == m ? bi : 0x7fffffff);
+    if (bi >= E) {  // cannot happen (k <= E keys >= 1): keep the index in range
       if (lane == 0) flag_error(a.err, kErrBadIndex);
       bi = j;
     }
+    const float bv = pf_key_value(m);
     if (j == 0) l0 = bv;
     if (lane == j) { my_l = bv; my_i = bi; }
-    if (lane == 0) row[bi] = -INFINITY;
+    if (lane == 0) row[bi] = 0u;
     __syncwarp();
   }
+  // fp32 softmax over the selected logits; a largest logit that is not finite leaves the
+  // weights undefined: reported as a device fault
+  if (lane == 0 && !(l0 > -INFINITY && l0 < INFINITY)) flag_error(a.err, kErrBadIndex);
   float w = lane < K ? __expf(my_l - l0) : 0.f;
   float sum = w;
 #pragma unroll

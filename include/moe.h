@@ -147,21 +147,27 @@ uint64_t moe_device_bytes(const moe_handle *h);
 moe_status moe_profile_enable(moe_handle *h, int32_t on);
 moe_status moe_profile_read(moe_handle *h, int32_t kind, float *total_ms, int32_t *launches);
 
-/* Routing for callers that cannot allocate device memory where they route (inside CUDA stream
- * capture, under a runtime that plans all device memory itself, or in a loop that must not take
- * cudaMalloc's implicit synchronisation).  The paper has no counterpart of this entry point: it
- * is the routing step of moe_forward (router logits with fp32 accumulation, top-k with equal
- * logits resolved to the lower expert index, fp32 softmax over the selected logits) without a
- * handle.  All pointers are device pointers on the current device: router_w n_experts x d_model
- * (router_dtype), router_bias n_experts fp32 or NULL, x n_tokens x d_model (x_dtype); outputs
- * topk_idx / topk_w n_tokens x top_k, descending logit.  It allocates nothing: its scratch (the
- * logits and an arrival counter, 32 KB) is a static device array that every GPU loading the
- * library holds until exit.  The first call on a device looks up that array's device address
- * and sets the kernel's shared-memory limit; make that first call before any stream capture.
- * Limits: n_tokens <= 8, n_experts <= 1024, d_model <= 4096 (a multiple of 128), top_k <= 32;
- * larger sizes return MOE_ERR_UNSUPPORTED, malformed arguments MOE_ERR_INVALID_ARGUMENT.
- * Every call shares the one array and leaves its contents behind; calls whose kernels may
- * overlap on one device race on it, so keep them in one stream order. */
+/* Routing without a handle and without any device allocation.  Some callers cannot allocate
+ * device memory at the point where they route: runtimes that plan every byte of device memory
+ * up front and pass kernels only the buffers they planned, and loops that must not take the
+ * device-wide synchronisation that cudaMalloc / cudaFree can imply.  This entry point has no
+ * counterpart in the paper: it is the routing step of moe_forward (router logits with fp32
+ * accumulation, top-k with equal logits resolved to the lower expert index and NaN logits taken
+ * after every numeric one, fp32 softmax over the selected logits) without a handle.
+ * All pointers are device pointers on the current device: router_w n_experts x d_model
+ * (router_dtype, row-major, 16-byte aligned: it is read 16 bytes at a time), router_bias
+ * n_experts fp32 or NULL, x n_tokens x d_model (x_dtype); outputs topk_idx / topk_w
+ * n_tokens x top_k, descending logit.  A selected -inf (or NaN) logit gets weight 0; a token whose
+ * largest selected logit is not finite gets NaN weights.
+ * It allocates nothing: its scratch (the logits and an arrival counter, 32 KB) is a file-scope
+ * device array that every GPU loading the library holds until the process exits.  The first call
+ * on a device looks up that array's device address and sets the kernel's shared-memory limit;
+ * make that first call before any stream capture.  Limits: n_tokens <= 8, n_experts <= 1024,
+ * d_model <= 4096 (a multiple of 128), top_k <= 32; larger sizes return MOE_ERR_UNSUPPORTED,
+ * malformed arguments (NULL, out of range, a misaligned router_w) MOE_ERR_INVALID_ARGUMENT.
+ * Every call shares the one array and leaves its contents behind (the arrival counter is cleared
+ * on the stream before each launch); calls whose kernels may overlap on one device race on it,
+ * so keep them in one stream order. */
 moe_status moe_route_noalloc(const void *router_w, int32_t router_dtype, const float *router_bias,
                              int32_t n_experts, int32_t d_model, int32_t top_k, const void *x,
                              int32_t x_dtype, int32_t n_tokens, int32_t *topk_idx, float *topk_w,

@@ -59,7 +59,14 @@ def rel_l2(y, y_ref, mask=None) -> float:
 
 
 def compare_routing(idx_gpu, idx_ref, margin, n_experts, counts_gpu=None, eps=TIE_EPS):
-    """Returns (n_mismatch, n_excluded).  Sets compared per non-excluded token; counts too."""
+    """Returns (n_mismatch, n_excluded).
+
+    * expert sets are compared per non-excluded token (oracle margin >= eps);
+    * per-expert token counts are compared over the non-excluded tokens (the GPU's rows of
+      those tokens against the oracle's), whatever the number of excluded tokens;
+    * ``counts_gpu`` (the GPU's expert_counts output over all tokens of the call) must equal
+      the histogram of the GPU's own index rows.
+    Every failed check adds one to n_mismatch."""
     idx_gpu = np.asarray(idx_gpu)
     idx_ref = np.asarray(idx_ref)
     keep = np.asarray(margin) >= eps
@@ -67,9 +74,13 @@ def compare_routing(idx_gpu, idx_ref, margin, n_experts, counts_gpu=None, eps=TI
     for t in range(idx_ref.shape[0]):
         if keep[t] and set(idx_gpu[t].tolist()) != set(idx_ref[t].tolist()):
             bad += 1
-    if counts_gpu is not None and keep.all():
-        ref_counts = np.bincount(idx_ref.reshape(-1), minlength=n_experts)
-        if not np.array_equal(np.asarray(counts_gpu), ref_counts):
+    kept_gpu = np.bincount(idx_gpu[keep].reshape(-1), minlength=n_experts)
+    kept_ref = np.bincount(idx_ref[keep].reshape(-1), minlength=n_experts)
+    if not np.array_equal(kept_gpu, kept_ref):
+        bad += 1
+    if counts_gpu is not None:
+        own = np.bincount(idx_gpu.reshape(-1), minlength=n_experts)
+        if not np.array_equal(np.asarray(counts_gpu), own):
             bad += 1
     return bad, int((~keep).sum())
 
