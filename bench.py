@@ -648,7 +648,7 @@ def bench_prefill(args, rank, world, local):
                            "l2": "each chunk reads the whole 36 GB stack"},
                 "tflops_whole_step": tfl, "frac_of_burst_peak_whole_step": tfl / peak_burst,
                 "mean_active_experts_per_layer": float(u.mean()),
-                "roofline": roof, "clocks": clocks, "gpu_launches": K * nl * 8})
+                "roofline": roof, "clocks": clocks, "gpu_launches": K * nl * 7})
     moe.close()
     return res
 

@@ -30,6 +30,8 @@ MOE_FMT_Q2_32 = 0
 MOE_FMT_CB35_32 = 1
 MOE_F32 = 0
 MOE_BF16 = 1
+MOE_BIAS_LOGIT = 0
+MOE_BIAS_SELECT = 1
 
 DECODE_MAX_TOKENS = 8
 
@@ -41,12 +43,13 @@ class moe_config(C.Structure):
         ("n_shared", C.c_int32), ("shared_d_ff", C.c_int32), ("fmt", C.c_int32),
         ("act_dtype", C.c_int32), ("router_dtype", C.c_int32), ("out_dtype", C.c_int32),
         ("max_tokens", C.c_int32), ("codebook_grid", C.c_void_p), ("device", C.c_int32),
+        ("bias_mode", C.c_int32), ("shared_gate", C.c_int32),
     ]
 
 
 class moe_layer_weights(C.Structure):
     _fields_ = [("router_w", C.c_void_p), ("router_bias", C.c_void_p),
-                ("expert_blocks", C.c_void_p), ("shared_blocks", C.c_void_p)]
+                ("expert_blocks", C.c_void_p), ("shared_blocks", C.c_void_p), ("shared_gate_w", C.c_void_p)]
 
 
 class moe_route_out(C.Structure):
@@ -204,7 +207,7 @@ class MoE:
 
     def __init__(self, *, n_layers, d_model, d_ff, n_experts, top_k, n_shared=0, shared_d_ff=None,
                  fmt=MOE_FMT_Q2_32, act_dtype=MOE_BF16, router_dtype=MOE_BF16, out_dtype=MOE_F32,
-                 max_tokens=8, codebook_grid=None, device=0):
+                 max_tokens=8, codebook_grid=None, device=0, bias_mode=MOE_BIAS_LOGIT, shared_gate=0):
         self._grid = None
         if codebook_grid is not None:
             import numpy as np
@@ -213,16 +216,18 @@ class MoE:
         self.cfg = moe_config(C.sizeof(moe_config), n_layers, d_model, d_ff, n_experts, top_k, n_shared,
                               shared_d_ff if shared_d_ff is not None else d_ff, fmt, act_dtype, router_dtype,
                               out_dtype, max_tokens,
-                              None if self._grid is None else self._grid.ctypes.data, device)
+                              None if self._grid is None else self._grid.ctypes.data, device, bias_mode,
+                              int(shared_gate))
         self.h = moe_create(self.cfg)
 
     def _check(self, st: int, what: str):
         if st != MOE_OK:
             raise MoeError(st, f"{what}: {moe_last_error(self.h)}")
 
-    def load_layer(self, layer, router_w, router_bias, expert_blocks, shared_blocks=None):
-        w = moe_layer_weights(_ptr(router_w), _ptr(router_bias), _ptr(expert_blocks), _ptr(shared_blocks))
-        self._keep = (router_w, router_bias, expert_blocks, shared_blocks)
+    def load_layer(self, layer, router_w, router_bias, expert_blocks, shared_blocks=None, shared_gate_w=None):
+        w = moe_layer_weights(_ptr(router_w), _ptr(router_bias), _ptr(expert_blocks), _ptr(shared_blocks),
+                              _ptr(shared_gate_w))
+        self._keep = (router_w, router_bias, expert_blocks, shared_blocks, shared_gate_w)
         self._check(moe_load_layer(self.h, layer, w, _stream()), "moe_load_layer")
 
     def forward(self, layer, x, y, n_tokens=None, route=None):

@@ -127,6 +127,8 @@ void plan_workspace(moe_handle *h, Carve &c) {
   }
   const int td = D / kTileRows;
   w.logits = c.take<float>(static_cast<uint64_t>(kDecodeMaxTokens) * E);
+  w.raw_logits = c.take<float>(static_cast<uint64_t>(kDecodeMaxTokens) * E);
+  w.gate_logit = c.take<float>(kDecodeMaxTokens);
   w.sel = c.take<int>(kDecodeMaxTokens * K);
   w.route_sync = c.take<unsigned>(2);
   w.route_idx = c.take<int>(kDecodeMaxTokens * K);
@@ -284,7 +286,9 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
       (g.router_dtype != MOE_F32 && g.router_dtype != MOE_BF16) ||
       (g.out_dtype != MOE_F32 && g.out_dtype != MOE_BF16) || g.max_tokens < 1 || g.max_tokens > 8192 ||
       (g.fmt == MOE_FMT_CB35_32 && !g.codebook_grid) ||
-      g.d_ff > kMaxFF || (g.n_shared && g.shared_d_ff > kMaxFF) || g.d_model > kDecodeMaxD || g.device < 0;
+      g.d_ff > kMaxFF || (g.n_shared && g.shared_d_ff > kMaxFF) || g.d_model > kDecodeMaxD || g.device < 0 ||
+      (g.bias_mode != MOE_BIAS_LOGIT && g.bias_mode != MOE_BIAS_SELECT) || g.shared_gate < 0 ||
+      g.shared_gate > 1 || (g.shared_gate && g.n_shared != 1);
   if (bad) return MOE_ERR_INVALID_ARGUMENT;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || g.device >= ndev) {
@@ -301,6 +305,8 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
   h->sh.n_shared = g.n_shared;
   h->sh.fmt = g.fmt;
   h->sh.router_bf16 = g.router_dtype == MOE_BF16;
+  h->sh.bias_select = g.bias_mode == MOE_BIAS_SELECT;
+  h->sh.shared_gate = g.shared_gate;
   h->layers.assign(g.n_layers, LayerDev{});
   h->layer_mem.assign(g.n_layers, nullptr);
   h->layer_bytes.assign(g.n_layers, 0);
@@ -441,7 +447,7 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
   if (!h || !w) return MOE_ERR_INVALID_ARGUMENT;
   const moe_config &g = h->cfg;
   if (layer < 0 || layer >= g.n_layers) return fail(h, MOE_ERR_INVALID_ARGUMENT, "layer out of range");
-  if (!w->router_w || !w->expert_blocks || (g.n_shared && !w->shared_blocks))
+  if (!w->router_w || !w->expert_blocks || (g.n_shared && !w->shared_blocks) || (g.shared_gate && !w->shared_gate_w))
     return fail(h, MOE_ERR_INVALID_ARGUMENT, "missing weight pointer");
   DeviceGuard guard(g.device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -458,7 +464,9 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
   uint64_t ra, rs, rg, sa = 0, ss = 0, sg = 0;
   group_bytes(g.d_ff, E, ra, rs, rg);
   if (g.n_shared) group_bytes(g.shared_d_ff, 1, sa, ss, sg);
-  const uint64_t rw = align256(static_cast<uint64_t>(E) * D * dtype_size(g.router_dtype));
+  // router rows, then the shared expert's gate vector as row E
+  const uint64_t rrow = static_cast<uint64_t>(D) * dtype_size(g.router_dtype);
+  const uint64_t rw = align256(static_cast<uint64_t>(E + g.shared_gate) * rrow);
   const uint64_t bias_b = align256(static_cast<uint64_t>(E) * 4);
   const uint64_t total = ra + rs + rg + sa + ss + sg + rw + bias_b;
   // replace an earlier load of this layer
@@ -500,6 +508,11 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
   e = cudaMemcpyAsync(router_dst, w->router_w, static_cast<size_t>(E) * D * dtype_size(g.router_dtype),
                       cudaMemcpyDefault, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "router copy");
+  if (g.shared_gate) {
+    e = cudaMemcpyAsync(static_cast<char *>(router_dst) + static_cast<uint64_t>(E) * rrow, w->shared_gate_w, rrow,
+                        cudaMemcpyDefault, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "gate copy");
+  }
   if (w->router_bias)
     e = cudaMemcpyAsync(const_cast<float *>(L.bias), w->router_bias, static_cast<size_t>(E) * 4, cudaMemcpyDefault, st);
   else
@@ -555,7 +568,8 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
   };
   if ((s = load_group(L.routed, w->expert_blocks, E)) != MOE_OK) return s;
   if (g.n_shared && (s = load_group(L.shared, w->shared_blocks, 1)) != MOE_OK) return s;
-  if (!is_device_ptr(w->router_w) || (w->router_bias && !is_device_ptr(w->router_bias)))
+  if (!is_device_ptr(w->router_w) || (w->router_bias && !is_device_ptr(w->router_bias)) ||
+      (g.shared_gate && !is_device_ptr(w->shared_gate_w)))
     cudaStreamSynchronize(st);
   L.loaded = true;
   h->layers[layer] = L;

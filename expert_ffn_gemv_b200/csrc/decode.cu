@@ -135,6 +135,12 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 __device__ __forceinline__ void softmax_store(const DecodeArgs &a, int t, int lane, float my_l, float l0, int my_i,
                                               bool wr) {
   const int K = a.sh.k;
+  if (a.sh.bias_select) {  // selection by logit + bias, weights from the unbiased logits
+    my_l = lane < K ? __ldcg(a.ws.raw_logits + t * a.sh.e + my_i) : -INFINITY;
+    l0 = my_l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l0 = fmaxf(l0, __shfl_xor_sync(0xffffffffu, l0, o));
+  }
   if (lane == 0 && !(l0 > -INFINITY && l0 < INFINITY)) flag_error(a.err, kErrBadIndex);
   float w = lane < K ? __expf(my_l - l0) : 0.f;
   float sum = w;
@@ -414,6 +420,7 @@ template <bool RBF16, bool XBF16>
 __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
   __shared__ float red[kRouteWarps][kDecodeMaxTokens];
   const int D = a.sh.d, E = a.sh.e, n = a.n;
+  const int ER = E + a.sh.shared_gate;  // router rows: the experts, then the shared expert's gate
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int e = blockIdx.x * kRouteExperts + (warp >> 1), c0 = (warp & 1) * (D / 2);
   const int G = D / 16;  // 8-column groups per half
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
   float w[kRouteMaxG][8];
 #pragma unroll
   for (int i = 0; i < kRouteMaxG; ++i)
-    if (e < E && lane + 32 * i < G) load_row8<RBF16>(a.L.router_w, static_cast<int64_t>(e) * D + c0 + 8 * (lane + 32 * i), w[i]);
+    if (e < ER && lane + 32 * i < G) load_row8<RBF16>(a.L.router_w, static_cast<int64_t>(e) * D + c0 + 8 * (lane + 32 * i), w[i]);
   griddep_wait();
   griddep_launch();
   // the work queue and the h counters of this layer's GEMV kernel start empty (the previous
@@ -472,7 +479,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
 #pragma unroll
   for (int t = 0; t < kDecodeMaxTokens; ++t) {
     acc[t] = 0.f;
-    if (e < E && t < n) {
+    if (e < ER && t < n) {
       float xv[kRouteMaxG][8];
 #pragma unroll
       for (int i = 0; i < kRouteMaxG; ++i)
@@ -499,7 +506,13 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
   __syncthreads();
   if (tid < kRouteExperts * kDecodeMaxTokens) {
     const int j = tid / kDecodeMaxTokens, t = tid - j * kDecodeMaxTokens, ej = blockIdx.x * kRouteExperts + j;
-    if (t < n && ej < E) a.ws.logits[t * E + ej] = (red[2 * j][t] + red[2 * j + 1][t]) + a.L.bias[ej];
+    const float l = red[2 * j][t] + red[2 * j + 1][t];
+    if (t < n && ej < E) {
+      a.ws.logits[t * E + ej] = l + a.L.bias[ej];
+      if (a.sh.bias_select) a.ws.raw_logits[t * E + ej] = l;
+    } else if (t < n && ej == E && a.sh.shared_gate) {
+      a.ws.gate_logit[t] = l;
+    }
   }
 
   // ---- the last m = min(n, CTAs) CTAs to finish take the top-k (warp per token) once every
@@ -1434,7 +1447,8 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
   }
   const int64_t i = static_cast<int64_t>(t) * D + d;
   const float xs = a.residual ? load_act(a.x, i, a.x_bf16) : 0.f;
-  const float sh = a.sh.n_shared ? __ldcg(a.ws.o + i) : 0.f;  // u = 0 serves token t in slot t
+  float sh = a.sh.n_shared ? __ldcg(a.ws.o + i) : 0.f;  // u = 0 serves token t in slot t
+  if (a.sh.shared_gate) sh *= 1.0f / (1.0f + __expf(-__ldcg(a.ws.gate_logit + t)));
   __syncthreads();
   float v[kMaxTopK];
 #pragma unroll
@@ -1546,7 +1560,7 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
   cudaError_t err;
   // 1. router logits + input quantisation
   {
-    const int grid = (a.sh.e + kRouteExperts - 1) / kRouteExperts;
+    const int grid = (a.sh.e + a.sh.shared_gate + kRouteExperts - 1) / kRouteExperts;
     const int sm = a.sh.e > 1024 ? a.sh.e * 4 : 0;  // one logit row for the shared-memory top-k
     rec(a, kProfRoute, 0, st);
     if (a.sh.router_bf16)

@@ -49,7 +49,7 @@ struct ExpertGroup {
 };
 
 struct LayerDev {
-  const void *router_w;  // E x D, router dtype
+  const void *router_w;  // (E + shared_gate) x D, router dtype; row E is the shared expert's gate
   const float *bias;     // E
   ExpertGroup routed;
   ExpertGroup shared;    // count 0 when there is no shared expert
@@ -63,6 +63,8 @@ struct Shape {
   int n_shared;   // 0 or 1
   int fmt;        // MOE_FMT_*
   int router_bf16;
+  int bias_select;  // 1: the router bias enters the selection only (weights from unbiased logits)
+  int shared_gate;  // 1: the shared expert's output is scaled by sigmoid(g . x); g is router row E
 };
 
 // GEMV input of one token over one 64-column chunk (the layer input x for gate/up, the SwiGLU
@@ -85,7 +87,9 @@ static_assert(sizeof(ActRec) == 144, "ActRec is 9 x 16 bytes");
 // unit or several CTAs each take a run of segments (then the segment sums pass through the
 // partial buffers), so results do not depend on how the work was split.
 struct DecodeWs {
-  float *logits;        // [8][E]
+  float *logits;        // [8][E] selection scores (logit + bias)
+  float *raw_logits;    // [8][E] unbiased logits (selection-only bias)
+  float *gate_logit;    // [8] g . x of the gated shared expert
   int *sel;             // [8][k] selected experts per token, descending logit (the router's top-k)
   unsigned *route_sync; // [2] router CTAs done, top-k CTAs done
   int *route_idx;       // [8][k]

@@ -33,6 +33,8 @@ void plan_prefill_workspace(PrefillWs &w, const moe_config &g, char *base, uint6
   w.rows_max = static_cast<int>(n * (K + g.n_shared));
   w.fmax = fmax;
   w.logits = static_cast<float *>(take(n * E * 4));
+  w.raw_logits = static_cast<float *>(take(g.bias_mode == MOE_BIAS_SELECT ? n * E * 4 : 4));
+  w.gate_logit = static_cast<float *>(take(n * 4));
   w.route_idx = static_cast<int *>(take(n * K * 4));
   w.route_w = static_cast<float *>(take(n * K * 4));
   w.counts = static_cast<int *>(take((E + 1) * 4));
@@ -64,6 +66,7 @@ __global__ void __launch_bounds__(256) k_pf_router(PrefillArgs a) {
   __shared__ float As[kRtK][kRtM + 4];
   __shared__ float Bs[kRtK][kRtN + 4];
   const int D = a.sh.d, E = a.sh.e, n = a.n;
+  const int ER = E + a.sh.shared_gate;  // router rows: the experts, then the shared expert's gate
   const int t0 = blockIdx.x * kRtM, e0 = blockIdx.y * kRtN;
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
   float acc[4][4] = {};
@@ -76,9 +79,9 @@ __global__ void __launch_bounds__(256) k_pf_router(PrefillArgs a) {
       const int t = t0 + r, e = e0 + r;
       xv[i] = t < n ? pf_load_act(a.x, static_cast<int64_t>(t) * D + k0 + c, a.x_bf16) : 0.f;
       if (RBF16)
-        wv[i] = e < E ? __bfloat162float(static_cast<const __nv_bfloat16 *>(a.L.router_w)[static_cast<int64_t>(e) * D + k0 + c]) : 0.f;
+        wv[i] = e < ER ? __bfloat162float(static_cast<const __nv_bfloat16 *>(a.L.router_w)[static_cast<int64_t>(e) * D + k0 + c]) : 0.f;
       else
-        wv[i] = e < E ? static_cast<const float *>(a.L.router_w)[static_cast<int64_t>(e) * D + k0 + c] : 0.f;
+        wv[i] = e < ER ? static_cast<const float *>(a.L.router_w)[static_cast<int64_t>(e) * D + k0 + c] : 0.f;
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -108,7 +111,12 @@ __global__ void __launch_bounds__(256) k_pf_router(PrefillArgs a) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int e = e0 + tx * 4 + j;
-      if (e < E) a.ws.logits[static_cast<int64_t>(t) * E + e] = acc[i][j] + a.L.bias[e];
+      if (e < E) {
+        a.ws.logits[static_cast<int64_t>(t) * E + e] = acc[i][j] + a.L.bias[e];
+        if (a.sh.bias_select) a.ws.raw_logits[static_cast<int64_t>(t) * E + e] = acc[i][j];
+      } else if (e == E && a.sh.shared_gate) {
+        a.ws.gate_logit[t] = acc[i][j];
+      }
     }
   }
 }
@@ -161,6 +169,12 @@ __global__ void __launch_bounds__(256) k_pf_topk(PrefillArgs a) {
   }
   // fp32 softmax over the selected logits; a largest logit that is not finite leaves the
   // weights undefined: reported as a device fault
+  if (a.sh.bias_select) {  // selection by logit + bias, weights from the unbiased logits
+    my_l = lane < K ? a.ws.raw_logits[static_cast<int64_t>(t) * E + my_i] : -INFINITY;
+    l0 = my_l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l0 = fmaxf(l0, __shfl_xor_sync(0xffffffffu, l0, o));
+  }
   if (lane == 0 && !(l0 > -INFINITY && l0 < INFINITY)) flag_error(a.err, kErrBadIndex);
   float w = lane < K ? __expf(my_l - l0) : 0.f;
   float sum = w;
@@ -247,7 +261,7 @@ __global__ void __launch_bounds__(256) k_pf_scatter(PrefillArgs a) {
     t = static_cast<int>(asg - static_cast<int64_t>(n) * K);
     j = K;
     pos = a.ws.offsets[E] + t;
-    w = 1.f;
+    w = a.sh.shared_gate ? 1.0f / (1.0f + __expf(-a.ws.gate_logit[t])) : 1.f;  // gated shared expert
   }
   if (lane == 0) {
     a.ws.row_token[pos] = t;
@@ -884,7 +898,7 @@ cudaError_t launch_prefill_layer(const PrefillArgs &a, cudaStream_t st) {
   pf_rec(a, kProfRoute, 0, st);
   if ((err = cudaMemsetAsync(a.ws.counts, 0, sizeof(int) * (E + 1), st)) != cudaSuccess) return err;
   {
-    dim3 grid((n + kRtM - 1) / kRtM, (E + kRtN - 1) / kRtN);
+    dim3 grid((n + kRtM - 1) / kRtM, (E + a.sh.shared_gate + kRtN - 1) / kRtN);
     if (a.sh.router_bf16)
       k_pf_router<true><<<grid, 256, 0, st>>>(a);
     else

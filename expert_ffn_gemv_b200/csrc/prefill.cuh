@@ -20,7 +20,9 @@ struct PrefillWs {
   CUtensorMap tmap_hs;   // TMA view of hs
   int max_tokens;
   int rows_max;          // max_tokens * (k + n_shared)
-  float *logits;         // [n][E]
+  float *logits;         // [n][E] selection scores (logit + bias)
+  float *raw_logits;     // [n][E] unbiased logits (selection-only bias)
+  float *gate_logit;     // [n]    g . x of the gated shared expert
   int *route_idx;        // [n][k]
   float *route_w;        // [n][k]
   int *counts;           // [E + 1]   rows per group (group E = shared)

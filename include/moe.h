@@ -7,6 +7,8 @@
  *   w_j    = softmax of the selected logits (fp32)
  *   o_e    = Wd_e (silu(Wg_e x_t) * (Wu_e x_t))   SwiGLU expert FFN, silu(z) = z sigmoid(z)
  *   y_t    = sum_{j in S} w_j o_j + o_shared(x_t)
+ * Variants (moe_config): a selection-only router bias (bias_mode) and a sigmoid-gated shared
+ * expert (shared_gate), y_t = sum_j w_j o_j + sigmoid(g . x_t) o_shared(x_t).
  * A stack applies layers first..first+n-1 with a residual add, x <- x + y, kept in fp32.
  * Sources: the hao.cnyes.com Strata feature article, "Strata 到底是什麼" (48 layers x 512
  * experts, about 10 routed per token) and its section 1 (router and shared expert always
@@ -59,6 +61,10 @@ typedef enum {
 
 typedef enum { MOE_FMT_Q2_32 = 0, MOE_FMT_CB35_32 = 1 } moe_format;
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+/* How the router bias enters: MOE_BIAS_LOGIT adds b to the logits used for the selection and for
+ * the weights (the plain definition above); MOE_BIAS_SELECT selects the top_k of (logit + b) and
+ * weighs them by the softmax of their unbiased logits (a bias that only balances expert load). */
+typedef enum { MOE_BIAS_LOGIT = 0, MOE_BIAS_SELECT = 1 } moe_bias_mode;
 
 typedef struct moe_handle moe_handle; /* opaque */
 
@@ -79,6 +85,9 @@ typedef struct {
   int32_t max_tokens;     /* largest n_tokens per call, 1..8192: sizes the workspace */
   const int8_t *codebook_grid; /* host, 256 x 4 int8, copied at create; required iff CB35 */
   int32_t device;         /* CUDA device ordinal */
+  int32_t bias_mode;      /* moe_bias_mode */
+  int32_t shared_gate;    /* 1: o_shared is scaled by sigmoid(g . x_t), g a d_model vector given
+                             per layer (requires n_shared = 1); 0: weight 1 */
 } moe_config;
 
 typedef struct {
@@ -86,6 +95,8 @@ typedef struct {
   const float *router_bias;  /* host or device: n_experts fp32, or NULL (= 0) */
   const void *expert_blocks; /* host or device: n_experts experts, interchange bytes (above) */
   const void *shared_blocks; /* host or device: the shared expert; NULL iff n_shared == 0 */
+  const void *shared_gate_w; /* host or device: d_model values g (router_dtype); required iff
+                                cfg.shared_gate, else ignored */
 } moe_layer_weights;
 
 typedef struct {             /* device pointers, each may be NULL */

@@ -49,7 +49,11 @@ class _Layer(C.Structure):
         ("top_k", C.c_int), ("n_shared", C.c_int), ("shared_d_ff", C.c_int),
         ("grid", C.c_void_p), ("router_w", C.c_void_p), ("router_dtype", C.c_int),
         ("bias", C.c_void_p), ("experts", C.c_void_p), ("shared", C.c_void_p),
+        ("shared_gate", C.c_void_p), ("bias_mode", C.c_int),
     ]
+
+BIAS_LOGIT = 0
+BIAS_SELECT = 1
 
 
 def lib():
@@ -70,6 +74,9 @@ def lib():
         _lib.or_expert_ffn.argtypes = [I, P, I, I, P, P, P, P]
         _lib.or_router_logits.argtypes = [P, I, P, I, I, P, P]
         _lib.or_topk_softmax.argtypes = [P, I, I, P, P, P]
+        _lib.or_topk_select_softmax.argtypes = [P, P, I, I, P, P, P]
+        _lib.or_sigmoid.restype = C.c_double
+        _lib.or_sigmoid.argtypes = [C.c_double]
         _lib.or_moe_layer.argtypes = [P, P, I, P, P, P, P, P, I]
         _lib.or_moe_layer.restype = I
         _lib.or_route.argtypes = [P, P, I, P, P, P]
@@ -152,6 +159,20 @@ def router_logits(router_w, router_dtype, bias, x):
     return out
 
 
+def topk_select_softmax(score, wlogit, k):
+    sc = _c(score, np.float64)
+    wl = _c(wlogit, np.float64)
+    idx = np.empty(k, dtype=np.int32)
+    w = np.empty(k, dtype=np.float64)
+    m = np.empty(1, dtype=np.float64)
+    lib().or_topk_select_softmax(_p(sc), _p(wl), sc.size, k, _p(idx), _p(w), _p(m))
+    return idx, w, float(m[0])
+
+
+def sigmoid(z: float) -> float:
+    return lib().or_sigmoid(float(z))
+
+
 def topk_softmax(logits, k):
     lg = _c(logits, np.float64)
     idx = np.empty(k, dtype=np.int32)
@@ -169,7 +190,8 @@ class Layer:
     """
 
     def __init__(self, *, fmt, d_model, d_ff, n_experts, top_k, n_shared, shared_d_ff,
-                 router_w, router_dtype, bias=None, experts=None, shared=None, grid=None):
+                 router_w, router_dtype, bias=None, experts=None, shared=None, grid=None,
+                 shared_gate=None, bias_mode=BIAS_LOGIT):
         self.fmt, self.d_model, self.d_ff = fmt, d_model, d_ff
         self.n_experts, self.top_k = n_experts, top_k
         self.n_shared, self.shared_d_ff = n_shared, shared_d_ff
@@ -178,6 +200,9 @@ class Layer:
         self.bias = None if bias is None else _c(bias, np.float32)
         self.grid = None if grid is None else _c(grid, np.int8)
         self.shared = None if shared is None else _c(shared, np.uint8)
+        self.shared_gate = None if shared_gate is None else _c(
+            shared_gate, np.float32 if router_dtype == F32 else np.uint16)
+        self.bias_mode = int(bias_mode)
         self._experts: dict[int, np.ndarray] = {}
         if experts is not None:
             if isinstance(experts, dict):
@@ -196,7 +221,8 @@ class Layer:
             ptrs[e] = b.ctypes.data
         s = _Layer(self.fmt, self.d_model, self.d_ff, self.n_experts, self.top_k, self.n_shared,
                    self.shared_d_ff, _p(self.grid), _p(self.router_w), self.router_dtype,
-                   _p(self.bias), C.cast(ptrs, C.c_void_p), _p(self.shared))
+                   _p(self.bias), C.cast(ptrs, C.c_void_p), _p(self.shared), _p(self.shared_gate),
+                   self.bias_mode)
         return s, ptrs
 
     def route(self, x: np.ndarray):

@@ -131,34 +131,64 @@ void or_router_logits(const void *router_w, int router_dtype, const float *bias,
   }
 }
 
-/* Selection by repeated maximum: the j-th pick is the largest logit not yet taken; a strict
- * comparison keeps the lower index among equal logits. */
-void or_topk_softmax(const double *logits, int n_experts, int k, int32_t *idx, double *w,
-                     double *margin) {
+/* Selection by repeated maximum over `score`: the j-th pick is the largest score not yet taken;
+ * a strict comparison keeps the lower index among equal scores.  The weights are the softmax of
+ * `wlogit` over the picked experts (shifted by its largest value there). */
+void or_topk_select_softmax(const double *score, const double *wlogit, int n_experts, int k,
+                            int32_t *idx, double *w, double *margin) {
   char *taken = (char *)calloc((size_t)n_experts, 1);
   double lmax, sum = 0.0, next = INFINITY;
   int j, e;
   for (j = 0; j < k; ++j) {
     int best = -1;
     for (e = 0; e < n_experts; ++e)
-      if (!taken[e] && (best < 0 || logits[e] > logits[best])) best = e;
+      if (!taken[e] && (best < 0 || score[e] > score[best])) best = e;
     taken[best] = 1;
     idx[j] = best;
   }
   if (k < n_experts) {
     int best = -1;
     for (e = 0; e < n_experts; ++e)
-      if (!taken[e] && (best < 0 || logits[e] > logits[best])) best = e;
-    next = logits[best];
+      if (!taken[e] && (best < 0 || score[e] > score[best])) best = e;
+    next = score[best];
   }
-  if (margin) *margin = k < n_experts ? logits[idx[k - 1]] - next : INFINITY;
-  lmax = logits[idx[0]];
+  if (margin) *margin = k < n_experts ? score[idx[k - 1]] - next : INFINITY;
+  lmax = wlogit[idx[0]];
+  for (j = 1; j < k; ++j)
+    if (wlogit[idx[j]] > lmax) lmax = wlogit[idx[j]];
   for (j = 0; j < k; ++j) {
-    w[j] = exp(logits[idx[j]] - lmax);
+    w[j] = exp(wlogit[idx[j]] - lmax);
     sum += w[j];
   }
   for (j = 0; j < k; ++j) w[j] /= sum;
   free(taken);
+}
+
+void or_topk_softmax(const double *logits, int n_experts, int k, int32_t *idx, double *w,
+                     double *margin) {
+  or_topk_select_softmax(logits, logits, n_experts, k, idx, w, margin);
+}
+
+double or_sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+/* The router of one token: the selection scores and the logits the weights use (equal unless
+ * the bias is selection-only). */
+static void route_token(const or_layer *L, const double *x, double *score, double *wlogit) {
+  int e;
+  or_router_logits(L->router_w, L->router_dtype, NULL, L->n_experts, L->d_model, x, wlogit);
+  for (e = 0; e < L->n_experts; ++e) {
+    double b = L->bias ? (double)L->bias[e] : 0.0;
+    score[e] = wlogit[e] + b;
+    if (L->bias_mode != OR_BIAS_SELECT) wlogit[e] = score[e];
+  }
+}
+
+/* sigmoid(gate . x) of the gated shared expert (1 without a gate) */
+static double shared_scale(const or_layer *L, const double *x) {
+  double z;
+  if (!L->shared_gate) return 1.0;
+  or_router_logits(L->shared_gate, L->router_dtype, NULL, 1, L->d_model, x, &z);
+  return or_sigmoid(z);
 }
 
 static int check_shapes(const or_layer *L) {
@@ -170,17 +200,22 @@ static int check_shapes(const or_layer *L) {
   return 0;
 }
 
+/* Tokens are independent: the loop over them runs on OpenMP threads (same arithmetic per token). */
 int or_route(const or_layer *L, const double *x, int n, int32_t *idx, double *w, double *margin) {
   int t, rc = check_shapes(L);
   if (rc) return rc;
-  double *logits = (double *)malloc(sizeof(double) * L->n_experts);
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
   for (t = 0; t < n; ++t) {
-    or_router_logits(L->router_w, L->router_dtype, L->bias, L->n_experts, L->d_model,
-                     x + (size_t)t * L->d_model, logits);
-    or_topk_softmax(logits, L->n_experts, L->top_k, idx + (size_t)t * L->top_k,
-                    w + (size_t)t * L->top_k, margin ? margin + t : NULL);
+    double *score = (double *)malloc(sizeof(double) * L->n_experts);
+    double *wlogit = (double *)malloc(sizeof(double) * L->n_experts);
+    route_token(L, x + (size_t)t * L->d_model, score, wlogit);
+    or_topk_select_softmax(score, wlogit, L->n_experts, L->top_k, idx + (size_t)t * L->top_k,
+                           w + (size_t)t * L->top_k, margin ? margin + t : NULL);
+    free(score);
+    free(wlogit);
   }
-  free(logits);
   return 0;
 }
 
@@ -214,8 +249,9 @@ int or_moe_layer(const or_layer *L, const double *x, int n, double *y, int32_t *
         for (d = 0; d < D; ++d) yt[d] += w[(size_t)t * k + j] * o[d];
       }
       if (L->n_shared) {
+        double gs = shared_scale(L, xt);
         or_expert_ffn(L->fmt, L->shared, D, L->shared_d_ff, L->grid, xt, NULL, o);
-        for (d = 0; d < D; ++d) yt[d] += o[d];
+        for (d = 0; d < D; ++d) yt[d] += gs * o[d];
       }
       free(o);
     }

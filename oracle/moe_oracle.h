@@ -19,6 +19,11 @@
  *   4. per selected expert and the shared expert: g = Wg x, u = Wu x,
  *      h = silu(g) * u with silu(z) = z / (1 + exp(-z)), o = Wd h
  *   5. y = sum_j w_j o_j + o_shared      (a stack adds y to x after every layer)
+ * Two variants of steps 2-3 and 5 (off by default; readings of what checkpoints of this model
+ * family use, the pages name only "the router" and "the shared expert"):
+ *   - selection-only bias: S = the k largest (l_e + b_e), w = softmax over the unbiased l of S;
+ *   - gated shared expert: o_shared is multiplied by sigmoid(gate . x), gate a D-vector stored
+ *     like a router row.
  * Weights are dequantised block by block from the interchange bytes:
  *   Q2   (10 B / 32 weights): fp16 scale s, 2-bit codes q, w = s * (q - 1.5)
  *   CB35 (14 B / 32 weights): fp16 scale s, 8 grid-row indices (4 weights each),
@@ -51,7 +56,15 @@ typedef struct {
   const float *bias;    /* E, or NULL (= 0) */
   const uint8_t *const *experts; /* E pointers to [gate][up][down] blocks; NULL = not supplied */
   const uint8_t *shared;         /* shared expert blocks or NULL when n_shared == 0 */
+  /* variants (both off = the plain definition above) */
+  const void *shared_gate; /* D values (router_dtype) or NULL: o_shared is scaled by
+                              sigmoid(sum_d gate[d] x[d]) */
+  int bias_mode;           /* OR_BIAS_LOGIT (0): b enters selection and weights;
+                              OR_BIAS_SELECT (1): S = top-k of (logit + b), w = softmax of the
+                              unbiased logits of S */
 } or_layer;
+
+enum { OR_BIAS_LOGIT = 0, OR_BIAS_SELECT = 1 };
 
 /* exact conversions */
 double or_f16_to_f64(uint16_t h);
@@ -78,6 +91,12 @@ void or_router_logits(const void *router_w, int router_dtype, const float *bias,
  * (+inf when k == E).  idx/w in descending logit order. */
 void or_topk_softmax(const double *logits, int n_experts, int k, int32_t *idx, double *w,
                      double *margin);
+/* selection by `score` (as above), softmax over `wlogit` of the selected experts; margin on the
+ * scores.  or_topk_softmax(l) is or_topk_select_softmax(l, l). */
+void or_topk_select_softmax(const double *score, const double *wlogit, int n_experts, int k,
+                            int32_t *idx, double *w, double *margin);
+/* sigmoid(z) = 1 / (1 + exp(-z)) */
+double or_sigmoid(double z);
 /* one layer over n tokens: x (n x D) -> y (n x D).  idx, w (n x k), margin (n),
  * counts (E) may be NULL.  n_threads <= 0: OpenMP default.  Returns 0, or -1 when a
  * selected expert's pointer is NULL, or -2 on bad shapes. */

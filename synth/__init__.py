@@ -67,6 +67,7 @@ T_ROUTER = 1
 T_BIAS_PERM = 2
 T_X = 3
 T_GRID = 4
+T_SHARED_GATE = 5
 T_EXPERT = 16
 F_SCALE = 0
 F_CODES = 1
@@ -173,6 +174,8 @@ class Workload:
     beta: float = 0.5
     n_layers: int = 1
     n_tokens: int = 1
+    bias_select: bool = False   # router bias used for the selection only
+    shared_gate: bool = False   # sigmoid-gated shared expert (gate vector like a router row)
     extra: dict = field(default_factory=dict, compare=False, hash=False)
 
     @property
@@ -219,6 +222,15 @@ def gen_router(wl: Workload, seed: int, layer: int) -> np.ndarray:
     w = words_np(stream_key(seed, wl.wid, layer, T_ROUTER), 0, n)
     tab = normal_table(1.0 / math.sqrt(wl.d_model), wl.router_dtype)
     return tab[w & 0xFFFF].reshape(wl.n_experts, wl.d_model)
+
+
+def gen_shared_gate(wl: Workload, seed: int, layer: int) -> np.ndarray | None:
+    """Gate vector of a sigmoid-gated shared expert [D], stored like a router row (bf16 bits or
+    fp32), N(0, 1/D); None without a gate."""
+    if not (wl.shared_gate and wl.n_shared):
+        return None
+    w = words_np(stream_key(seed, wl.wid, layer, T_SHARED_GATE), 0, wl.d_model)
+    return normal_table(1.0 / math.sqrt(wl.d_model), wl.router_dtype)[w & 0xFFFF]
 
 
 def gen_bias(wl: Workload, seed: int, layer: int) -> np.ndarray | None:
@@ -388,6 +400,18 @@ def gen_router_torch(wl: Workload, seed: int, layer: int, device):
     if wl.router_dtype == DT_BF16:
         return v.view(torch.bfloat16).reshape(wl.n_experts, wl.d_model)
     return v.reshape(wl.n_experts, wl.d_model)
+
+
+def gen_shared_gate_torch(wl: Workload, seed: int, layer: int, device):
+    import torch
+
+    if not (wl.shared_gate and wl.n_shared):
+        return None
+    w = words_torch(stream_key(seed, wl.wid, layer, T_SHARED_GATE), 0, wl.d_model, device)
+    tab = _torch_table(("router", wl.d_model, wl.router_dtype),
+                       normal_table(1.0 / math.sqrt(wl.d_model), wl.router_dtype), device)
+    v = tab[w & 0xFFFF]
+    return v.view(torch.bfloat16) if wl.router_dtype == DT_BF16 else v
 
 
 def gen_x_torch(wl: Workload, seed: int, n_tokens: int, pass_idx: int, device, start_token: int = 0):

@@ -29,7 +29,8 @@ def oracle_layer(wl: synth.Workload, seed: int, layer: int, full: bool = True, g
         n_shared=wl.n_shared, shared_d_ff=wl.shared_d_ff, router_w=synth.gen_router(wl, seed, layer),
         router_dtype=wl.router_dtype, bias=synth.gen_bias(wl, seed, layer),
         experts=synth.gen_layer_experts(wl, seed, layer) if full else None,
-        shared=synth.gen_shared(wl, seed, layer), grid=grid)
+        shared=synth.gen_shared(wl, seed, layer), grid=grid, shared_gate=synth.gen_shared_gate(wl, seed, layer),
+        bias_mode=oracle.BIAS_SELECT if wl.bias_select else oracle.BIAS_LOGIT)
 
 
 def supply_from_generator(wl: synth.Workload, seed: int, layer_of=lambda l: l):
@@ -92,7 +93,8 @@ def moe_for(wl: synth.Workload, n_layers: int, max_tokens: int, seed: int = 0, o
     return P.MoE(n_layers=n_layers, d_model=wl.d_model, d_ff=wl.d_ff, n_experts=wl.n_experts, top_k=wl.top_k,
                  n_shared=wl.n_shared, shared_d_ff=wl.shared_d_ff, fmt=wl.fmt, act_dtype=wl.act_dtype,
                  router_dtype=wl.router_dtype, out_dtype=P.MOE_F32 if out_dtype is None else out_dtype,
-                 max_tokens=max_tokens, codebook_grid=grid, device=0)
+                 max_tokens=max_tokens, codebook_grid=grid, device=0,
+                 bias_mode=P.MOE_BIAS_SELECT if wl.bias_select else P.MOE_BIAS_LOGIT, shared_gate=int(wl.shared_gate))
 
 
 def load_layer_host(moe, slot: int, wl: synth.Workload, seed: int, layer: int):
@@ -101,7 +103,7 @@ def load_layer_host(moe, slot: int, wl: synth.Workload, seed: int, layer: int):
     router = np.ascontiguousarray(synth.gen_router(wl, seed, layer))
     bias = synth.gen_bias(wl, seed, layer)
     shared = synth.gen_shared(wl, seed, layer)
-    moe.load_layer(slot, router, bias, experts, shared)
+    moe.load_layer(slot, router, bias, experts, shared, synth.gen_shared_gate(wl, seed, layer))
 
 
 def load_layer_device(moe, slot: int, wl: synth.Workload, seed: int, layer: int, chunk: int = 64):
@@ -121,7 +123,8 @@ def load_layer_device(moe, slot: int, wl: synth.Workload, seed: int, layer: int,
     router = synth.gen_router_torch(wl, seed, layer, dev).contiguous()
     b = synth.gen_bias(wl, seed, layer)
     bias = None if b is None else torch.from_numpy(b).to(dev)
-    moe.load_layer(slot, router, bias, blocks, shared)
+    gate = synth.gen_shared_gate_torch(wl, seed, layer, dev)
+    moe.load_layer(slot, router, bias, blocks, shared, gate)
     torch.cuda.synchronize()
     del blocks, shared
 

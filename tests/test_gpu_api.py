@@ -24,16 +24,17 @@ def P():
 def _cfg(P, **kw):
     base = dict(n_layers=1, d_model=256, d_ff=128, n_experts=16, top_k=2, n_shared=0, shared_d_ff=128,
                 fmt=P.MOE_FMT_Q2_32, act_dtype=P.MOE_BF16, router_dtype=P.MOE_BF16, out_dtype=P.MOE_F32,
-                max_tokens=8, codebook_grid=None, device=0)
+                max_tokens=8, codebook_grid=None, device=0, bias_mode=0, shared_gate=0)
     base.update(kw)
     return P.moe_config(C.sizeof(P.moe_config), *[base[k] for k in (
         "n_layers", "d_model", "d_ff", "n_experts", "top_k", "n_shared", "shared_d_ff", "fmt", "act_dtype",
-        "router_dtype", "out_dtype", "max_tokens", "codebook_grid", "device")])
+        "router_dtype", "out_dtype", "max_tokens", "codebook_grid", "device", "bias_mode", "shared_gate")])
 
 
 @pytest.mark.parametrize("bad", [dict(d_model=200), dict(d_ff=96), dict(top_k=0), dict(top_k=17),
                                  dict(n_shared=2), dict(fmt=7), dict(max_tokens=0), dict(max_tokens=9000),
-                                 dict(fmt=1), dict(device=999), dict(n_experts=0)])
+                                 dict(fmt=1), dict(device=999), dict(n_experts=0), dict(bias_mode=2),
+                                 dict(shared_gate=1), dict(shared_gate=2, n_shared=1)])
 def test_create_rejects_bad_config(P, bad):
     h = C.c_void_p()
     assert P.lib().moe_create(C.byref(_cfg(P, **bad)), C.byref(h)) == P.MOE_ERR_INVALID_ARGUMENT

@@ -214,3 +214,29 @@ def test_stack_one_layer_equals_forward_plus_x(torch_cuda):
     torch.cuda.synchronize()
     assert torch.equal(out, x.float() + y)
     moe.close()
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+def test_stack_equals_chained_layers_bitwise(torch_cuda, fmt):
+    """Inside a stack each layer's combine also writes the next layer's activation records; a
+    chain of single-layer calls (residual added in fp32 by the caller) quantises its input in
+    the router kernel instead.  Both must give the same bits."""
+    torch = torch_cuda
+    wl = synth.small_workload(fmt=fmt, d_model=512, d_ff=256, n_experts=32, top_k=4, n_layers=3,
+                              act_dtype=synth.DT_F32)  # fp32 inputs, so each chained call takes the fp32 residual
+    nl, seed = 3, 8
+    moe = moe_for(wl, nl, 8, seed=seed)
+    for l in range(nl):
+        load_layer_device(moe, l, wl, seed, l)
+    for n in (1, 8):
+        x = x_device(wl, seed, n, pass_idx=n)
+        out = torch.empty((n, wl.d_model), dtype=torch.float32, device="cuda")
+        moe.forward_stack(0, nl, x, out)
+        cur = x.clone()
+        for l in range(nl):
+            y = torch.empty_like(cur)
+            moe.forward(l, cur, y)
+            cur = cur + y
+        torch.cuda.synchronize()
+        assert torch.equal(out, cur), f"{n} tokens: max diff {(out - cur).abs().max().item()}"
+    moe.close()

@@ -403,3 +403,85 @@ def test_threads_do_not_change_results():
     a = L.forward(x, n_threads=1)["y"]
     b = L.forward(x, n_threads=4)["y"]
     assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------ variants: selection-only bias, gated shared expert
+def test_select_only_bias_hand_worked():
+    # logits (2, 1, 0, -1), bias (0, 0, 3, 0), k = 2: scores (2, 1, 3, -1) select experts 2 then 0;
+    # the weights use the unbiased logits of {2, 0} = (0, 2): w = (1, e^2) / (1 + e^2)
+    l = np.array([2.0, 1.0, 0.0, -1.0])
+    b = np.array([0.0, 0.0, 3.0, 0.0])
+    idx, w, m = oracle.topk_select_softmax(l + b, l, 2)
+    e2 = math.e ** 2
+    assert list(idx) == [2, 0]
+    assert w[0] == pytest.approx(1 / (1 + e2), rel=1e-15)
+    assert w[1] == pytest.approx(e2 / (1 + e2), rel=1e-15)
+    assert m == 1.0  # score of the 2nd pick (2) minus the best unpicked score (1)
+    # with the bias in the weights too, the same selection weighs (3, 2)
+    idx2, w2, _ = oracle.topk_softmax(l + b, 2)
+    assert list(idx2) == [2, 0] and w2[0] == pytest.approx(math.e / (math.e + 1), rel=1e-15)
+
+
+def _unit_router_layer(bias, bias_mode, D=32, E=4, k=2):
+    W = np.zeros((E, D), dtype=np.float32)
+    for e in range(E):
+        W[e, e] = 1.0
+    return oracle.Layer(fmt=oracle.FMT_Q2, d_model=D, d_ff=32, n_experts=E, top_k=k, n_shared=0,
+                        shared_d_ff=32, router_w=W, router_dtype=oracle.F32, bias=bias, bias_mode=bias_mode)
+
+
+def test_select_only_bias_through_the_router():
+    # unit router rows: logit e = x[e]; the layer's route() applies the bias mode
+    x = np.zeros((1, 32))
+    x[0, :4] = [2.0, 1.0, 0.0, -1.0]
+    b = np.array([0.0, 0.0, 3.0, 0.0], dtype=np.float32)
+    e2 = math.e ** 2
+    idx, w, m = _unit_router_layer(b, oracle.BIAS_SELECT).route(x)
+    assert list(idx[0]) == [2, 0] and m[0] == 1.0
+    assert np.allclose(w[0], [1 / (1 + e2), e2 / (1 + e2)], rtol=1e-15)
+    idx, w, m = _unit_router_layer(b, oracle.BIAS_LOGIT).route(x)
+    assert list(idx[0]) == [2, 0]
+    assert np.allclose(w[0], [math.e / (math.e + 1), 1 / (math.e + 1)], rtol=1e-15)
+    # a zero bias makes the two modes equal
+    z = np.zeros(4, dtype=np.float32)
+    a = _unit_router_layer(z, oracle.BIAS_SELECT).route(x)
+    c = _unit_router_layer(z, oracle.BIAS_LOGIT).route(x)
+    assert all(np.array_equal(u, v) for u, v in zip(a, c))
+
+
+def test_sigmoid_closed_forms():
+    assert oracle.sigmoid(0.0) == 0.5
+    assert oracle.sigmoid(math.log(3.0)) == pytest.approx(0.75, rel=1e-15)
+    assert oracle.sigmoid(-math.log(3.0)) == pytest.approx(0.25, rel=1e-15)
+    assert oracle.sigmoid(50.0) == pytest.approx(1.0, abs=1e-15)
+
+
+def _gated(wl, gate, seed=0):
+    L = _layer(wl, seed)
+    L2 = oracle.Layer(fmt=wl.fmt, d_model=wl.d_model, d_ff=wl.d_ff, n_experts=wl.n_experts, top_k=wl.top_k,
+                      n_shared=wl.n_shared, shared_d_ff=wl.shared_d_ff, router_w=L.router_w,
+                      router_dtype=wl.router_dtype, bias=L.bias, experts=synth.gen_layer_experts(wl, seed, 0),
+                      shared=L.shared, shared_gate=gate)
+    return L, L2
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+def test_gated_shared_expert_closed_forms(fmt):
+    """y_gated = y_routed + sigmoid(gate . x) o_shared: with gate = 0 the shared term is halved
+    exactly; with gate = c x / |x|^2 (fp32 router dtype) the scale is sigmoid(c)."""
+    wl = synth.small_workload(fmt=fmt, router_dtype=synth.DT_F32, act_dtype=synth.DT_F32)
+    x = _x(wl, 1)[0]
+    grid = synth.gen_grid(wl, 0) if fmt == synth.FMT_CB35 else None
+    o_s = _dense_ffn(fmt, synth.gen_shared(wl, 0, 0), wl.d_model, wl.shared_d_ff, x, grid)
+    for gate, scale in ((np.zeros(wl.d_model, dtype=np.float32), 0.5),
+                        ((math.log(3.0) * x / np.dot(x, x)).astype(np.float32), None)):
+        L, Lg = _gated(wl, gate)
+        if grid is not None:
+            L.grid = Lg.grid = np.ascontiguousarray(grid)
+        y = L.forward(x[None])["y"][0]
+        yg = Lg.forward(x[None])["y"][0]
+        if scale is None:  # the fp32-rounded gate: scale from its exact dot product
+            scale = 1.0 / (1.0 + math.exp(-float(np.dot(gate.astype(np.float64), x))))
+            assert abs(scale - 0.75) < 1e-6
+        assert np.allclose(y - yg, (1.0 - scale) * o_s, rtol=1e-9, atol=1e-12 * np.abs(o_s).max())
+        assert np.array_equal(L.forward(x[None])["idx"], Lg.forward(x[None])["idx"])

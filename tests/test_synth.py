@@ -66,3 +66,18 @@ def test_zipf_bias():
     assert np.allclose(srt, 0.5 * np.log(r ** -1.1 / h), rtol=1e-6)
     assert synth.gen_bias(synth.TINY, 0, 0) is None
     assert not np.array_equal(synth.gen_bias(synth.DECODE, 0, 1), b.astype(np.float32))
+
+
+def test_numpy_torch_shared_gate_identical():
+    import dataclasses
+
+    for base in (synth.DECODE, synth.TINY):
+        wl = dataclasses.replace(base, shared_gate=True, n_shared=1)
+        g = synth.gen_shared_gate(wl, 3, 1)
+        gt = synth.gen_shared_gate_torch(wl, 3, 1, "cpu")
+        assert g.shape == (wl.d_model,)
+        if wl.router_dtype == synth.DT_BF16:
+            assert np.array_equal(gt.view(torch.int16).numpy().view(np.uint16), g)
+        else:
+            assert np.array_equal(gt.numpy(), g)
+    assert synth.gen_shared_gate(synth.DECODE, 3, 1) is None  # no gate unless asked for
