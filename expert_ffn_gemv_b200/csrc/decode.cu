@@ -49,9 +49,6 @@ constexpr int kRing = 4;                        // most stages of the bulk-copy 
 #define MOE_GEMV_UNROLL 1                       // chunks of a stage in flight per iteration
 #endif
 constexpr int kGemvUnroll = MOE_GEMV_UNROLL;
-#ifndef MOE_STREAMS_PER_SM
-#define MOE_STREAMS_PER_SM 6                    // GEMV pieces wanted in flight per SM (K split when fewer)
-#endif
 // ring depth: 4 stages for Q2; 3 for CB35, whose stages and grid table are larger
 #ifndef MOE_Q2_RING
 #define MOE_Q2_RING 4
@@ -360,10 +357,11 @@ __device__ __forceinline__ int udiv_small(int a, int b) {
   return q;
 }
 
-// Pieces per unit: K is cut only when there are fewer units than about min_streams (e.g. one
-// token's ~11 experts), so that enough pieces are in flight.  Returns the run length in segments.
-__device__ __forceinline__ int piece_run(int nseg, int units_total, int min_streams) {
-  int p = udiv_small(min_streams + units_total - 1, units_total);
+// Pieces per unit: floor(CTAs / units), so that K is cut only when the units are fewer than the
+// CTAs (e.g. one token's ~11 experts); a cut that cannot shorten the busiest CTA's queue would
+// only add partial sums and tickets.  Returns the run length in segments.
+__device__ __forceinline__ int piece_run(int nseg, int units_total, int ctas) {
+  int p = udiv_small(ctas, units_total);
   p = min(max(p, 1), nseg);
   return udiv_small(nseg + p - 1, p);
 }
@@ -1535,7 +1533,7 @@ cudaError_t configure_decode_kernels() {
 static int gemv_smem(int fmt, int umax) { return ring_plan(fmt, 1, kStageSlots, umax).total; }
 
 
-// Persistent grid: SMs x resident CTAs of the GEMV kernel; min_streams = MOE_STREAMS_PER_SM x SMs.
+// Persistent grid: SMs x resident CTAs of the GEMV kernel; min_streams = the grid (see piece_run).
 cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_streams) {
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1552,7 +1550,7 @@ cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_stream
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   *grid_gemv = nsm * occ;
-  *min_streams = MOE_STREAMS_PER_SM * nsm;
+  *min_streams = nsm * occ;
   return cudaSuccess;
 }
 

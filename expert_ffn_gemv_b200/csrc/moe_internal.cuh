@@ -116,7 +116,7 @@ struct DecodeWs {
   int gu_nseg;          // gate/up: K segments (d_model / 64 / gu_seg)
   int dn_nseg;          // down: most K segments of any expert
   int grid_gemv;        // persistent grid of the GEMV kernel
-  int min_streams;      // pieces wanted in flight (about two per SM)
+  int min_streams;      // the grid: units are cut into floor(grid / units) pieces
 };
 
 // ------------------------------------------------------------------------------------------
