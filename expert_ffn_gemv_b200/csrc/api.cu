@@ -17,6 +17,8 @@ struct moe_handle {
   Shape sh;
   std::vector<LayerDev> layers;
   std::vector<void *> layer_mem;
+  std::vector<CUtensorMap> router_maps;  // per layer: TMA view of the bf16 router rows (prompt chunks)
+  std::vector<uint8_t> router_map_ok;
   std::vector<uint64_t> layer_bytes;
   int8_t *grid_d = nullptr;
   void *ws_mem = nullptr;
@@ -234,6 +236,13 @@ moe_status run_layer(moe_handle *h, int layer, const void *x, int x_bf16, void *
     a.spin_limit = h->spin_limit;
     a.ev = ev;
     a.prof_mask = h->prof_mask;
+    // router logits on the tensor cores: bf16 router rows, and room in the gather buffer for
+    // x's two bf16 parts (a bf16 x needs one)
+    const int rows_per_token = h->cfg.top_k + h->cfg.n_shared;
+    if (h->router_map_ok[layer] && (x_bf16 || rows_per_token >= 2)) {
+      a.tc_router = 1;
+      a.tmap_router = h->router_maps[layer];
+    }
     e = launch_prefill_layer(a, st);
   }
   if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
@@ -309,6 +318,8 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
   h->sh.shared_gate = g.shared_gate;
   h->layers.assign(g.n_layers, LayerDev{});
   h->layer_mem.assign(g.n_layers, nullptr);
+  h->router_maps.resize(g.n_layers);
+  h->router_map_ok.assign(g.n_layers, 0);
   h->layer_bytes.assign(g.n_layers, 0);
   DeviceGuard guard(g.device);
   if (!guard.ok) {
@@ -573,6 +584,11 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
     cudaStreamSynchronize(st);
   L.loaded = true;
   h->layers[layer] = L;
+  h->router_map_ok[layer] = 0;
+  if (g.max_tokens > kDecodeMaxTokens && g.router_dtype == MOE_BF16 &&
+      make_router_tensor_map(&h->router_maps[layer], L.router_w, D, E + g.shared_gate) == cudaSuccess)
+    h->router_map_ok[layer] = 1;
+  cudaGetLastError();
   return MOE_OK;
 }
 

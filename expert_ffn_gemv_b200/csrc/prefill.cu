@@ -760,6 +760,144 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
 }
 
 // ------------------------------------------------------------------------------------------
+// router on the tensor cores (bf16 router rows)
+// ------------------------------------------------------------------------------------------
+// x as two bf16 parts, x_hi = bf16(x) and x_lo = bf16(x - x_hi), into the gather buffer (rows
+// 0 .. n-1: x_hi, rows n .. 2n-1: x_lo; free until the scatter); x_hi + x_lo keeps x to 2^-17 of
+// its magnitude.  A bf16 x is exact in x_hi alone (lo = 0: no x_lo rows).
+__global__ void __launch_bounds__(256) k_pf_xsplit(PrefillArgs a, int lo) {
+  const int64_t total = static_cast<int64_t>(a.n) * a.sh.d;
+  const int64_t i8 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (i8 >= total) return;
+  float v[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v[q] = pf_load_act(a.x, i8 + q, a.x_bf16);
+  __nv_bfloat162 h[4], l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    h[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    const float2 hf = __bfloat1622float2(h[q]);
+    l[q] = __floats2bfloat162_rn(v[2 * q] - hf.x, v[2 * q + 1] - hf.y);
+  }
+  *reinterpret_cast<uint4 *>(a.ws.xs + i8) = *reinterpret_cast<const uint4 *>(h);
+  if (lo) *reinterpret_cast<uint4 *>(a.ws.xs + total + i8) = *reinterpret_cast<const uint4 *>(l);
+}
+
+// Logits of 128 router rows x 256 tokens per CTA: tcgen05.mma kind::f16 (bf16 router rows as A,
+// M = 128; the tokens' x_hi and x_lo as B, N = 256), both parts into one fp32 accumulator in TMEM,
+// K-steps of 64 through a 2-stage TMA ring; then + bias (the gate row: g . x; selection-only bias:
+// the unbiased logits too).  One thread issues the loads and the MMAs; four warps read TMEM.
+constexpr int kRtA = 128 * 128, kRtB = kPfBN * 128, kRtStage = kRtA + 2 * kRtB;
+constexpr int kRtBytes = 1024 + 1024 + 2 * kRtStage;
+
+__global__ void __launch_bounds__(128, 1) k_pf_router_tc(const __grid_constant__ PrefillArgs a, int lo) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2]
+  uint64_t *empty = full + 2;                          // [2]
+  uint64_t *acc_full = empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
+  unsigned char *stages = smem + 1024;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int D = a.sh.d, E = a.sh.e, ER = E + a.sh.shared_gate, n = a.n;
+  const int mtiles = (ER + 127) / 128;
+  const int m0 = (blockIdx.x % mtiles) * 128, t0 = (blockIdx.x / mtiles) * kPfBN;
+  const int nk = D / kChunk;
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kPfBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t lim = a.spin_limit;
+  volatile int abort_flag_v = 0;
+  volatile int *abort_flag = &abort_flag_v;
+  if (tid == 0) {
+    const uint32_t tx = kRtA + kRtB * (lo ? 2 : 1);
+    int issued = 0;
+    auto load = [&](int s) {
+      ++issued;
+      unsigned char *sb = stages + (s & 1) * kRtStage;
+      mbar_arrive_expect_tx(&full[s & 1], tx);
+      tma_load_2d(sb, &a.tmap_router, s * kChunk, m0, &full[s & 1]);
+      tma_load_2d(sb + kRtA, &a.ws.tmap_xs, s * kChunk, t0, &full[s & 1]);
+      if (lo) tma_load_2d(sb + kRtA + kRtB, &a.ws.tmap_xs, s * kChunk, n + t0, &full[s & 1]);
+    };
+    load(0);
+    if (nk > 1) load(1);
+    const uint32_t idesc = idesc_bf16(kPfBN);
+    const uint64_t d0 = sw128_desc(smem_u32(stages));
+    bool ok = true;
+    int s = 0;
+    for (; s < nk && ok; ++s) {
+      const int st = s & 1;
+      if (!(ok = pf_wait(&full[st], (s >> 1) & 1u, lim, abort_flag, a.err))) break;
+      tc_fence_after();
+      const uint64_t ad = d0 + static_cast<uint64_t>((st * kRtStage) >> 4);
+      const uint64_t bh = d0 + static_cast<uint64_t>((st * kRtStage + kRtA) >> 4);
+      const uint64_t bl = d0 + static_cast<uint64_t>((st * kRtStage + kRtA + kRtB) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) tc_mma(tmem, ad + 2 * kk, bh + 2 * kk, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+      if (lo) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) tc_mma(tmem, ad + 2 * kk, bl + 2 * kk, idesc, 1u);
+      }
+      tc_commit(&empty[st]);
+      if (s + 2 < nk) {  // the stage is free once its MMAs have read it
+        if (!(ok = pf_wait(&empty[st], (s >> 1) & 1u, lim, abort_flag, a.err))) break;
+        load(s + 2);
+      }
+    }
+    if (ok) tc_commit(acc_full);
+    // nothing may be in flight when the CTA leaves: the last stages' loads and MMAs
+    for (int k = (issued > 2 ? issued - 2 : 0); k < issued; ++k)
+      mbar_wait_bounded(&full[k & 1], (k >> 1) & 1u, kDrainLimit);
+    if (s > 0) mbar_wait_bounded(&empty[(s - 1) & 1], ((s - 1) >> 1) & 1u, kDrainLimit);
+    if (!ok) flag_error(a.err, kErrTimeout);
+  }
+  __syncwarp();
+  // epilogue: warp w reads TMEM lanes 32w .. 32w+31 = router rows m0 + 32w + lane
+  const bool have = mbar_wait_bounded(acc_full, 0, lim);
+  tc_fence_after();
+  const int e = m0 + 32 * warp + lane;
+  if (have) {
+    const float b = e < E ? a.L.bias[e] : 0.f;
+    for (int c0 = 0; c0 < kPfBN; c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32_nowait(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int t = t0 + c0 + i;
+        if (t >= n) break;
+        const float l = __uint_as_float(v[i]);
+        if (e < E) {
+          a.ws.logits[static_cast<int64_t>(t) * E + e] = l + b;
+          if (a.sh.bias_select) a.ws.raw_logits[static_cast<int64_t>(t) * E + e] = l;
+        } else if (e == E && a.sh.shared_gate) {
+          a.ws.gate_logit[t] = l;
+        }
+      }
+    }
+  } else if (tid == 0) {
+    flag_error(a.err, kErrTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kPfBN);
+}
+
+// ------------------------------------------------------------------------------------------
 // combine: y[t] = sum_j outs[pos(t, j)] + outs[pos(t, shared)] (+ x[t]), slot order
 // ------------------------------------------------------------------------------------------
 // CTA per token, thread = 8 consecutive columns: 16-byte loads of the token's K + 1 weighted
@@ -848,6 +986,7 @@ cudaError_t configure_prefill_kernels() {
                              PfPlan<MOE_FMT_CB35_32, 1>::kBytes);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_pf_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * kMaxExperts * 4);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_pf_router_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kRtBytes);
   return e;
 }
 
@@ -863,7 +1002,8 @@ static inline void pf_rec(const PrefillArgs &a, int kind, int end, cudaStream_t 
 
 // 2-D tensor map over a bf16 [rows][cols] row-major buffer: boxes of 64 columns x kPfBN rows with
 // the 128-byte swizzle (the UMMA K-major layout); rows past the end read as zeros.
-static cudaError_t make_tmap(CUtensorMap *map, void *base, uint64_t cols, uint64_t rows) {
+static cudaError_t make_tmap(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                             uint32_t box_rows = kPfBN) {
   using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -878,9 +1018,9 @@ static cudaError_t make_tmap(CUtensorMap *map, void *base, uint64_t cols, uint64
   }
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(kPfBN)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -892,12 +1032,24 @@ cudaError_t make_prefill_tensor_maps(PrefillWs &w, int d_model) {
   return e;
 }
 
+cudaError_t make_router_tensor_map(CUtensorMap *map, const void *router_w, int d_model, int router_rows) {
+  return make_tmap(map, router_w, static_cast<uint64_t>(d_model), static_cast<uint64_t>(router_rows), 128);
+}
+
 cudaError_t launch_prefill_layer(const PrefillArgs &a, cudaStream_t st) {
   cudaError_t err;
   const int E = a.sh.e, K = a.sh.k, n = a.n;
   pf_rec(a, kProfRoute, 0, st);
   if ((err = cudaMemsetAsync(a.ws.counts, 0, sizeof(int) * (E + 1), st)) != cudaSuccess) return err;
-  {
+  if (a.tc_router) {
+    const int lo = a.x_bf16 ? 0 : 1;  // a bf16 x has no low part
+    const int64_t total = static_cast<int64_t>(n) * a.sh.d;
+    k_pf_xsplit<<<static_cast<unsigned>((total / 8 + 255) / 256), 256, 0, st>>>(a, lo);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int tiles = ((E + a.sh.shared_gate + 127) / 128) * ((n + kPfBN - 1) / kPfBN);
+    k_pf_router_tc<<<tiles, 128, kRtBytes, st>>>(a, lo);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  } else {
     dim3 grid((n + kRtM - 1) / kRtM, (E + a.sh.shared_gate + kRtN - 1) / kRtN);
     if (a.sh.router_bf16)
       k_pf_router<true><<<grid, 256, 0, st>>>(a);

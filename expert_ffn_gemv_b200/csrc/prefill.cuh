@@ -42,6 +42,8 @@ struct PrefillWs {
 };
 
 struct PrefillArgs {
+  CUtensorMap tmap_router;  // TMA view of the layer's bf16 router rows (boxes of 64 x 128), if tc_router
+  int tc_router;            // 1: router logits on the tensor cores (bf16 router rows), else CUDA cores
   Shape sh;
   LayerDev L;
   PrefillWs ws;
@@ -64,6 +66,8 @@ struct PrefillArgs {
 
 void plan_prefill_workspace(PrefillWs &w, const moe_config &g, char *base, uint64_t &off);
 cudaError_t make_prefill_tensor_maps(PrefillWs &w, int d_model);
+// TMA view of a layer's bf16 router rows (router_rows x d_model), for the tensor-core router
+cudaError_t make_router_tensor_map(CUtensorMap *map, const void *router_w, int d_model, int router_rows);
 cudaError_t configure_prefill_kernels();
 cudaError_t launch_prefill_layer(const PrefillArgs &a, cudaStream_t st);
 
