@@ -414,11 +414,23 @@ constexpr int kEpiThreads = 256;
 constexpr int kDeqThreads = 32 * kDeqWarps;
 constexpr int kDeqSub = kDeqWarps / 8;                 // threads sharing one (row, block)
 
+#ifndef MOE_PF_STAGES0
+#define MOE_PF_STAGES0 4
+#endif
+#ifndef MOE_PF_ABUFS0
+#define MOE_PF_ABUFS0 2
+#endif
+#ifndef MOE_PF_STAGES1
+#define MOE_PF_STAGES1 5
+#endif
+#ifndef MOE_PF_ABUFS1
+#define MOE_PF_ABUFS1 2
+#endif
 template <int FMT, int MODE>
 struct PfPlan {
   static constexpr int NM = MODE == 0 ? 2 : 1;
-  static constexpr int kStages = MODE == 0 ? 4 : 5;            // (raw + B) stages
-  static constexpr int kABufs = 2;                              // bf16 A buffers
+  static constexpr int kStages = MODE == 0 ? MOE_PF_STAGES0 : MOE_PF_STAGES1;  // (raw + B) stages
+  static constexpr int kABufs = MODE == 0 ? MOE_PF_ABUFS0 : MOE_PF_ABUFS1;     // bf16 A buffers
   static constexpr int kAcc = MODE == 0 ? 1 : 2;               // accumulator buffers
   static constexpr int kATile = 128 * 128;                      // 128 x 64 bf16
   static constexpr int kBTile = kPfBN * 128;                    // kPfBN x 64 bf16
