@@ -24,6 +24,7 @@ _lib = None
 
 FMT_Q2 = 0
 FMT_CB35 = 1
+FMT_NVFP4 = 2
 F32 = 0
 BF16 = 1
 F64 = 2
@@ -67,6 +68,13 @@ def lib():
         _lib.or_bf16_to_f64.argtypes = [C.c_uint16]
         _lib.or_convert_to_f64.argtypes = [P, I, C.c_size_t, P]
         _lib.or_dequant_block.argtypes = [I, P, P, P]
+        _lib.or_e2m1_to_f64.restype = C.c_double
+        _lib.or_e2m1_to_f64.argtypes = [I]
+        _lib.or_e4m3_to_f64.restype = C.c_double
+        _lib.or_e4m3_to_f64.argtypes = [C.c_uint8]
+        _lib.or_block_weights.argtypes = [I]
+        _lib.or_matrix_bytes.restype = C.c_size_t
+        _lib.or_matrix_bytes.argtypes = [I, I, I]
         _lib.or_dequant_matrix.argtypes = [I, P, I, I, P, P]
         _lib.or_matvec.argtypes = [I, P, I, I, P, P, P]
         _lib.or_silu.restype = C.c_double
@@ -110,12 +118,29 @@ def to_f64(a: np.ndarray, dtype: int) -> np.ndarray:
     return out
 
 
+def e2m1_to_f64(code: int) -> float:
+    return lib().or_e2m1_to_f64(int(code))
+
+
+def e4m3_to_f64(b: int) -> float:
+    return lib().or_e4m3_to_f64(int(b))
+
+
+def block_weights(fmt: int) -> int:
+    return lib().or_block_weights(fmt)
+
+
+def matrix_bytes(fmt: int, rows: int, cols: int) -> int:
+    return lib().or_matrix_bytes(fmt, rows, cols)
+
+
 def dequant_block(fmt: int, blk: np.ndarray, grid: np.ndarray | None = None) -> np.ndarray:
+    """One block's weights (32; NVFP4: 16, without its matrix's tensor scale)."""
     b = _c(blk, np.uint8)
     g = None if grid is None else _c(grid, np.int8)
     out = np.empty(32, dtype=np.float64)
     lib().or_dequant_block(fmt, _p(b), _p(g), _p(out))
-    return out
+    return out[:block_weights(fmt)]
 
 
 def dequant_matrix(fmt, blocks, rows, cols, grid=None) -> np.ndarray:

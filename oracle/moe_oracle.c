@@ -48,7 +48,41 @@ void or_convert_to_f64(const void *src, int dtype, size_t n, double *dst) {
   }
 }
 
-int or_block_bytes(int fmt) { return fmt == OR_FMT_Q2 ? 10 : 14; }
+int or_block_bytes(int fmt) { return fmt == OR_FMT_Q2 ? 10 : fmt == OR_FMT_CB35 ? 14 : 9; }
+int or_block_weights(int fmt) { return fmt == OR_FMT_NVFP4 ? 16 : 32; }
+/* bytes before a matrix's blocks: NVFP4 starts every matrix with its fp32 tensor scale */
+int or_matrix_header(int fmt) { return fmt == OR_FMT_NVFP4 ? 4 : 0; }
+size_t or_matrix_bytes(int fmt, int rows, int cols) {
+  return (size_t)or_matrix_header(fmt) + (size_t)rows * (cols / or_block_weights(fmt)) * or_block_bytes(fmt);
+}
+
+/* FP4 E2M1 (1 sign, 2 exponent, 1 mantissa bit; no infinities or NaN): exponent 0 is
+ * subnormal, m * 0.5; otherwise 2^(e - 1) * (1 + m / 2). */
+double or_e2m1_to_f64(int code) {
+  int e = (code >> 1) & 3, m = code & 1;
+  double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return (code & 8) ? -v : v;
+}
+
+/* FP8 E4M3 in its finite form (bias 7, no infinities, 0x7F / 0xFF are NaN): exponent 0 is
+ * subnormal, m / 8 * 2^-6; otherwise 2^(e - 7) * (1 + m / 8). */
+double or_e4m3_to_f64(uint8_t b) {
+  int e = (b >> 3) & 15, m = b & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+  return (b & 0x80) ? -v : v;
+}
+
+static float le_f32(const uint8_t *p) {
+  uint32_t u = (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* tensor scale of a matrix (1 unless NVFP4) */
+static double matrix_scale(int fmt, const uint8_t *mat) { return fmt == OR_FMT_NVFP4 ? (double)le_f32(mat) : 1.0; }
 
 /* One 32-weight block.
  * Q2:   bytes 0-1 fp16 scale (little endian); weight i's 2-bit code q sits in byte 2 + i/4 at
@@ -56,8 +90,16 @@ int or_block_bytes(int fmt) { return fmt == OR_FMT_Q2 ? 10 : 14; }
  * CB35: bytes 0-1 fp16 scale; byte 2+g is the grid row for weights 4g..4g+3; bytes 10-13 a
  *       little-endian 32-bit sign mask, bit i set negates weight i; w_i = s * sign * grid[row][i%4]. */
 void or_dequant_block(int fmt, const uint8_t *blk, const int8_t *grid, double w[32]) {
-  double s = or_f16_to_f64((uint16_t)(blk[0] | (blk[1] << 8)));
+  double s;
   int i;
+  if (fmt == OR_FMT_NVFP4) {
+    /* NVFP4 (16 weights): byte 0 the E4M3 block scale, bytes 1-8 the E2M1 codes, weight i in
+     * byte 1 + i/2 (low nibble for even i); w_i = s * e2m1(code_i) (times the tensor scale) */
+    s = or_e4m3_to_f64(blk[0]);
+    for (i = 0; i < 16; ++i) w[i] = s * or_e2m1_to_f64((blk[1 + i / 2] >> (4 * (i % 2))) & 15);
+    return;
+  }
+  s = or_f16_to_f64((uint16_t)(blk[0] | (blk[1] << 8)));
   if (fmt == OR_FMT_Q2) {
     for (i = 0; i < 32; ++i) {
       int q = (blk[2 + i / 4] >> (2 * (i % 4))) & 3;
@@ -75,23 +117,28 @@ void or_dequant_block(int fmt, const uint8_t *blk, const int8_t *grid, double w[
   }
 }
 
-void or_dequant_matrix(int fmt, const uint8_t *blocks, int rows, int cols, const int8_t *grid,
-                       double *out) {
-  int bb = or_block_bytes(fmt), nb = cols / 32, r, b;
+void or_dequant_matrix(int fmt, const uint8_t *mat, int rows, int cols, const int8_t *grid, double *out) {
+  int bb = or_block_bytes(fmt), bw = or_block_weights(fmt), nb = cols / bw, r, b, i;
+  const double g = matrix_scale(fmt, mat);
+  const uint8_t *blocks = mat + or_matrix_header(fmt);
   for (r = 0; r < rows; ++r)
-    for (b = 0; b < nb; ++b)
-      or_dequant_block(fmt, blocks + ((size_t)r * nb + b) * bb, grid, out + (size_t)r * cols + 32 * b);
+    for (b = 0; b < nb; ++b) {
+      double *o = out + (size_t)r * cols + bw * b;
+      or_dequant_block(fmt, blocks + ((size_t)r * nb + b) * bb, grid, o);
+      for (i = 0; i < bw; ++i) o[i] *= g;
+    }
 }
 
-void or_matvec(int fmt, const uint8_t *blocks, int rows, int cols, const int8_t *grid,
-               const double *x, double *y) {
-  int bb = or_block_bytes(fmt), nb = cols / 32, r, b, i;
+void or_matvec(int fmt, const uint8_t *mat, int rows, int cols, const int8_t *grid, const double *x, double *y) {
+  int bb = or_block_bytes(fmt), bw = or_block_weights(fmt), nb = cols / bw, r, b, i;
+  const double g = matrix_scale(fmt, mat);
+  const uint8_t *blocks = mat + or_matrix_header(fmt);
   double w[32];
   for (r = 0; r < rows; ++r) {
     double acc = 0.0;
     for (b = 0; b < nb; ++b) {
       or_dequant_block(fmt, blocks + ((size_t)r * nb + b) * bb, grid, w);
-      for (i = 0; i < 32; ++i) acc += w[i] * x[32 * b + i];
+      for (i = 0; i < bw; ++i) acc += g * w[i] * x[bw * b + i];
     }
     y[r] = acc;
   }
@@ -101,7 +148,7 @@ double or_silu(double z) { return z / (1.0 + exp(-z)); }
 
 void or_expert_ffn(int fmt, const uint8_t *expert, int d_model, int d_ff, const int8_t *grid,
                    const double *x, double *h, double *y) {
-  size_t mat = (size_t)d_ff * d_model / 32 * or_block_bytes(fmt);
+  size_t mat = or_matrix_bytes(fmt, d_ff, d_model); /* gate and up; down has the same size */
   double *g = (double *)malloc(sizeof(double) * d_ff);
   double *u = (double *)malloc(sizeof(double) * d_ff);
   double *hh = (double *)malloc(sizeof(double) * d_ff);
@@ -192,6 +239,7 @@ static double shared_scale(const or_layer *L, const double *x) {
 }
 
 static int check_shapes(const or_layer *L) {
+  if (L->fmt != OR_FMT_Q2 && L->fmt != OR_FMT_CB35 && L->fmt != OR_FMT_NVFP4) return -2;
   if (L->d_model <= 0 || L->d_model % 32 || L->d_ff <= 0 || L->d_ff % 32) return -2;
   if (L->top_k < 1 || L->top_k > L->n_experts) return -2;
   if (L->n_shared < 0 || L->n_shared > 1) return -2;

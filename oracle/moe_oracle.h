@@ -28,6 +28,9 @@
  *   Q2   (10 B / 32 weights): fp16 scale s, 2-bit codes q, w = s * (q - 1.5)
  *   CB35 (14 B / 32 weights): fp16 scale s, 8 grid-row indices (4 weights each),
  *        32 sign bits, w = s * sign * grid[idx][i % 4]
+ *   NVFP4 (9 B / 16 weights, after a 4-byte fp32 tensor scale g per matrix): an FP8 E4M3 block
+ *        scale s and 16 FP4 E2M1 codes, w = g * s * e2m1(code)  (the pages list an NVIDIA-only
+ *        NVFP4 file among the supported models: hao.cnyes.com, "支援的模型與版本")
  */
 #ifndef MOE_ORACLE_H
 #define MOE_ORACLE_H
@@ -39,7 +42,7 @@
 extern "C" {
 #endif
 
-enum { OR_FMT_Q2 = 0, OR_FMT_CB35 = 1 };
+enum { OR_FMT_Q2 = 0, OR_FMT_CB35 = 1, OR_FMT_NVFP4 = 2 };
 enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
 
 typedef struct {
@@ -72,14 +75,17 @@ double or_bf16_to_f64(uint16_t b);
 void or_convert_to_f64(const void *src, int dtype, size_t n, double *dst);
 
 int or_block_bytes(int fmt);
-/* dequantise one 32-weight block */
+int or_block_weights(int fmt);
+int or_matrix_header(int fmt);
+size_t or_matrix_bytes(int fmt, int rows, int cols);
+double or_e2m1_to_f64(int code);
+double or_e4m3_to_f64(uint8_t b);
+/* dequantise one block (32 weights; NVFP4: 16, without the matrix's tensor scale) */
 void or_dequant_block(int fmt, const uint8_t *blk, const int8_t *grid, double w[32]);
-/* dequantise a rows x cols matrix stored as row-major blocks along the columns */
-void or_dequant_matrix(int fmt, const uint8_t *blocks, int rows, int cols, const int8_t *grid,
-                       double *out);
-/* y = W x, W given as blocks (rows x cols), dequantised block by block */
-void or_matvec(int fmt, const uint8_t *blocks, int rows, int cols, const int8_t *grid,
-               const double *x, double *y);
+/* dequantise a rows x cols matrix (its header, then row-major blocks along the columns) */
+void or_dequant_matrix(int fmt, const uint8_t *mat, int rows, int cols, const int8_t *grid, double *out);
+/* y = W x, W given as a matrix of blocks (rows x cols), dequantised block by block */
+void or_matvec(int fmt, const uint8_t *mat, int rows, int cols, const int8_t *grid, const double *x, double *y);
 double or_silu(double z);
 /* one expert's SwiGLU FFN: y (D) = Wd (silu(Wg x) * (Wu x)); h (F) optional */
 void or_expert_ffn(int fmt, const uint8_t *expert, int d_model, int d_ff, const int8_t *grid,

@@ -26,6 +26,9 @@ shared expert, 2-bit and 3.5-bit block files):
 * 2-bit codes: uniform, the bytes of hash words;
 * codebook grid 256x4 int8, entries uniform over {1, 3, ..., 15};
 * codebook indices (uint8) and sign bits: uniform, bytes of hash words;
+* NVFP4: E2M1 codes uniform (bytes of hash words); E4M3 block scales with exponent field
+  5..8 and mantissa 0..7 uniform (0.25 .. 3.75); the matrix's fp32 tensor scale
+  2^-8 (1 + u/8), u uniform in 0..7;
 * N(0, sigma^2) activations / router weights: 16 hash bits index a table of
   the 65,536 mid-quantiles sigma * Phi^-1((u + 1/2) / 65536), rounded to the
   storage dtype (bf16 round-to-nearest-even, or fp32);
@@ -39,6 +42,9 @@ Block interchange layouts (what ``moe_load_layer`` and the oracle consume):
 * CB35 (14 bytes / 32 weights): bytes 0-1 fp16 scale, bytes 2-9 grid row
   indices (byte 2+g covers weights 4g .. 4g+3), bytes 10-13 a little-endian
   uint32 of sign bits (bit i set: weight i negated).
+* NVFP4 (9 bytes / 16 weights, after a 4-byte little-endian fp32 tensor scale at
+  the start of every matrix): byte 0 the E4M3 block scale, bytes 1-8 the E2M1
+  codes, weight i in byte 1 + i/2 (low nibble for even i).
 
 Blocks run along a matrix row (the reduction dimension); rows are contiguous.
 An expert is [gate (F x D)][up (F x D)][down (D x F)]; experts are contiguous
@@ -57,7 +63,10 @@ M32 = 0xFFFFFFFF
 
 FMT_Q2 = 0
 FMT_CB35 = 1
-BLOCK_BYTES = {FMT_Q2: 10, FMT_CB35: 14}
+FMT_NVFP4 = 2
+BLOCK_BYTES = {FMT_Q2: 10, FMT_CB35: 14, FMT_NVFP4: 9}
+BLOCK_WEIGHTS = {FMT_Q2: 32, FMT_CB35: 32, FMT_NVFP4: 16}
+MATRIX_HEADER = {FMT_Q2: 0, FMT_CB35: 0, FMT_NVFP4: 4}  # NVFP4: the matrix's fp32 tensor scale
 
 DT_F32 = 0
 DT_BF16 = 1
@@ -73,6 +82,7 @@ F_SCALE = 0
 F_CODES = 1
 F_IDX = 2
 F_SIGN = 3
+F_TSCALE = 4
 
 
 # ----------------------------------------------------------------------------------------------
@@ -182,9 +192,12 @@ class Workload:
     def block_bytes(self) -> int:
         return BLOCK_BYTES[self.fmt]
 
-    def expert_bytes(self, shared: bool = False) -> int:
+    def matrix_bytes(self, shared: bool = False) -> int:
         f = self.shared_d_ff if shared else self.d_ff
-        return 3 * f * self.d_model // 32 * self.block_bytes
+        return MATRIX_HEADER[self.fmt] + f * self.d_model // BLOCK_WEIGHTS[self.fmt] * self.block_bytes
+
+    def expert_bytes(self, shared: bool = False) -> int:
+        return 3 * self.matrix_bytes(shared)
 
 
 # The five synthetic workloads (sizes of the pages' model; see module docstring)
@@ -195,8 +208,9 @@ VERIFY = Workload("verify-stack-48L-8tok-q2", 2, 2048, 768, 512, 10, 1, 768, n_l
 CODEBOOK = Workload("codebook-stack-48L-cb35", 3, 2048, 768, 512, 10, 1, 768, fmt=FMT_CB35,
                     n_layers=48, n_tokens=8)
 PREFILL = Workload("prefill-stack-48L-q2", 4, 2048, 768, 512, 10, 1, 768, n_layers=48, n_tokens=8192)
+NVFP4 = Workload("nvfp4-stack-48L", 5, 2048, 768, 512, 10, 1, 768, fmt=FMT_NVFP4, n_layers=48, n_tokens=8)
 
-WORKLOADS = {w.wid: w for w in (TINY, DECODE, VERIFY, CODEBOOK, PREFILL)}
+WORKLOADS = {w.wid: w for w in (TINY, DECODE, VERIFY, CODEBOOK, PREFILL, NVFP4)}
 
 
 def small_workload(**kw) -> Workload:
@@ -254,7 +268,21 @@ def gen_x(wl: Workload, seed: int, n_tokens: int, pass_idx: int = 0, start_token
     return normal_table(1.0, wl.act_dtype)[w & 0xFFFF].reshape(n_tokens, d)
 
 
+def _nvfp4_matrix_np(key_base: tuple, rows: int, cols: int) -> np.ndarray:
+    nb = rows * cols // 16
+    head = np.array([2.0 ** -8 * (1 + int(words_np(stream_key(*key_base, F_TSCALE), 0, 1)[0] & 7) / 8)],
+                    dtype=np.float32).view(np.uint8)
+    out = np.empty((nb, 9), dtype=np.uint8)
+    sw = words_np(stream_key(*key_base, F_SCALE), 0, nb)
+    out[:, 0] = (((5 + (sw & 3)) << 3) | ((sw >> 2) & 7)).astype(np.uint8)
+    c = words_np(stream_key(*key_base, F_CODES), 0, 2 * nb).astype(np.uint32)
+    out[:, 1:9] = c.view(np.uint8).reshape(nb, 8)
+    return np.concatenate([head, out.reshape(-1)])
+
+
 def _matrix_blocks_np(wl: Workload, key_base: tuple, rows: int, cols: int) -> np.ndarray:
+    if wl.fmt == FMT_NVFP4:
+        return _nvfp4_matrix_np(key_base, rows, cols)
     nb = rows * cols // 32
     bb = wl.block_bytes
     out = np.empty((nb, bb), dtype=np.uint8)
@@ -356,10 +384,14 @@ def gen_experts_torch(wl: Workload, seed: int, layer: int, experts, out):
     f = wl.shared_d_ff if shared else wl.d_ff
     bb = wl.block_bytes
     stab = _torch_table("scale", scale_table_f16(), dev)
-    nb = f * d // 32  # blocks per matrix (gate, up and down have the same count)
+    nb = f * d // BLOCK_WEIGHTS[wl.fmt]  # blocks per matrix (gate, up and down have the same count)
     off = 0
     for m in range(3):
         keys = [(seed, wl.wid, layer, T_EXPERT, e, m) for e in experts]
+        if wl.fmt == FMT_NVFP4:
+            _nvfp4_matrices_torch(keys, nb, out[:, off:off + 4 + nb * 9])
+            off += 4 + nb * 9
+            continue
 
         def kk(field_id):
             ks = [stream_key(*k, field_id) for k in keys]
@@ -387,6 +419,31 @@ def gen_experts_torch(wl: Workload, seed: int, layer: int, experts, out):
             sg = words(F_SIGN, nb)
             view[:, :, 10:14] = _u32_bytes_torch(sg).reshape(len(experts), nb, 4)
         off += nb * bb
+
+
+def _nvfp4_matrices_torch(keys, nb: int, out):
+    """NVFP4 matrices (one per key) into out (uint8 [len(keys), 4 + 9 nb]): the fp32 tensor scale,
+    then the blocks (the numpy recipe of _nvfp4_matrix_np)."""
+    import torch
+
+    dev = out.device
+    heads = np.array([2.0 ** -8 * (1 + int(words_np(stream_key(*k, F_TSCALE), 0, 1)[0] & 7) / 8) for k in keys],
+                     dtype=np.float32).view(np.uint8).reshape(len(keys), 4)
+    out[:, 0:4] = torch.from_numpy(heads).to(dev)
+
+    def words(field_id, count):
+        ks = [stream_key(*k, field_id) for k in keys]
+        k0 = torch.tensor([a for a, _ in ks], dtype=torch.int64, device=dev)[:, None]
+        k1 = torch.tensor([b for _, b in ks], dtype=torch.int64, device=dev)[:, None]
+        i = torch.arange(count, dtype=torch.int64, device=dev)[None, :]
+        return hash32((hash32(i ^ k0) + k1) & M32)
+
+    view = out[:, 4:].view(len(keys), nb, 9)
+    sw = words(F_SCALE, nb)
+    view[:, :, 0] = (((5 + (sw & 3)) << 3) | ((sw >> 2) & 7)).to(torch.uint8)
+    del sw
+    c = words(F_CODES, 2 * nb)
+    view[:, :, 1:9] = _u32_bytes_torch(c).reshape(len(keys), nb, 8)
 
 
 def gen_router_torch(wl: Workload, seed: int, layer: int, device):

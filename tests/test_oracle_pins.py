@@ -89,14 +89,15 @@ def test_dequant_matrix_block_placement():
 
 
 # ------------------------------------------------------------------ matvec: brute force
-@pytest.mark.parametrize("fmt", [oracle.FMT_Q2, oracle.FMT_CB35])
+@pytest.mark.parametrize("fmt", [oracle.FMT_Q2, oracle.FMT_CB35, oracle.FMT_NVFP4])
 def test_matvec_equals_dense_bruteforce(fmt):
     wl = synth.small_workload(d_model=64, d_ff=96, fmt=fmt)
     e = synth.gen_expert(wl, 3, 0, 1)
     grid = synth.gen_grid(wl, 3) if fmt == oracle.FMT_CB35 else None
     rng = np.random.default_rng(0)
     x = rng.standard_normal(64)
-    mat = 96 * 64 // 32 * wl.block_bytes
+    mat = wl.matrix_bytes()
+    assert mat == oracle.matrix_bytes(fmt, 96, 64)
     gate_dense = oracle.dequant_matrix(fmt, e[:mat], 96, 64, grid)
     y = oracle.matvec(fmt, e[:mat], 96, 64, x, grid)
     assert np.allclose(y, gate_dense @ x, rtol=1e-12, atol=1e-12)
@@ -257,7 +258,7 @@ def _x(wl, n, seed=0):
 
 def _dense_ffn(fmt, blocks, D, F, x, grid=None):
     """Textbook SwiGLU FFN on dense fp64 matrices (numpy matmul)."""
-    mat = F * D // 32 * (10 if fmt == oracle.FMT_Q2 else 14)
+    mat = oracle.matrix_bytes(fmt, F, D)
     Wg = oracle.dequant_matrix(fmt, blocks[:mat], F, D, grid)
     Wu = oracle.dequant_matrix(fmt, blocks[mat:2 * mat], F, D, grid)
     Wd = oracle.dequant_matrix(fmt, blocks[2 * mat:], D, F, grid)
@@ -265,7 +266,7 @@ def _dense_ffn(fmt, blocks, D, F, x, grid=None):
     return Wd @ (g / (1 + np.exp(-g)) * u)
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35, synth.FMT_NVFP4])
 def test_weights_sum_to_one_and_counts(fmt):
     wl = synth.small_workload(fmt=fmt)
     L = _layer(wl)
@@ -276,7 +277,7 @@ def test_weights_sum_to_one_and_counts(fmt):
         assert len(set(r["idx"][t])) == wl.top_k
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35, synth.FMT_NVFP4])
 def test_top1_equals_dense_expert_plus_shared(fmt):
     wl = synth.small_workload(fmt=fmt, top_k=1, d_model=128, d_ff=96, shared_d_ff=64)
     L = _layer(wl, seed=4)
@@ -485,3 +486,60 @@ def test_gated_shared_expert_closed_forms(fmt):
             assert abs(scale - 0.75) < 1e-6
         assert np.allclose(y - yg, (1.0 - scale) * o_s, rtol=1e-9, atol=1e-12 * np.abs(o_s).max())
         assert np.array_equal(L.forward(x[None])["idx"], Lg.forward(x[None])["idx"])
+
+
+# ------------------------------------------------------------------ NVFP4 blocks
+@pytest.mark.parametrize("code,val", [
+    (0, 0.0), (1, 0.5), (2, 1.0), (3, 1.5), (4, 2.0), (5, 3.0), (6, 4.0), (7, 6.0),
+    (9, -0.5), (10, -1.0), (13, -3.0), (15, -6.0),
+])
+def test_e2m1_decode(code, val):
+    assert oracle.e2m1_to_f64(code) == val
+
+
+def test_e2m1_negative_zero():
+    v = oracle.e2m1_to_f64(8)
+    assert v == 0.0 and math.copysign(1.0, v) == -1.0
+
+
+@pytest.mark.parametrize("b,val", [
+    (0x38, 1.0), (0x40, 2.0), (0x3C, 1.5), (0x41, 2.25), (0x37, 0.9375), (0x7E, 448.0),
+    (0x08, 2.0 ** -6), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x00, 0.0), (0xB8, -1.0),
+])
+def test_e4m3_decode(b, val):
+    assert oracle.e4m3_to_f64(b) == val
+
+
+def test_e4m3_nan():
+    assert math.isnan(oracle.e4m3_to_f64(0x7F)) and math.isnan(oracle.e4m3_to_f64(0xFF))
+
+
+def test_nvfp4_block_golden():
+    gd = _read_golden("nvfp4_block.txt")
+    blk = np.array([int(b, 16) for b in gd["bytes"]], dtype=np.uint8)
+    k = np.array([int(v) for v in gd["k"]], dtype=np.float64)
+    w = oracle.dequant_block(oracle.FMT_NVFP4, blk)
+    assert w.shape == (16,)
+    assert np.array_equal(w, k * 2.25 / 2)
+
+
+def test_nvfp4_matrix_tensor_scale_and_layout():
+    """Header = the fp32 tensor scale; blocks of 16 row-major along the columns: a 2 x 32
+    matrix of 4 hand-set blocks, dequantised and compared element by element."""
+    g = np.array([0.75], dtype=np.float32)
+    blocks = []
+    for r in range(2):
+        for b in range(2):
+            scale = 0x38 + 8 * (2 * r + b)  # 1, 2, 4, 8 (exponent steps of one)
+            codes = [(2 * r + b + i) % 8 for i in range(16)]  # positive codes
+            byts = [codes[2 * j] | (codes[2 * j + 1] << 4) for j in range(8)]
+            blocks.append([scale] + byts)
+    mat = np.concatenate([g.view(np.uint8), np.array(blocks, dtype=np.uint8).reshape(-1)])
+    assert mat.size == oracle.matrix_bytes(oracle.FMT_NVFP4, 2, 32)
+    W = oracle.dequant_matrix(oracle.FMT_NVFP4, mat, 2, 32)
+    e2m1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for r in range(2):
+        for b in range(2):
+            s = 2.0 ** (2 * r + b)
+            for i in range(16):
+                assert W[r, 16 * b + i] == 0.75 * s * e2m1[(2 * r + b + i) % 8]

@@ -81,3 +81,18 @@ def test_numpy_torch_shared_gate_identical():
         else:
             assert np.array_equal(gt.numpy(), g)
     assert synth.gen_shared_gate(synth.DECODE, 3, 1) is None  # no gate unless asked for
+
+
+def test_nvfp4_expert_bytes_identical_and_sized():
+    wl = synth.small_workload(fmt=synth.FMT_NVFP4, d_model=256, d_ff=128, n_experts=4, top_k=2)
+    assert wl.matrix_bytes() == 4 + 128 * 256 // 16 * 9
+    out = torch.empty((2, wl.expert_bytes()), dtype=torch.uint8)
+    synth.gen_experts_torch(wl, 3, 1, [1, 2], out)
+    for i, e in enumerate((1, 2)):
+        assert np.array_equal(out[i].numpy(), synth.gen_expert(wl, 3, 1, e))
+    # E4M3 scales within the recipe (exponent field 5..8, sign 0), tensor scales 2^-8 (1 + u/8)
+    m = synth.gen_expert(wl, 3, 1, 1)[:wl.matrix_bytes()]
+    g = float(m[:4].view(np.float32)[0])
+    assert g * 256 * 8 in range(8, 16)
+    s = m[4:].reshape(-1, 9)[:, 0]
+    assert np.all((s >> 3) >= 5) and np.all((s >> 3) <= 8) and np.all(s < 0x80)
