@@ -10,9 +10,11 @@ Default workload (one JSON line on stdout, rank 0):
 
 Also: --workload decode (1 token through 16 model-scale layers of seeds 0-15, one step = the 16
 layers), --workload codebook (3.5-bit codebook blocks, 48 independent layers on the same x),
---workload prefill (1,180 / 8,192-token chunks through the stack, grouped GEMM path).
+--workload prefill (1,180 / 8,192-token chunks through the stack, grouped GEMM path),
+--workload nvfp4 (the verify stack with NVFP4 blocks: E2M1 weights, E4M3 block scales, fp32
+tensor scale per matrix).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload verify|decode|codebook|prefill]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload verify|nvfp4|decode|codebook|prefill]
   python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample, same metric
 
 Multi-GPU: replicas only (each rank holds the full stack and its own token stream; no
@@ -260,12 +262,20 @@ def oracle_sample_stack(wl, seed, n_tokens, n_layers_sample, pass_idx=0, threads
 
 
 # ------------------------------------------------------------------------------------ verify stack
+WEIGHTS_DESC = {synth.FMT_Q2: "Q2 2-bit blocks, 10 B / 32 weights",
+                synth.FMT_CB35: "CB35 3.5-bit codebook blocks, 14 B / 32 weights",
+                synth.FMT_NVFP4: "NVFP4 blocks (E2M1 x E4M3 scale, 9 B / 16 weights, fp32 tensor scale per matrix)"}
+GEMV_DTYPE = {synth.FMT_Q2: "q2 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
+              synth.FMT_CB35: "cb35 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
+              synth.FMT_NVFP4: "nvfp4 (2 x e2m1 int8) x int16 acts (dp2a, i32) -> f32 accumulate"}
+
+
 def verify_config(wl, L):
     """The workload description both arms print (static: identical in the reference arm)."""
     return {"workload": wl.name, "d_model": wl.d_model, "d_ff": wl.d_ff, "n_experts": wl.n_experts,
             "top_k": wl.top_k, "n_shared": wl.n_shared, "layers": L, "tokens_per_pass": wl.n_tokens,
-            "weights": "Q2 2-bit blocks, 10 B / 32 weights", "router_bias": "Zipf(1.1), beta 0.5",
-            "l2": "inputs larger than L2: each pass reads ~4 GB of distinct expert blocks (126 MB L2)",
+            "weights": WEIGHTS_DESC[wl.fmt], "router_bias": "Zipf(1.1), beta 0.5",
+            "l2": "inputs larger than L2: each pass reads several GB of distinct expert blocks (126 MB L2)",
             "parallelism": "replicas (one process per GPU, no data-path collective)"}
 
 
@@ -291,7 +301,7 @@ def bench_verify(args, rank, world, local):
 
     import expert_ffn_gemv_b200 as P
 
-    wl = synth.VERIFY
+    wl = synth.NVFP4 if args.workload == "nvfp4" else synth.VERIFY
     L = args.layers
     n = wl.n_tokens
     K, W = args.steps, args.warmup
@@ -385,7 +395,7 @@ def bench_verify(args, rank, world, local):
     hbm_peak = pk["hbm_gbs"]
     achieved = gemv_bytes_last / (gu_ms / 1e3) / 1e9 if gu_ms > 0 else None
     src = source_hash("expert_ffn_gemv_b200/csrc/decode.cu", "expert_ffn_gemv_b200/csrc/moe_internal.cuh")
-    traffic = profiled_traffic("k_gemv", "verify", src, gemv_bytes_last / max(gu_cnt, 1))
+    traffic = profiled_traffic("k_gemv", args.workload, src, gemv_bytes_last / max(gu_cnt, 1))
     res = {
         "metric": METRIC,
         "value": value,
@@ -397,7 +407,7 @@ def bench_verify(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "q2 blocks x int16 acts (dp2a, i32) -> f32 accumulate",
+        "dtype": GEMV_DTYPE[wl.fmt],
         "data": "synthetic (seeded integer-hash generator, random-init weights)",
         "config": verify_config(wl, L),
         "resident_weight_gb": round(moe.device_bytes() / 1e9, 2),
@@ -662,7 +672,7 @@ def bench_reference(args):
     sys.path.insert(0, str(ROOT / "tests"))
     from helpers import oracle_layer, supply_from_generator
 
-    wl = synth.VERIFY
+    wl = synth.NVFP4 if args.workload == "nvfp4" else synth.VERIFY
     L, n, seed = args.layers, wl.n_tokens, args.seed
     cache = {}
 
@@ -726,7 +736,7 @@ def main():
     ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["verify", "decode", "codebook", "prefill"], default="verify")
+    ap.add_argument("--workload", choices=["verify", "nvfp4", "decode", "codebook", "prefill"], default="verify")
     ap.add_argument("--chunk", type=int, default=8192, help="prefill chunk tokens")
     ap.add_argument("--layers", type=int, default=48)
     ap.add_argument("--seed", type=int, default=0)
@@ -748,7 +758,7 @@ def main():
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         return relaunch(args.gpus)
     rank, world, local = dist_setup(args.gpus, "gloo" if args.plumbing_check else "nccl")
-    fn = {"verify": bench_verify, "decode": bench_decode_layers, "codebook": bench_codebook,
+    fn = {"verify": bench_verify, "nvfp4": bench_verify, "decode": bench_decode_layers, "codebook": bench_codebook,
           "prefill": bench_prefill}[args.workload]
     if args.plumbing_check:
         fn = bench_plumbing

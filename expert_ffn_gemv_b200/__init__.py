@@ -28,6 +28,7 @@ MOE_ERR_DEVICE_FAULT = 7
 
 MOE_FMT_Q2_32 = 0
 MOE_FMT_CB35_32 = 1
+MOE_FMT_NVFP4_16 = 2
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_BIAS_LOGIT = 0

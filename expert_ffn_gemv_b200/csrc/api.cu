@@ -290,7 +290,7 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
       g.d_ff < kTileRows || g.d_ff % kTileRows || g.n_experts < 1 || g.n_experts > kMaxExperts ||
       g.top_k < 1 || g.top_k > g.n_experts || g.top_k > kMaxTopK || g.n_shared < 0 || g.n_shared > 1 ||
       (g.n_shared && (g.shared_d_ff < kTileRows || g.shared_d_ff % kTileRows)) ||
-      (g.fmt != MOE_FMT_Q2_32 && g.fmt != MOE_FMT_CB35_32) ||
+      (g.fmt != MOE_FMT_Q2_32 && g.fmt != MOE_FMT_CB35_32 && g.fmt != MOE_FMT_NVFP4_16) ||
       (g.act_dtype != MOE_F32 && g.act_dtype != MOE_BF16) ||
       (g.router_dtype != MOE_F32 && g.router_dtype != MOE_BF16) ||
       (g.out_dtype != MOE_F32 && g.out_dtype != MOE_BF16) || g.max_tokens < 1 || g.max_tokens > 8192 ||
@@ -463,23 +463,30 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
   DeviceGuard guard(g.device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D = g.d_model, E = g.n_experts;
-  const int BB = g.fmt == MOE_FMT_Q2_32 ? 10 : 14;
-  const bool cb = g.fmt == MOE_FMT_CB35_32;
-  // plane sizes
-  auto group_bytes = [&](int f, int count, uint64_t &a, uint64_t &s, uint64_t &gg) {
+  const bool nv = g.fmt == MOE_FMT_NVFP4_16;
+  const bool has_g = has_plane_g(g.fmt);
+  const int abytes = plane_a_bytes(g.fmt);
+  // interchange bytes of one matrix (NVFP4: its fp32 tensor scale, then 9-byte blocks of 16)
+  auto mat_bytes_of = [&](int f) -> uint64_t {
     const uint64_t fd = static_cast<uint64_t>(f) * D;
-    a = align256(fd / 4 * 3 * count);
-    s = align256(fd / 64 * 4 * 3 * count);
-    gg = cb ? align256(fd / 64 * 8 * 3 * count) : 0;
+    return nv ? 4 + fd / 16 * 9 : fd / 32 * (g.fmt == MOE_FMT_Q2_32 ? 10 : 14);
   };
-  uint64_t ra, rs, rg, sa = 0, ss = 0, sg = 0;
-  group_bytes(g.d_ff, E, ra, rs, rg);
-  if (g.n_shared) group_bytes(g.shared_d_ff, 1, sa, ss, sg);
+  // plane sizes (+ NVFP4 tensor scales)
+  auto group_bytes = [&](int f, int count, uint64_t &a, uint64_t &s, uint64_t &gg, uint64_t &t) {
+    const uint64_t fd = static_cast<uint64_t>(f) * D;
+    a = align256(fd / 64 * abytes * 3 * count);
+    s = align256(fd / 64 * 4 * 3 * count);
+    gg = has_g ? align256(fd / 64 * 8 * 3 * count) : 0;
+    t = nv ? align256(static_cast<uint64_t>(3) * count * 4) : 0;
+  };
+  uint64_t ra, rs, rg, rt, sa = 0, ss = 0, sg = 0, st_ = 0;
+  group_bytes(g.d_ff, E, ra, rs, rg, rt);
+  if (g.n_shared) group_bytes(g.shared_d_ff, 1, sa, ss, sg, st_);
   // router rows, then the shared expert's gate vector as row E
   const uint64_t rrow = static_cast<uint64_t>(D) * dtype_size(g.router_dtype);
   const uint64_t rw = align256(static_cast<uint64_t>(E + g.shared_gate) * rrow);
   const uint64_t bias_b = align256(static_cast<uint64_t>(E) * 4);
-  const uint64_t total = ra + rs + rg + sa + ss + sg + rw + bias_b;
+  const uint64_t total = ra + rs + rg + rt + sa + ss + sg + st_ + rw + bias_b;
   // replace an earlier load of this layer
   if (h->layer_mem[layer]) {
     cudaStreamSynchronize(st);
@@ -495,22 +502,24 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
   h->layer_bytes[layer] = total;
   char *p = static_cast<char *>(mem);
   LayerDev L{};
-  auto fill_group = [&](ExpertGroup &G, int f, int count, uint64_t a, uint64_t sb, uint64_t gb) {
+  auto fill_group = [&](ExpertGroup &G, int f, int count, uint64_t a, uint64_t sb, uint64_t gb, uint64_t tb) {
     const uint64_t fd = static_cast<uint64_t>(f) * D;
     G.a = reinterpret_cast<uint8_t *>(p);
     p += a;
     G.s = reinterpret_cast<__half2 *>(p);
     p += sb;
-    G.g = cb ? reinterpret_cast<uint2 *>(p) : nullptr;
+    G.g = has_g ? reinterpret_cast<uint2 *>(p) : nullptr;
     p += gb;
-    G.a_mat = static_cast<int64_t>(fd / 4);
+    G.ts = nv ? reinterpret_cast<float *>(p) : nullptr;
+    p += tb;
+    G.a_mat = static_cast<int64_t>(fd / 64 * abytes);
     G.s_mat = static_cast<int64_t>(fd / 64);
     G.g_mat = static_cast<int64_t>(fd / 64);
     G.f = f;
     G.count = count;
   };
-  fill_group(L.routed, g.d_ff, E, ra, rs, rg);
-  if (g.n_shared) fill_group(L.shared, g.shared_d_ff, 1, sa, ss, sg);
+  fill_group(L.routed, g.d_ff, E, ra, rs, rg, rt);
+  if (g.n_shared) fill_group(L.shared, g.shared_d_ff, 1, sa, ss, sg, st_);
   L.router_w = p;
   void *router_dst = p;
   p += rw;
@@ -533,7 +542,7 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
   // expert blocks: repack on the device, staging host sources in batches
   auto load_group = [&](const ExpertGroup &G, const void *src, int count) -> moe_status {
     const int f = G.f;
-    const uint64_t mat_bytes = static_cast<uint64_t>(f) * D / 32 * BB;
+    const uint64_t mat_bytes = mat_bytes_of(f);
     const uint64_t exp_bytes = 3 * mat_bytes;
     const bool dev_src = is_device_ptr(src);
     int batch = count;
@@ -563,7 +572,8 @@ moe_status moe_load_layer(moe_handle *h, int32_t layer, const moe_layer_weights 
         const int64_t slots = static_cast<int64_t>(f) * D / kChunk;  // per matrix
         const int64_t first = (static_cast<int64_t>(e0) * 3 + m) * slots;
         cudaError_t ke = launch_repack(s8 + m * mat_bytes, static_cast<int64_t>(exp_bytes), g.fmt, rows, cols, nb,
-                                       3 * slots, G.a + first * 16, G.s + first, cb ? G.g + first : nullptr, st);
+                                       3 * slots, G.a + first * abytes, G.s + first, has_g ? G.g + first : nullptr,
+                                       nv ? G.ts + static_cast<int64_t>(e0) * 3 + m : nullptr, 3, st);
         if (ke != cudaSuccess) {
           rs2 = cuda_fail(h, ke, "repack");
           break;

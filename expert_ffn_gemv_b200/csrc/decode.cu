@@ -30,6 +30,8 @@
 #include <stdlib.h>
 #include <limits.h>
 
+#include <cuda_fp8.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -53,7 +55,7 @@ constexpr int kGemvUnroll = MOE_GEMV_UNROLL;
 #ifndef MOE_Q2_RING
 #define MOE_Q2_RING 4
 #endif
-__host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_CB35_32 ? 3 : MOE_Q2_RING; }
+__host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_Q2_32 ? MOE_Q2_RING : 3; }
 constexpr int kGuStageChunks = 2;               // gate/up: chunks per stage
 constexpr int kDnStageChunks = 4;               // down: chunks per stage (one K segment)
 constexpr int kStageSlots = 2 * kGuStageChunks;   // (matrix, chunk) slots of a stage: 4 either way
@@ -68,6 +70,12 @@ constexpr int kPartStride = kDecodeMaxTokens * kTileRows;  // floats per (segmen
 // and the activation factor times (1/2) / 64.
 constexpr int kQ2SumMul = -192;
 constexpr float kQ2Factor = 0.5f / 64.0f;
+
+// Factor folded into the activation records besides 2^-e: Q2 (1/2 of the block value, 1/64 of
+// the in-place code masks), NVFP4 (the integer operands are 2 x the E2M1 values).
+__host__ __device__ inline float rec_factor(int fmt) {
+  return fmt == MOE_FMT_Q2_32 ? kQ2Factor : fmt == MOE_FMT_NVFP4_16 ? 0.5f : 1.0f;
+}
 
 __device__ __forceinline__ float load_act(const void *x, int64_t i, int bf16) {
   if (bf16) return __bfloat162float(static_cast<const __nv_bfloat16 *>(x)[i]);
@@ -466,7 +474,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
       sm += __shfl_xor_sync(0xffffffffu, sm, 4);
       if ((lane & 7) == 0) rec->m[(lane >> 3) & 1] = a.sh.fmt == MOE_FMT_Q2_32 ? kQ2SumMul * sm : sm;
       if ((lane & 15) == 0) {
-        rec->f = pow2f(-ex) * (a.sh.fmt == MOE_FMT_Q2_32 ? kQ2Factor : 1.0f);
+        rec->f = pow2f(-ex) * rec_factor(a.sh.fmt);
         rec->pad = 0u;
       }
     }
@@ -837,11 +845,11 @@ __host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax, int uma
   p.stage0 = off;
   int so = 0;
   p.a = so;
-  so += align128(nr * cmax * kTileRows * 16);
+  so += align128(nr * cmax * kTileRows * plane_a_bytes(fmt));
   p.s = so;
   so += align128(nr * cmax * kTileRows * 4);
   p.g = so;
-  if (fmt == MOE_FMT_CB35_32) so += align128(nr * cmax * kTileRows * 8);
+  if (has_plane_g(fmt)) so += align128(nr * cmax * kTileRows * 8);
   p.rec = so;
   so += align128(kUnitTok * cmax * static_cast<int>(sizeof(ActRec)));
   p.stage = so;
@@ -926,19 +934,113 @@ __device__ __forceinline__ void gemv_stage(const unsigned char *st, const RingPl
   }
 }
 
+// NVFP4: the four E4M3 block scales of a slot as floats
+__device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float (&f)[4]) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
+}
+
+// NVFP4: the int8 operands (2 x E2M1 value) of weights 4q .. 4q+3: the magnitude selector picks
+// bytes of the table {0, 1, 2, 3, 4, 6, 8, 12}; the sign bits negate (never a zero, see the repack).
+__device__ __forceinline__ uint32_t nv_operand(uint32_t sel, uint32_t sgn, int g) {
+  const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, sel & 0x7777u);
+  const uint32_t m = prmt_sign_bytes(sgn << (7 - g));
+  return (mag ^ m) + (m & 0x01010101u);
+}
+
+// NVFP4 GEMV of NR matrices over the nch chunks of a stage, tokens 0 .. TN-1: per 16-weight block
+// an exact integer dot product (8 dp2a), scaled by the block's E4M3 scale; the activation factor
+// per chunk; the matrices' tensor scales come at the unit's end.
+template <int TN, int NR, int CMAX>
+__device__ __forceinline__ void gemv_stage_nv(const unsigned char *st, const RingPlan &P, int nch,
+                                              float (&acc)[2][kUnitTok]) {
+  constexpr uint32_t kRec = sizeof(ActRec);
+  const int r = threadIdx.x;
+  const uint32_t base = smem_u32(st);
+  const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g, rec = base + P.rec;
+#pragma unroll 1
+  for (int c = 0; c < nch; ++c) {
+    uint32_t A[NR][8];
+    uint2 G[NR];
+    float sc[NR][4];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+      const uint32_t row = (m * CMAX + c) * kTileRows + r;
+      const uint4 a0 = lds_u128(pa + row * 32), a1 = lds_u128(pa + row * 32 + 16);
+      A[m][0] = a0.x; A[m][1] = a0.y; A[m][2] = a0.z; A[m][3] = a0.w;
+      A[m][4] = a1.x; A[m][5] = a1.y; A[m][6] = a1.z; A[m][7] = a1.w;
+      G[m] = lds_u64(pg + row * 8);
+      e4m3x4_to_float(lds_u32(ps + row * 4), sc[m]);
+    }
+    float cacc[NR][TN];
+#pragma unroll
+    for (int m = 0; m < NR; ++m)
+#pragma unroll
+      for (int t = 0; t < TN; ++t) cacc[m][t] = 0.f;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {  // 16-weight blocks: groups q = 4b .. 4b+3, words 2b, 2b+1
+      uint32_t v[NR][4];
+#pragma unroll
+      for (int m = 0; m < NR; ++m)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int q = 4 * b + j;
+          const uint32_t w = A[m][q >> 1];
+          v[m][j] = nv_operand((q & 1) ? (w >> 16) : w, (q < 8) ? G[m].x : G[m].y, q & 7);
+        }
+#pragma unroll
+      for (int t = 0; t < TN; ++t) {
+        const uint32_t ra = rec + (t * CMAX + c) * kRec + 32 * b;  // 16 int16 = weights 16b .. 16b+15
+        const uint4 u0 = lds_u128(ra), u1 = lds_u128(ra + 16);
+        const int pr[8] = {static_cast<int>(u0.x), static_cast<int>(u0.y), static_cast<int>(u0.z), static_cast<int>(u0.w),
+                           static_cast<int>(u1.x), static_cast<int>(u1.y), static_cast<int>(u1.z), static_cast<int>(u1.w)};
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+          int d0 = 0, d1 = 0;
+#pragma unroll
+          for (int j = 0; j < 4; j += 2) {
+            d0 = __dp2a_lo(pr[2 * j], static_cast<int>(v[m][j]), d0);
+            d1 = __dp2a_lo(pr[2 * j + 2], static_cast<int>(v[m][j + 1]), d1);
+            d0 = __dp2a_hi(pr[2 * j + 1], static_cast<int>(v[m][j]), d0);
+            d1 = __dp2a_hi(pr[2 * j + 3], static_cast<int>(v[m][j + 1]), d1);
+          }
+          cacc[m][t] = fmaf(static_cast<float>(d0 + d1), sc[m][b], cacc[m][t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < TN; ++t) {
+      const float f = __uint_as_float(lds_u32(rec + (t * CMAX + c) * kRec + offsetof(ActRec, f)));
+#pragma unroll
+      for (int m = 0; m < NR; ++m) acc[m][t] = fmaf(cacc[m][t], f, acc[m][t]);
+    }
+  }
+}
+
 // 1 .. kUnitTok tokens (a unit serves at most kUnitTok tokens).
 template <int FMT, int NR, int CMAX>
 __device__ __forceinline__ void gemv_dispatch(int nt, const unsigned char *st, const RingPlan &P, int nch,
                                               uint32_t tab, float (&acc)[2][kUnitTok]) {
-  if (kUnitTok <= 2 || nt <= 2) {
-    if (nt == 1)
-      gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc);
-    else
-      gemv_stage<FMT, 0, (kUnitTok < 2 ? kUnitTok : 2), NR, CMAX>(st, P, nch, tab, acc);
-  } else if (nt == 3) {
-    gemv_stage<FMT, 0, (kUnitTok < 3 ? kUnitTok : 3), NR, CMAX>(st, P, nch, tab, acc);
+  if constexpr (FMT == MOE_FMT_NVFP4_16) {
+    static_assert(kUnitTok == 1, "NVFP4 units hold one token");
+    gemv_stage_nv<1, NR, CMAX>(st, P, nch, acc);
   } else {
-    gemv_stage<FMT, 0, (kUnitTok < 4 ? kUnitTok : 4), NR, CMAX>(st, P, nch, tab, acc);
+    if (kUnitTok <= 2 || nt <= 2) {
+      if (nt == 1)
+        gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc);
+      else
+        gemv_stage<FMT, 0, (kUnitTok < 2 ? kUnitTok : 2), NR, CMAX>(st, P, nch, tab, acc);
+    } else if (nt == 3) {
+      gemv_stage<FMT, 0, (kUnitTok < 3 ? kUnitTok : 3), NR, CMAX>(st, P, nch, tab, acc);
+    } else {
+      gemv_stage<FMT, 0, (kUnitTok < 4 ? kUnitTok : 4), NR, CMAX>(st, P, nch, tab, acc);
+    }
   }
 }
 
@@ -999,7 +1101,8 @@ template <int FMT>
 __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H,
                                          int first_task) {
   constexpr int RING = ring_depth(FMT);
-  constexpr int kPlanes = FMT == MOE_FMT_CB35_32 ? 3 : 2;
+  constexpr int kPlanes = has_plane_g(FMT) ? 3 : 2;
+  constexpr int kAB = plane_a_bytes(FMT);
   const int lane = threadIdx.x & 31;
   const int D = a.sh.d, E = a.sh.e, TD = D / kTileRows;
   const int *tb = reinterpret_cast<const int *>(smem + P.table);
@@ -1057,7 +1160,7 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
       if (round > 0) ok = ring_wait(H, &H->empty[slot], (round - 1) & 1u, a.spin_limit);
       if (!ok) break;
       const int nch = min(sch, cend - c0);
-      const uint32_t wbytes = nch * kTileRows * (FMT == MOE_FMT_CB35_32 ? 28 : 20);
+      const uint32_t wbytes = nch * kTileRows * plane_bytes(FMT);
       const uint32_t rbytes = nch * static_cast<uint32_t>(sizeof(ActRec));
       if (lane == 0) {
         StageInfo &in = H->info[slot];
@@ -1083,8 +1186,8 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
         const int64_t mat = static_cast<int64_t>(eidx) * 3 + (gu ? m : 2);
         const int64_t slot0 = (static_cast<int64_t>(mt) * nc + c0) * kTileRows;
         if (pl == 0)
-          bulk_g2s_hint(st + P.a + m * cmax * kTileRows * 16, G.a + mat * G.a_mat + slot0 * 16,
-                        nch * kTileRows * 16, &H->full[slot], pol);
+          bulk_g2s_hint(st + P.a + m * cmax * kTileRows * kAB, G.a + mat * G.a_mat + slot0 * kAB,
+                        nch * kTileRows * kAB, &H->full[slot], pol);
         else if (pl == 1)
           bulk_g2s_hint(st + P.s + m * cmax * kTileRows * 4, G.s + mat * G.s_mat + slot0, nch * kTileRows * 4,
                         &H->full[slot], pol);
@@ -1207,6 +1310,13 @@ __device__ __forceinline__ bool unit_ticket(const DecodeArgs &a, RingHdr *H, Con
   return ok && H->flag[fb];
 }
 
+// expert id of active expert u (E: the shared expert), from the CTA's task table
+__device__ __forceinline__ int unit_expert(const RingHdr *H, int u) {
+  const int *tb = reinterpret_cast<const int *>(reinterpret_cast<const unsigned char *>(H) +
+                                                align128(static_cast<int>(sizeof(RingHdr))));
+  return tb[kTabHead + u * kTabInts];
+}
+
 template <int FMT>
 __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in) {
   const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
@@ -1229,6 +1339,17 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
                         tok0 * kTileRows, nseg,
                     ntok, tot);
     if (r == 0) *ticket = 0u;
+  }
+  if (FMT == MOE_FMT_NVFP4_16) {  // the gate and up matrices' tensor scales
+    const int ex = unit_expert(H, u);
+    const ExpertGroup &Gp = ex == a.sh.e ? a.L.shared : a.L.routed;
+    const int eidx = ex == a.sh.e ? 0 : ex;
+    const float tg = Gp.ts[eidx * 3], tu = Gp.ts[eidx * 3 + 1];
+#pragma unroll
+    for (int t = 0; t < kUnitTok; ++t) {
+      tot[0][t] *= tg;
+      tot[1][t] *= tu;
+    }
   }
   // SwiGLU, then h of each token quantised over the tile's 128 rows
   const int wb = cs.nwmax++ & 1;
@@ -1261,7 +1382,7 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (lane == 0) rec->m[warp & 1] = FMT == MOE_FMT_Q2_32 ? kQ2SumMul * sum : sum;
       if ((r & 63) == 0) {
-        rec->f = pow2f(-e) * (FMT == MOE_FMT_Q2_32 ? kQ2Factor : 1.0f);
+        rec->f = pow2f(-e) * rec_factor(FMT);
         rec->pad = 0u;
       }
     }
@@ -1293,6 +1414,12 @@ __device__ __forceinline__ bool dn_finish(const DecodeArgs &a, RingHdr *H, ConsS
     sum_segments<1>(a.ws.dn_part + static_cast<int64_t>(u * TD + mt) * a.ws.dn_nseg * kPartStride + tok0 * kTileRows,
                     nseg, ntok, tot);
     if (r == 0) *ticket = 0u;
+  }
+  if (a.sh.fmt == MOE_FMT_NVFP4_16) {  // the down matrix's tensor scale
+    const int ex = unit_expert(H, u);
+    const float td = (ex == a.sh.e ? a.L.shared : a.L.routed).ts[(ex == a.sh.e ? 0 : ex) * 3 + 2];
+#pragma unroll
+    for (int t = 0; t < kUnitTok; ++t) tot[0][t] *= td;
   }
   const int row = mt * kTileRows + r;
 #pragma unroll
@@ -1518,7 +1645,8 @@ cudaError_t configure_decode_kernels() {
                       (const void *)k_route<false, true>,
                       (const void *)k_route<false, false>,
                       (const void *)k_gemv<MOE_FMT_Q2_32>,
-                      (const void *)k_gemv<MOE_FMT_CB35_32>};
+                      (const void *)k_gemv<MOE_FMT_CB35_32>,
+                      (const void *)k_gemv<MOE_FMT_NVFP4_16>};
   for (const void *k : ks) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, k);
@@ -1546,7 +1674,9 @@ cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_stream
   const int sm = gemv_smem(fmt, umax);
   e = fmt == MOE_FMT_Q2_32
           ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<MOE_FMT_Q2_32>, kGemvThreads, sm)
-          : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<MOE_FMT_CB35_32>, kGemvThreads, sm);
+      : fmt == MOE_FMT_CB35_32
+          ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<MOE_FMT_CB35_32>, kGemvThreads, sm)
+          : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<MOE_FMT_NVFP4_16>, kGemvThreads, sm);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   *grid_gemv = nsm * occ;
@@ -1574,8 +1704,9 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
   {
     const int sm = gemv_smem(a.sh.fmt, a.ws.umax);
     rec(a, kProfGateUp, 0, st);
-    err = a.sh.fmt == MOE_FMT_Q2_32 ? launch_pdl(k_gemv<MOE_FMT_Q2_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a)
-                                    : launch_pdl(k_gemv<MOE_FMT_CB35_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a);
+    err = a.sh.fmt == MOE_FMT_Q2_32     ? launch_pdl(k_gemv<MOE_FMT_Q2_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a)
+          : a.sh.fmt == MOE_FMT_CB35_32 ? launch_pdl(k_gemv<MOE_FMT_CB35_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a)
+                                        : launch_pdl(k_gemv<MOE_FMT_NVFP4_16>, a.ws.grid_gemv, kGemvThreads, sm, st, a);
     if (err != cudaSuccess) return err;
     rec(a, kProfGateUp, 1, st);
   }

@@ -13,6 +13,10 @@
 // codes of weights 16w+4kk .. 16w+4kk+3 as bytes 0..3, the operand order of dp2a.
 // CB35 sign word of a block: byte j, bit g is the sign of weight 4g + j, so shifting left by
 // 7 - g puts the signs of group g in the byte msbs, where prmt can replicate them.
+// NVFP4: plane A holds 32 B per (row, chunk): the E2M1 magnitude indices (0..7) as 4-bit prmt
+// selectors, selector q (bits 16 (q % 2) of word q / 2) = weights 4q .. 4q+3; plane G the sign
+// bits in the CB35 arrangement (negative zero stored as zero); plane S the four E4M3 block
+// scales; the matrices' fp32 tensor scales sit in a small array of their own.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -37,11 +41,17 @@ constexpr uint32_t kErrTimeout = 1u;
 constexpr uint32_t kErrBadIndex = 2u;
 
 // One group of experts with equal shapes (all routed experts, or the shared expert).
+// device plane bytes per (row, 64-weight chunk)
+__host__ __device__ constexpr int plane_a_bytes(int fmt) { return fmt == MOE_FMT_NVFP4_16 ? 32 : 16; }
+__host__ __device__ constexpr bool has_plane_g(int fmt) { return fmt != MOE_FMT_Q2_32; }
+__host__ __device__ constexpr int plane_bytes(int fmt) { return plane_a_bytes(fmt) + 4 + (has_plane_g(fmt) ? 8 : 0); }
+
 struct ExpertGroup {
   uint8_t *a;          // plane A of expert 0, matrix 0
-  __half2 *s;          // plane S
-  uint2 *g;            // plane G (CB35) or nullptr
-  int64_t a_mat;       // bytes of plane A per matrix   = F * D / 4
+  __half2 *s;          // plane S (NVFP4: four E4M3 bytes per slot)
+  uint2 *g;            // plane G (CB35, NVFP4) or nullptr
+  float *ts;           // NVFP4: tensor scales [expert][gate, up, down], else nullptr
+  int64_t a_mat;       // bytes of plane A per matrix   = F * D / 4 (NVFP4: F * D / 2)
   int64_t s_mat;       // half2 per matrix              = F * D / 64
   int64_t g_mat;       // uint2 per matrix              = F * D / 64
   int f;               // d_ff of this group
@@ -257,8 +267,8 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)
 // launchers (host side, defined in the .cu files)
 // ------------------------------------------------------------------------------------------
 cudaError_t launch_repack(const uint8_t *src, int64_t src_stride, int fmt, int rows, int cols,
-                          int n_mats, int64_t dst_stride, uint8_t *a, __half2 *s, uint2 *g,
-                          cudaStream_t st);
+                          int n_mats, int64_t dst_stride, uint8_t *a, __half2 *s, uint2 *g, float *ts,
+                          int ts_stride, cudaStream_t st);
 
 struct DecodeArgs {
   Shape sh;

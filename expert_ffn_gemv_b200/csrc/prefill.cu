@@ -15,6 +15,8 @@
 // The shared expert is group E (all tokens).  Nothing here uses cluster multicast.
 #include <float.h>
 
+#include <cuda_fp8.h>
+
 #include "prefill.cuh"
 
 namespace moe {
@@ -429,12 +431,13 @@ constexpr int kDeqSub = kDeqWarps / 8;                 // threads sharing one (r
 template <int FMT, int MODE>
 struct PfPlan {
   static constexpr int NM = MODE == 0 ? 2 : 1;
-  static constexpr int kStages = MODE == 0 ? MOE_PF_STAGES0 : MOE_PF_STAGES1;  // (raw + B) stages
+  // (raw + B) stages; NVFP4's larger raw planes leave room for three gate/up stages
+  static constexpr int kStages = MODE == 0 ? (FMT == MOE_FMT_NVFP4_16 ? 3 : MOE_PF_STAGES0) : MOE_PF_STAGES1;
   static constexpr int kABufs = MODE == 0 ? MOE_PF_ABUFS0 : MOE_PF_ABUFS1;     // bf16 A buffers
   static constexpr int kAcc = MODE == 0 ? 1 : 2;               // accumulator buffers
   static constexpr int kATile = 128 * 128;                      // 128 x 64 bf16
   static constexpr int kBTile = kPfBN * 128;                    // kPfBN x 64 bf16
-  static constexpr int kRawA = 128 * 16, kRawS = 128 * 4, kRawG = FMT == MOE_FMT_CB35_32 ? 128 * 8 : 0;
+  static constexpr int kRawA = 128 * plane_a_bytes(FMT), kRawS = 128 * 4, kRawG = has_plane_g(FMT) ? 128 * 8 : 0;
   static constexpr int kRawM = kRawA + kRawS + kRawG;
   static constexpr int kRaw = NM * kRawM;
   static constexpr int kStage = kBTile + ((kRaw + 1023) & ~1023);  // B tile, then the raw blocks
@@ -590,9 +593,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
           for (int m = 0; m < NM; ++m) {
             const int64_t mat = static_cast<int64_t>(c.eidx) * 3 + (MODE == 0 ? m : 2);
             unsigned char *rm = raw + m * PL::kRawM;
-            bulk_g2s(rm, G.a + mat * G.a_mat + slot0 * 16, PL::kRawA, &full[st]);
+            bulk_g2s(rm, G.a + mat * G.a_mat + slot0 * plane_a_bytes(FMT), PL::kRawA, &full[st]);
             bulk_g2s(rm + PL::kRawA, G.s + mat * G.s_mat + slot0, PL::kRawS, &full[st]);
-            if (FMT == MOE_FMT_CB35_32)
+            if (has_plane_g(FMT))
               bulk_g2s(rm + PL::kRawA + PL::kRawS, G.g + mat * G.g_mat + slot0, PL::kRawG, &full[st]);
           }
           tma_load_2d(sb, bmap, s * kChunk, c.pt.rows0, &full[st]);
@@ -621,6 +624,42 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
         for (int m = 0; m < NM; ++m) {
           if (kDeqSub > 1 && NM == 2 && m != sub) continue;  // gate/up: one matrix per share
           const unsigned char *rm = raw + m * PL::kRawM;
+          unsigned char *at = ab + m * PL::kATile;
+          if constexpr (FMT == MOE_FMT_NVFP4_16) {
+            // NVFP4: weights 32h .. 32h+31 of the chunk: two 16-weight blocks; the int8 operands
+            // (2 x E2M1) go to bf16 as (192 + v) by a byte permute, then one bf16 FMA with s / 2
+            // gives v s / 2 exactly (the tensor scale is applied in the epilogue)
+            const uint4 Aw = reinterpret_cast<const uint4 *>(rm)[2 * r + h];
+            const uint32_t aw[4] = {Aw.x, Aw.y, Aw.z, Aw.w};
+            const uint32_t sgn = reinterpret_cast<const uint32_t *>(rm + PL::kRawA + PL::kRawS)[2 * r + h];
+            const uint32_t sw = reinterpret_cast<const uint32_t *>(rm + PL::kRawA)[r];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              if (kDeqSub > 1 && NM == 1 && cc / kItems != sub) continue;
+              const uint32_t sb = (sw >> (8 * (2 * h + (cc >> 1)))) & 0xFFu;
+              const __half_raw shr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(sb), __NV_E4M3);
+              const float sf = __half2float(*reinterpret_cast<const __half *>(&shr));
+              const __nv_bfloat162 s2 = __floats2bfloat162_rn(0.5f * sf, 0.5f * sf);
+              const __nv_bfloat162 c2 = __floats2bfloat162_rn(-96.0f * sf, -96.0f * sf);
+              uint32_t o[4];
+#pragma unroll
+              for (int gg = 0; gg < 2; ++gg) {
+                const int g = 2 * cc + gg;  // group of 4 weights within the half
+                const uint32_t w = aw[g >> 1];
+                const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, ((g & 1) ? (w >> 16) : w) & 0x7777u);
+                const uint32_t mk = prmt_sign_bytes(sgn << (7 - g));
+                const uint32_t v = (mag ^ mk) + (mk & 0x01010101u);
+                const uint32_t u = (v ^ 0x80808080u) - 0x40404040u;  // v + 64 per byte, in 52 .. 76
+                const uint32_t lo = __byte_perm(u, 0x43434343u, 0x5140), hi = __byte_perm(u, 0x43434343u, 0x5342);
+                const __nv_bfloat162 r0 = __hfma2(*reinterpret_cast<const __nv_bfloat162 *>(&lo), s2, c2);
+                const __nv_bfloat162 r1 = __hfma2(*reinterpret_cast<const __nv_bfloat162 *>(&hi), s2, c2);
+                o[2 * gg] = *reinterpret_cast<const uint32_t *>(&r0);
+                o[2 * gg + 1] = *reinterpret_cast<const uint32_t *>(&r1);
+              }
+              *reinterpret_cast<uint4 *>(at + sw128_off(r, 4 * h + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            continue;
+          }
           const uint4 A = reinterpret_cast<const uint4 *>(rm)[r];
           const __half2 sc2 = reinterpret_cast<const __half2 *>(rm + PL::kRawA)[r];
           const float sc = __half2float(h ? __high2half(sc2) : __low2half(sc2));
@@ -630,7 +669,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
             const uint2 G2 = reinterpret_cast<const uint2 *>(rm + PL::kRawA + PL::kRawS)[r];
             sgn = h ? G2.y : G2.x;
           }
-          unsigned char *at = ab + m * PL::kATile;
           // Q2: the block's four bf16 values s (q - 1.5), q = 0..3, as bytes 0..7 of (T0, T1); a
           // prmt selector built from two codes picks the bf16 pair of two consecutive weights
           uint32_t T0 = 0, T1 = 0;
@@ -734,6 +772,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
       tc_fence_after();
       const PfTile &pt = c.pt;
       const int row = pt.mt * kTileRows + 32 * q + lane;
+      float tsa = 1.f, tsb = 1.f;  // NVFP4: the matrices' tensor scales (gate, up; or down)
+      if (FMT == MOE_FMT_NVFP4_16) {
+        const float *ts = (c.shared ? a.L.shared : a.L.routed).ts + c.eidx * 3;
+        tsa = MODE == 0 ? ts[0] : ts[2];
+        tsb = ts[1];
+      }
       const uint32_t acc = tmem + b * (NM * kPfBN) + (static_cast<uint32_t>(32 * q) << 16);
       for (int c0 = 32 * e; c0 < pt.cnt; c0 += 64) {
         uint32_t g[32];
@@ -745,8 +789,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             if (c0 + i < pt.cnt) {
-              const float z = __uint_as_float(g[i]);
-              const float h = __fdividef(z, 1.0f + __expf(-z)) * __uint_as_float(u[i]);
+              const float z = __uint_as_float(g[i]) * tsa;
+              const float h = __fdividef(z, 1.0f + __expf(-z)) * (__uint_as_float(u[i]) * tsb);
               a.ws.hs[static_cast<int64_t>(pt.rows0 + c0 + i) * fmax + row] = __float2bfloat16_rn(h);
             }
           }
@@ -758,7 +802,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
           for (int i = 0; i < 32; ++i) {
             const float wr = __shfl_sync(0xffffffffu, wl, i);
             if (c0 + i < pt.cnt)
-              a.ws.outs[static_cast<int64_t>(pt.rows0 + c0 + i) * D + row] = __float2bfloat16_rn(__uint_as_float(g[i]) * wr);
+              a.ws.outs[static_cast<int64_t>(pt.rows0 + c0 + i) * D + row] =
+                  __float2bfloat16_rn(__uint_as_float(g[i]) * tsa * wr);
           }
         }
       }
@@ -997,6 +1042,12 @@ cudaError_t configure_prefill_kernels() {
     e = cudaFuncSetAttribute(k_pf_gemm<MOE_FMT_CB35_32, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PfPlan<MOE_FMT_CB35_32, 1>::kBytes);
   if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_pf_gemm<MOE_FMT_NVFP4_16, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PfPlan<MOE_FMT_NVFP4_16, 0>::kBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_pf_gemm<MOE_FMT_NVFP4_16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PfPlan<MOE_FMT_NVFP4_16, 1>::kBytes);
+  if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_pf_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * kMaxExperts * 4);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_pf_router_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kRtBytes);
   return e;
@@ -1083,15 +1134,19 @@ cudaError_t launch_prefill_layer(const PrefillArgs &a, cudaStream_t st) {
   pf_rec(a, kProfGateUp, 0, st);
   if (a.sh.fmt == MOE_FMT_Q2_32)
     k_pf_gemm<MOE_FMT_Q2_32, 0><<<grid, kPfThreads, PfPlan<MOE_FMT_Q2_32, 0>::kBytes, st>>>(a);
-  else
+  else if (a.sh.fmt == MOE_FMT_CB35_32)
     k_pf_gemm<MOE_FMT_CB35_32, 0><<<grid, kPfThreads, PfPlan<MOE_FMT_CB35_32, 0>::kBytes, st>>>(a);
+  else
+    k_pf_gemm<MOE_FMT_NVFP4_16, 0><<<grid, kPfThreads, PfPlan<MOE_FMT_NVFP4_16, 0>::kBytes, st>>>(a);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   pf_rec(a, kProfGateUp, 1, st);
   pf_rec(a, kProfDown, 0, st);
   if (a.sh.fmt == MOE_FMT_Q2_32)
     k_pf_gemm<MOE_FMT_Q2_32, 1><<<grid, kPfThreads, PfPlan<MOE_FMT_Q2_32, 1>::kBytes, st>>>(a);
-  else
+  else if (a.sh.fmt == MOE_FMT_CB35_32)
     k_pf_gemm<MOE_FMT_CB35_32, 1><<<grid, kPfThreads, PfPlan<MOE_FMT_CB35_32, 1>::kBytes, st>>>(a);
+  else
+    k_pf_gemm<MOE_FMT_NVFP4_16, 1><<<grid, kPfThreads, PfPlan<MOE_FMT_NVFP4_16, 1>::kBytes, st>>>(a);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   {
     const int threads = max(64, a.sh.d / kPfCombineCols);  // d_model <= 4096: at most 512; >= k + 1

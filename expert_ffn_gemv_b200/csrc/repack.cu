@@ -4,6 +4,48 @@
 
 namespace moe {
 
+// NVFP4: one thread per (matrix, row, chunk of 64 weights = interchange blocks 4c .. 4c+3):
+// magnitude indices into prmt selectors (plane A, 32 B), signs into the CB35 arrangement (plane
+// G; a negative zero is stored as zero), the four E4M3 scale bytes (plane S); the matrix's
+// tensor scale (its first 4 bytes) goes to ts[mi * ts_stride].
+__global__ void k_repack_nvfp4(const uint8_t *__restrict__ src, int64_t src_stride, int rows, int cols, int n_mats,
+                               int64_t dst_stride, uint8_t *__restrict__ a, uint32_t *__restrict__ s,
+                               uint2 *__restrict__ g, float *__restrict__ ts, int ts_stride) {
+  const int nc = cols / kChunk;
+  const int64_t per_mat = static_cast<int64_t>(rows) * nc;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (tid >= per_mat * n_mats) return;
+  const int64_t mat = tid / per_mat;
+  const int64_t rem = tid % per_mat;
+  const int row = static_cast<int>(rem / nc);
+  const int c = static_cast<int>(rem % nc);
+  const uint8_t *m0 = src + mat * src_stride;
+  if (row == 0 && c == 0) {
+    const uint32_t u = m0[0] | (m0[1] << 8) | (m0[2] << 16) | (static_cast<uint32_t>(m0[3]) << 24);
+    ts[mat * ts_stride] = __uint_as_float(u);
+  }
+  const uint8_t *b0 = m0 + 4 + (static_cast<int64_t>(row) * (cols / 16) + 4 * c) * 9;
+  const int64_t slot = mat * dst_stride + (static_cast<int64_t>(row / kTileRows) * nc + c) * kTileRows +
+                       (row % kTileRows);
+  uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sg[2] = {0, 0}, sc = 0;
+  for (int k = 0; k < 4; ++k) sc |= static_cast<uint32_t>(b0[9 * k]) << (8 * k);
+  for (int p = 0; p < 64; ++p) {
+    const uint8_t *blk = b0 + 9 * (p >> 4);
+    const int i = p & 15;
+    const uint32_t code = (blk[1 + (i >> 1)] >> (4 * (i & 1))) & 15u;
+    const uint32_t mag = code & 7u, neg = mag ? code >> 3 : 0u;
+    const int q = p >> 2, j = p & 3;
+    w[q >> 1] |= mag << (16 * (q & 1) + 4 * j);
+    const int i32 = p & 31;
+    sg[p >> 5] |= neg << (8 * (i32 & 3) + (i32 >> 2));
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(a) + 2 * slot;
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  g[slot] = make_uint2(sg[0], sg[1]);
+  s[slot] = sc;
+}
+
 // One thread per (matrix, row, chunk of 64 weights = interchange blocks 2c, 2c+1).
 // Matrix mi of the batch is read at src + mi * src_stride bytes and written at slot offset
 // mi * dst_stride (a slot is 16 B of plane A, one half2 of plane S, one uint2 of plane G).
@@ -65,13 +107,16 @@ __global__ void k_repack(const uint8_t *__restrict__ src, int64_t src_stride, in
 }
 
 cudaError_t launch_repack(const uint8_t *src, int64_t src_stride, int fmt, int rows, int cols,
-                          int n_mats, int64_t dst_stride, uint8_t *a, __half2 *s, uint2 *g,
-                          cudaStream_t st) {
+                          int n_mats, int64_t dst_stride, uint8_t *a, __half2 *s, uint2 *g, float *ts,
+                          int ts_stride, cudaStream_t st) {
   const int64_t total = static_cast<int64_t>(rows) * (cols / kChunk) * n_mats;
   if (total == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (total + threads - 1) / threads;
-  if (fmt == MOE_FMT_Q2_32)
+  if (fmt == MOE_FMT_NVFP4_16)
+    k_repack_nvfp4<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
+        src, src_stride, rows, cols, n_mats, dst_stride, a, reinterpret_cast<uint32_t *>(s), g, ts, ts_stride);
+  else if (fmt == MOE_FMT_Q2_32)
     k_repack<MOE_FMT_Q2_32><<<static_cast<unsigned>(blocks), threads, 0, st>>>(
         src, src_stride, rows, cols, n_mats, dst_stride, a, s, g);
   else

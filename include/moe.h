@@ -21,6 +21,10 @@
  *                   2*(i%4)); w = s * (q - 1.5)
  *   MOE_FMT_CB35_32 14 B: fp16 scale s, 8 index bytes (byte g: grid row of weights 4g..4g+3),
  *                   uint32 LE sign mask (bit i negates weight i); w = s * sign * grid[row][i%4]
+ *   MOE_FMT_NVFP4_16 9 B per 16 weights: FP8 E4M3 block scale s, 16 FP4 E2M1 codes (weight i
+ *                   in byte 1 + i/2, low nibble for even i); each matrix starts with a 4-byte LE
+ *                   fp32 tensor scale g; w = g * s * e2m1(code)  (hao.cnyes.com, the supported
+ *                   models list: an NVIDIA-only NVFP4 file)
  * An expert's bytes are [gate: d_ff x d_model][up: d_ff x d_model][down: d_model x d_ff],
  * each row-major in blocks; routed experts are contiguous in index order.
  *
@@ -59,7 +63,7 @@ typedef enum {
   MOE_ERR_DEVICE_FAULT = 7
 } moe_status;
 
-typedef enum { MOE_FMT_Q2_32 = 0, MOE_FMT_CB35_32 = 1 } moe_format;
+typedef enum { MOE_FMT_Q2_32 = 0, MOE_FMT_CB35_32 = 1, MOE_FMT_NVFP4_16 = 2 } moe_format;
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 /* How the router bias enters: MOE_BIAS_LOGIT adds b to the logits used for the selection and for
  * the weights (the plain definition above); MOE_BIAS_SELECT selects the top_k of (logit + b) and

@@ -28,7 +28,8 @@ shared expert, 2-bit and 3.5-bit block files):
 * codebook indices (uint8) and sign bits: uniform, bytes of hash words;
 * NVFP4: E2M1 codes uniform (bytes of hash words); E4M3 block scales with exponent field
   5..8 and mantissa 0..7 uniform (0.25 .. 3.75); the matrix's fp32 tensor scale
-  2^-8 (1 + u/8), u uniform in 0..7;
+  2^-9 (1 + u/8), u uniform in 0..7 (weight RMS ~0.014, that of the 2-bit blocks, so
+  that a 48-layer residual stack without norms stays bounded);
 * N(0, sigma^2) activations / router weights: 16 hash bits index a table of
   the 65,536 mid-quantiles sigma * Phi^-1((u + 1/2) / 65536), rounded to the
   storage dtype (bf16 round-to-nearest-even, or fp32);
@@ -270,7 +271,7 @@ def gen_x(wl: Workload, seed: int, n_tokens: int, pass_idx: int = 0, start_token
 
 def _nvfp4_matrix_np(key_base: tuple, rows: int, cols: int) -> np.ndarray:
     nb = rows * cols // 16
-    head = np.array([2.0 ** -8 * (1 + int(words_np(stream_key(*key_base, F_TSCALE), 0, 1)[0] & 7) / 8)],
+    head = np.array([2.0 ** -9 * (1 + int(words_np(stream_key(*key_base, F_TSCALE), 0, 1)[0] & 7) / 8)],
                     dtype=np.float32).view(np.uint8)
     out = np.empty((nb, 9), dtype=np.uint8)
     sw = words_np(stream_key(*key_base, F_SCALE), 0, nb)
@@ -427,7 +428,7 @@ def _nvfp4_matrices_torch(keys, nb: int, out):
     import torch
 
     dev = out.device
-    heads = np.array([2.0 ** -8 * (1 + int(words_np(stream_key(*k, F_TSCALE), 0, 1)[0] & 7) / 8) for k in keys],
+    heads = np.array([2.0 ** -9 * (1 + int(words_np(stream_key(*k, F_TSCALE), 0, 1)[0] & 7) / 8) for k in keys],
                      dtype=np.float32).view(np.uint8).reshape(len(keys), 4)
     out[:, 0:4] = torch.from_numpy(heads).to(dev)
 

@@ -9,6 +9,9 @@ from helpers import (TOL_DECODE, compare_routing, load_layer_device, load_layer_
 
 pytestmark = pytest.mark.gpu
 
+FORMATS = [synth.FMT_Q2, synth.FMT_CB35, synth.FMT_NVFP4]
+MODEL_SCALE = {synth.FMT_Q2: synth.VERIFY, synth.FMT_CB35: synth.CODEBOOK, synth.FMT_NVFP4: synth.NVFP4}
+
 
 @pytest.fixture(scope="module")
 def torch_cuda():
@@ -68,7 +71,7 @@ def test_tiny_layer_host_buffers(torch_cuda):
     moe.close()
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", FORMATS)
 @pytest.mark.parametrize("n", [1, 2, 3, 5, 8])
 def test_small_layer_tokens(torch_cuda, fmt, n):
     torch = torch_cuda
@@ -80,9 +83,10 @@ def test_small_layer_tokens(torch_cuda, fmt, n):
     moe.close()
 
 
-def test_host_and_device_loads_agree(torch_cuda):
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_host_and_device_loads_agree(torch_cuda, fmt):
     torch = torch_cuda
-    wl = synth.small_workload(d_model=256, d_ff=128, n_experts=16, top_k=3)
+    wl = synth.small_workload(fmt=fmt, d_model=256, d_ff=128, n_experts=16, top_k=3)
     a, b = moe_for(wl, 1, 8), moe_for(wl, 1, 8)
     load_layer_host(a, 0, wl, 2, 0)
     load_layer_device(b, 0, wl, 2, 0)
@@ -139,11 +143,11 @@ def test_decode_layer_model_scale(torch_cuda, seeds):
     moe.close()
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", FORMATS)
 def test_verify_batch_model_scale(torch_cuda, fmt):
     """8 tokens (1 + 7 verify batch) through one model-scale layer of each format."""
     torch = torch_cuda
-    wl = synth.VERIFY if fmt == synth.FMT_Q2 else synth.CODEBOOK
+    wl = MODEL_SCALE[fmt]
     moe = moe_for(wl, 1, 8)
     load_layer_device(moe, 0, wl, 0, 0)
     for n in (1, 8):
@@ -153,7 +157,7 @@ def test_verify_batch_model_scale(torch_cuda, fmt):
     moe.close()
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", FORMATS)
 def test_stack_teacher_forced_and_end_to_end(torch_cuda, fmt):
     """A 3-layer stack of small layers, 8 tokens: per-layer inputs captured on the GPU feed the
     oracle layer by layer (indices, counts, rel-L2 per layer), and the fp64 oracle stack from
@@ -216,7 +220,7 @@ def test_stack_one_layer_equals_forward_plus_x(torch_cuda):
     moe.close()
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", FORMATS)
 def test_stack_equals_chained_layers_bitwise(torch_cuda, fmt):
     """Inside a stack each layer's combine also writes the next layer's activation records; a
     chain of single-layer calls (residual added in fp32 by the caller) quantises its input in

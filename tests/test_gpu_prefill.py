@@ -47,7 +47,7 @@ def _check(torch, wl, seed, x, y, rb, L, sample=None, tol=TOL_PREFILL):
     return err
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35, synth.FMT_NVFP4])
 @pytest.mark.parametrize("n", [9, 37, 300])
 def test_small_prefill(torch_cuda, fmt, n):
     """Ragged token counts: tiles of 128 rows, partial tiles, empty experts, the shared expert."""
@@ -99,7 +99,8 @@ def _sample_tokens(idx_ref, keep, n_experts, rng, n_random):
     return rows[keep[rows]], int(counts[big]), int(small.size)
 
 
-@pytest.mark.parametrize("fmt,n", [(synth.FMT_Q2, 1180), (synth.FMT_Q2, 8192), (synth.FMT_CB35, 1180)])
+@pytest.mark.parametrize("fmt,n", [(synth.FMT_Q2, 1180), (synth.FMT_Q2, 8192), (synth.FMT_CB35, 1180),
+                                   (synth.FMT_NVFP4, 1180)])
 def test_prefill_chunk_model_scale(torch_cuda, fmt, n):
     """A prompt chunk (1,180 or 8,192 tokens) through one model-scale layer (d_model 2048, d_ff
     768, 512 experts top-10 + shared, Zipf router bias): expert sets of every token and the
@@ -107,7 +108,7 @@ def test_prefill_chunk_model_scale(torch_cuda, fmt, n):
     against its own index rows, and the outputs of sampled tokens (the largest expert group,
     experts with 1-15 tokens, a random draw) against the oracle token by token."""
     torch = torch_cuda
-    wl = synth.PREFILL if fmt == synth.FMT_Q2 else synth.CODEBOOK
+    wl = {synth.FMT_Q2: synth.PREFILL, synth.FMT_CB35: synth.CODEBOOK, synth.FMT_NVFP4: synth.NVFP4}[fmt]
     moe = moe_for(wl, 1, 8192)
     load_layer_device(moe, 0, wl, 0, 0)
     x, y, rb = _forward(torch, moe, wl, 0, n, pass_idx=5)
@@ -128,7 +129,7 @@ def test_prefill_chunk_model_scale(torch_cuda, fmt, n):
     moe.close()
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35, synth.FMT_NVFP4])
 def test_prefill_stack_teacher_forced(torch_cuda, fmt):
     torch = torch_cuda
     wl = synth.small_workload(fmt=fmt, d_model=256, d_ff=256, n_experts=16, top_k=4, n_shared=1, shared_d_ff=256)

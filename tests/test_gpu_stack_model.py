@@ -1,7 +1,8 @@
 """Model-scale stacks on the GPU against the fp64 oracle.
 
 * The 48-layer verify stack (2-bit blocks, d_model 2048, d_ff 768, 512 experts top-10 + shared,
-  Zipf router bias, 8 tokens = 1 + 7 verify batch, ~36 GB resident): every layer teacher-forced
+  Zipf router bias, 8 tokens = 1 + 7 verify batch, ~36 GB resident), and the same stack in NVFP4
+  blocks (~65 GB resident): every layer teacher-forced
   (the GPU's own input of the layer, captured through x_trace, fed to the oracle layer: expert
   sets, counts, max relative L2 <= 1e-3), and end to end from the same x over the first layers.
 * The codebook (3.5-bit) configuration: independent model-scale layers applied to the same x, at
@@ -52,9 +53,9 @@ def _oracle_layer_for(wl, seed, l, x):
     return L
 
 
-def test_verify_stack_48_layers_model_scale(torch_cuda):
+@pytest.mark.parametrize("wl", [synth.VERIFY, synth.NVFP4], ids=lambda w: w.name)
+def test_verify_stack_48_layers_model_scale(torch_cuda, wl):
     torch = torch_cuda
-    wl = synth.VERIFY
     nl, n, seed = wl.n_layers, wl.n_tokens, 0
     moe = moe_for(wl, nl, 8)
     _load_stack(moe, wl, seed, range(nl))
@@ -90,7 +91,7 @@ def test_verify_stack_48_layers_model_scale(torch_cuda):
     for r in recs:
         e2e_excl |= r["margin"] < TIE_EPS
     err_e2e = rel_l2(tr[n_e2e], ref_x, ~e2e_excl)
-    print(f"verify stack 48 layers x 8 tokens: teacher-forced max rel L2 {worst:.3e}, excluded near "
+    print(f"{wl.name} 48 layers x 8 tokens: teacher-forced max rel L2 {worst:.3e}, excluded near "
           f"ties {excluded} (token-layers); end to end over {n_e2e} layers {err_e2e:.3e}")
     assert err_e2e <= TOL_DECODE
     moe.close()

@@ -66,13 +66,13 @@ def test_variant_small_layer(variant, n):
     _run_and_check(torch, wl, 21, n, TOL_DECODE if n <= 8 else TOL_PREFILL)
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35])
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_CB35, synth.FMT_NVFP4])
 def test_variants_model_scale(fmt):
     """Both variants on one model-scale layer (d_model 2048, d_ff 768, 512 experts top-10 +
     shared, Zipf bias): an 8-token verify batch and a 1,180-token chunk (96 sampled tokens)."""
     import torch
 
-    base = synth.VERIFY if fmt == synth.FMT_Q2 else synth.CODEBOOK
+    base = {synth.FMT_Q2: synth.VERIFY, synth.FMT_CB35: synth.CODEBOOK, synth.FMT_NVFP4: synth.NVFP4}[fmt]
     wl = dataclasses.replace(base, bias_select=True, shared_gate=True)
     err8, ex8 = _run_and_check(torch, wl, 0, 8, TOL_DECODE, pass_idx=8, L=oracle_layer(wl, 0, 0, full=False))
     sample = np.random.default_rng(4).choice(1180, 96, replace=False)

@@ -90,9 +90,9 @@ def test_nvfp4_expert_bytes_identical_and_sized():
     synth.gen_experts_torch(wl, 3, 1, [1, 2], out)
     for i, e in enumerate((1, 2)):
         assert np.array_equal(out[i].numpy(), synth.gen_expert(wl, 3, 1, e))
-    # E4M3 scales within the recipe (exponent field 5..8, sign 0), tensor scales 2^-8 (1 + u/8)
+    # E4M3 scales within the recipe (exponent field 5..8, sign 0), tensor scales 2^-9 (1 + u/8)
     m = synth.gen_expert(wl, 3, 1, 1)[:wl.matrix_bytes()]
     g = float(m[:4].view(np.float32)[0])
-    assert g * 256 * 8 in range(8, 16)
+    assert g * 512 * 8 in range(8, 16)
     s = m[4:].reshape(-1, 9)[:, 0]
     assert np.all((s >> 3) >= 5) and np.all((s >> 3) <= 8) and np.all(s < 0x80)
