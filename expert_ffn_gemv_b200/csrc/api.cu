@@ -122,12 +122,6 @@ void plan_workspace(moe_handle *h, Carve &c) {
   const int ncd = D / kChunk;
   w.gu_seg = ncd % 4 == 0 ? 4 : 2;
   w.gu_nseg = ncd / w.gu_seg;
-  {
-    auto nseg = [](int f) { const int nc = f / kChunk; return nc / (nc % 4 == 0 ? 4 : 2); };
-    w.dn_nseg = nseg(g.d_ff);
-    if (g.n_shared && nseg(g.shared_d_ff) > w.dn_nseg) w.dn_nseg = nseg(g.shared_d_ff);
-  }
-  const int td = D / kTileRows;
   w.logits = c.take<float>(static_cast<uint64_t>(kDecodeMaxTokens) * E);
   w.raw_logits = c.take<float>(static_cast<uint64_t>(kDecodeMaxTokens) * E);
   w.gate_logit = c.take<float>(kDecodeMaxTokens);
@@ -138,14 +132,11 @@ void plan_workspace(moe_handle *h, Carve &c) {
   w.slotpos = c.take<int>(kDecodeMaxTokens * K);
   w.xrec = c.take<ActRec>(static_cast<uint64_t>(kDecodeMaxTokens) * ncd);
   const uint64_t hrows = static_cast<uint64_t>(umax) * kDecodeMaxTokens;
-  w.hrec = c.take<ActRec>(hrows * (fmax / kChunk));
   w.gu_part = c.take<float>(static_cast<uint64_t>(umax) * tmax * w.gu_nseg * 2 * kDecodeMaxTokens * kTileRows);
-  w.dn_part = c.take<float>(static_cast<uint64_t>(umax) * td * w.dn_nseg * kDecodeMaxTokens * kTileRows);
-  w.o = c.take<float>(hrows * D);
+  w.o = c.take<float>(hrows * tmax * D);
   w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * kDecodeMaxTokens);  // x token groups of a unit (at most one per token)
-  w.dn_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * td * kDecodeMaxTokens);
+  w.gu_depart = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * kDecodeMaxTokens);
   w.counters = c.take<unsigned>(2);
-  w.h_done = c.take<unsigned>(static_cast<uint64_t>(umax) * kDecodeMaxTokens);
   const uint64_t nt = static_cast<uint64_t>(g.max_tokens) * D;
   h->res[0] = c.take<float>(nt);
   h->res[1] = c.take<float>(nt);
@@ -161,12 +152,10 @@ moe_status check_device_error(moe_handle *h, cudaStream_t st) {
   __atomic_store_n(h->err_host, 0u, __ATOMIC_RELEASE);
   // a kernel that gave up may have left arrival counters set: clear them
   const DecodeWs &w = h->dws;
-  const int td = h->cfg.d_model / kTileRows;
   cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax * kDecodeMaxTokens, st);
-  cudaMemsetAsync(w.dn_ticket, 0, sizeof(unsigned) * w.umax * td * kDecodeMaxTokens, st);
+  cudaMemsetAsync(w.gu_depart, 0, sizeof(unsigned) * w.umax * w.tmax * kDecodeMaxTokens, st);
   cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * 2, st);
   cudaMemsetAsync(w.route_sync, 0, sizeof(unsigned) * 2, st);
-  cudaMemsetAsync(w.h_done, 0, sizeof(unsigned) * w.umax * kDecodeMaxTokens, st);
   if (e & kErrTimeout) return fail(h, MOE_ERR_TIMEOUT, "a device-side bounded wait ran out");
   return fail(h, MOE_ERR_DEVICE_FAULT, "a device-side check found an invalid routing index");
 }

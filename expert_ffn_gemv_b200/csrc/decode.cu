@@ -5,25 +5,28 @@
 //   k_route    router GEMV: CTA = 4 experts, warp = (expert, half of d_model), fp32 sums over
 //              the whole d_model (no cross-CTA reduction), logits + bias to global memory.  The
 //              CTAs also quantise the layer input into activation records (int16 + block sums +
-//              a power-of-two factor per 128 columns).
-//   k_gemv     persistent, one CTA per resident slot.  Every CTA first takes the top-k of each
-//              token from the logits (warp per token, argmax by warp reductions over
-//              order-preserving keys), the fp32 softmax over the selected logits, and builds the
-//              active-expert task table in its own shared memory (all CTAs build the same
-//              table; CTA 0 also writes the routing outputs).  Then a producer warp takes
-//              pieces (active expert, 128-row tile, token group, run of K segments) from one
-//              work queue -- gate/up pieces first, then down pieces -- and bulk-copies
-//              (cp.async.bulk) the rows of the piece straight from their low-bit planes, with
-//              the activation records of the unit's tokens, into a ring of shared-memory
-//              stages; four consumer warps (thread = row) unpack the codes with one ALU op per
-//              four weights and multiply them with the int16 activations by dp2a (int16 x int8
-//              -> int32).  The exact integer block sums are scaled by the fp16 block scale into
-//              fp32 sums, one per K segment; segment sums are added in segment order.  A gate/up
-//              unit's last piece applies SwiGLU and quantises h per (token, 128-row tile) into
-//              records and counts the tile on its (expert, token group); a down piece issues
-//              its weight copies at once and its h copies once that count is complete.
-//   k_combine  y = sum_j w_j o_j + o_shared (+ x), slots in descending-logit order.
-// No fp32 atomics, and the K segments are fixed by the matrix shapes: results are
+//              a power-of-two factor per 128 columns); the last CTAs to finish take the top-k
+//              of each token (warp per token over order-preserving keys) and the fp32 softmax
+//              over the selected logits.
+//   k_gemv     persistent, one CTA per resident slot.  Every CTA first builds the active-expert
+//              task table in its own shared memory from the selections (all CTAs build the same
+//              table; CTA 0 also writes the routing outputs).  Then a producer warp takes pieces
+//              from one work queue -- a piece is (active expert, 128-row gate/up tile j, token
+//              group, run of K segments) -- and bulk-copies (cp.async.bulk) the rows of the
+//              piece straight from their low-bit planes, with the activation records of the
+//              unit's tokens, into a ring of shared-memory stages, followed by the rows of the
+//              down matrix over K-slice j (the 128 values of h that tile j makes) for the
+//              piece's share of the output tiles.  Four consumer warps (thread = row) unpack the
+//              codes with one ALU op per four weights and multiply them with the int16
+//              activations by dp2a (int16 x int8 -> int32); the exact integer block sums are
+//              scaled by the block scale into fp32 sums, one per K segment, added in segment
+//              order.  At the end of the gate/up tile the consumers apply SwiGLU and quantise h
+//              into records in shared memory (the pieces of a split unit first meet, and each
+//              sums all of their segment partials), then run the down stages against them: no h
+//              leaves the CTA and no down stage waits for another CTA's gate/up work.
+//   k_combine  y = sum_j w_j o_j + o_shared (+ x), slots in descending-logit order; o_j is the
+//              sum of expert j's K-slice outputs in slice order.
+// No fp32 atomics, and the K segments and slices are fixed by the matrix shapes: results are
 // bit-reproducible and independent of which tokens share a call and of how the work queue
 // split the units among CTAs.
 #include <float.h>
@@ -51,11 +54,17 @@ constexpr int kRing = 4;                        // most stages of the bulk-copy 
 #define MOE_GEMV_UNROLL 1                       // chunks of a stage in flight per iteration
 #endif
 constexpr int kGemvUnroll = MOE_GEMV_UNROLL;
-// ring depth: 4 stages for Q2; 3 for CB35, whose stages and grid table are larger
+// ring depth: 4 stages for Q2; 3 for CB35, whose stages and grid table are larger; 2 for
+// NVFP4 (44-byte slots), so that four CTAs still fit on an SM
 #ifndef MOE_Q2_RING
 #define MOE_Q2_RING 4
 #endif
-__host__ __device__ constexpr int ring_depth(int fmt) { return fmt == MOE_FMT_Q2_32 ? MOE_Q2_RING : 3; }
+#ifndef MOE_NV_RING
+#define MOE_NV_RING 2
+#endif
+__host__ __device__ constexpr int ring_depth(int fmt) {
+  return fmt == MOE_FMT_Q2_32 ? MOE_Q2_RING : fmt == MOE_FMT_NVFP4_16 ? MOE_NV_RING : 3;
+}
 constexpr int kGuStageChunks = 2;               // gate/up: chunks per stage
 constexpr int kDnStageChunks = 4;               // down: chunks per stage (one K segment)
 constexpr int kStageSlots = 2 * kGuStageChunks;   // (matrix, chunk) slots of a stage: 4 either way
@@ -437,12 +446,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
     if (e < ER && lane + 32 * i < G) load_row8<RBF16>(a.L.router_w, static_cast<int64_t>(e) * D + c0 + 8 * (lane + 32 * i), w[i]);
   griddep_wait();
   griddep_launch();
-  // the work queue and the h counters of this layer's GEMV kernel start empty (the previous
-  // layer is done)
-  if (blockIdx.x == 0) {
-    if (tid < 2) a.ws.counters[tid] = 0u;
-    for (int i = tid; i < a.ws.umax * kMaxTokGroups; i += kRouteThreads) a.ws.h_done[i] = 0u;
-  }
+  // the work queue of this layer's GEMV kernel starts empty (the previous layer is done)
+  if (blockIdx.x == 0 && tid < 2) a.ws.counters[tid] = 0u;
 
   // ---- activation records: warp per (token, 128-column group), lane = 4 columns
   {
@@ -587,11 +592,11 @@ __host__ __device__ constexpr int table_scratch_bytes() {
   return kMaxExperts * 4 + 2 * (kMaxExperts / 32) * 4 + kDecodeMaxTokens * kMaxTopK * 4 + 2 * kMaxActive * 4 + 16;
 }
 
-// Top-k + softmax per token, the active-expert rows (u = 0: the shared expert; routed experts
-// follow in ascending id), K splits and first tasks of each active expert.  Every thread of the
-// CTA calls it; wr: also write the routing outputs (one CTA does).
+// The active-expert rows from the router's selections (u = 0: the shared expert; routed
+// experts follow in ascending id), the K split and the first task of each active expert.  Every
+// thread of the CTA calls it; wr: also write the routing outputs (one CTA does).
 __device__ void build_tables(const DecodeArgs &a, unsigned char *scratch, int *tb, bool wr) {
-  constexpr int kThreads = kGemvThreads, kWarps = kGemvThreads / 32;
+  constexpr int kThreads = kGemvThreads;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int D = a.sh.d, E = a.sh.e, K = a.sh.k, n = a.n;
   uint32_t *tokmask = reinterpret_cast<uint32_t *>(scratch);
@@ -639,9 +644,8 @@ __device__ void build_tables(const DecodeArgs &a, unsigned char *scratch, int *t
   // rows written by the thread of each expert's first token, and the combine's slots
   const int ns = a.sh.n_shared;
   const int na = ns + s_misc[2];
-  const int TD = D / kTileRows;
   auto rank_of = [&](int e) { return wpre[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u)); };
-  int ug = 0, ud = 0;
+  int ug = 0;
   for (int p = tid; p < n * K + ns; p += kThreads) {
     const bool shared = p == n * K;
     const int t = shared ? 0 : p / K, ex = shared ? E : s_idx[p];
@@ -662,54 +666,39 @@ __device__ void build_tables(const DecodeArgs &a, unsigned char *scratch, int *t
     }
     s_cnt[kMaxActive + u] = ng;
     ug += (F / kTileRows) * ng;
-    ud += TD * ng;
   }
   if (ug) atomicAdd(&s_misc[0], ug);
-  if (ud) atomicAdd(&s_misc[1], ud);
   if (wr && a.out_counts)
     for (int i = tid; i < E; i += kThreads) a.out_counts[i] = __popc(tokmask[i]);
   __syncthreads();
-  if (warp == 0) {  // K splits, task counts and first task of each active expert (prefix over u)
-    // a split depends on the unit totals and the matrix's K only: one gate/up split, one down
-    // split per d_ff (routed, shared)
-    int pg, pdr, pds = 0;
+  if (warp == 0) {  // K split, task counts and first task of each active expert (prefix over u)
+    // the split depends on the unit total and d_model only: one split for every unit
+    int pg;
     const int sg = unit_split(D / kChunk, s_misc[0], a.ws.min_streams, pg);
-    const int sdr = unit_split(a.L.routed.f / kChunk, s_misc[1], a.ws.min_streams, pdr);
-    const int sds = ns ? unit_split(a.L.shared.f / kChunk, s_misc[1], a.ws.min_streams, pds) : 0;
     const int tgr = (a.L.routed.f / kTileRows) * pg, tgs = ns ? (a.L.shared.f / kTileRows) * pg : 0;
-    int run0 = 0, run1 = 0;
+    int run0 = 0;
     for (int u0 = 0; u0 < na; u0 += 32) {
       const int u = u0 + lane;
-      int c0v = 0, c1v = 0;
+      int c0v = 0;
       if (u < na) {
         const bool sh = ns && u == 0;
         const int ng = s_cnt[kMaxActive + u];
-        int *row = tb + kTabHead + u * kTabInts;
-        row[11] = sg;
-        row[13] = sh ? sds : sdr;
+        tb[kTabHead + u * kTabInts + 11] = sg;
         c0v = (sh ? tgs : tgr) * ng;
-        c1v = ng * (sh ? pds : pdr);
       }
-      int i0 = c0v, i1 = c1v;
+      int i0 = c0v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int v0 = __shfl_up_sync(0xffffffffu, i0, o), v1 = __shfl_up_sync(0xffffffffu, i1, o);
-        if (lane >= o) {
-          i0 += v0;
-          i1 += v1;
-        }
+        const int v0 = __shfl_up_sync(0xffffffffu, i0, o);
+        if (lane >= o) i0 += v0;
       }
-      if (u < na) {
-        tb[kTabHead + u * kTabInts + 10] = run0 + i0 - c0v;
-        tb[kTabHead + u * kTabInts + 12] = run1 + i1 - c1v;
-      }
+      if (u < na) tb[kTabHead + u * kTabInts + 10] = run0 + i0 - c0v;
       run0 += __shfl_sync(0xffffffffu, i0, 31);
-      run1 += __shfl_sync(0xffffffffu, i1, 31);
     }
     if (lane == 0) {
       tb[0] = na;
       tb[1] = run0;
-      tb[2] = run1;
+      tb[2] = 0;
       tb[3] = 0;
     }
   }
@@ -803,11 +792,11 @@ __device__ __forceinline__ int q2_block_dot64(uint32_t w0, uint32_t w1, const in
 __host__ __device__ inline int align128(int v) { return (v + 127) & ~127; }
 
 // Shared memory of the GEMV kernels:
-//   [RingHdr][task table][stage 0] .. [stage kRing-1][grid table (CB35)]
+//   [RingHdr][task table][h records][stage 0] .. [stage kRing-1][grid table (CB35)]
 // A stage holds, for up to CMAX chunks: plane A [NR][CMAX][128][16 B], plane S [NR][CMAX][128]
 // [4 B], plane G [NR][CMAX][128][8 B] (CB35), then the records [8 tokens][CMAX][144 B].
 struct RingPlan {
-  int table, stage0, a, s, g, rec, stage, tab, total;
+  int table, hrec, stage0, a, s, g, rec, stage, tab, total;
 };
 
 // Per-stage description written by the producer before it arms the stage's barrier.
@@ -823,6 +812,7 @@ struct StageInfo {
   int c0;      // first chunk of the stage
 };
 constexpr int kPieceStart = 1, kSegStart = 2, kSegEnd = 4, kPieceEnd = 8;
+constexpr int kDnStage = 16, kDnPair = 32;  // a down stage; of two output tiles
 __device__ __forceinline__ int info_pieces(int flags) { return (flags >> 8) & 0xFF; }
 __device__ __forceinline__ int info_nseg(int flags) { return (flags >> 16) & 0xFF; }
 __device__ __forceinline__ int info_tok0(int flags) { return flags >> 24; }
@@ -842,6 +832,8 @@ __host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax, int uma
   RingPlan p;
   p.table = align128(static_cast<int>(sizeof(RingHdr)));
   int off = p.table + align128((kTabHead + kTabInts * umax) * 4);
+  p.hrec = off;  // h records of the current gate/up unit: [token][2 chunks]
+  off += align128(kUnitTok * (kTileRows / kChunk) * static_cast<int>(sizeof(ActRec)));
   p.stage0 = off;
   int so = 0;
   p.a = so;
@@ -913,10 +905,10 @@ __device__ __forceinline__ void chunk_tokens(const uint4 (&A)[NR], const float2 
 // GEMV of NR matrices (1 or 2) over the nch chunks of one stage for tokens T0 .. T0+TN-1.
 template <int FMT, int T0, int TN, int NR, int CMAX>
 __device__ __forceinline__ void gemv_stage(const unsigned char *st, const RingPlan &P, int nch, uint32_t tab,
-                                           float (&acc)[2][kUnitTok]) {
+                                           uint32_t rec, float (&acc)[2][kUnitTok]) {
   const int r = threadIdx.x, lane = r & 31;
   const uint32_t base = smem_u32(st);
-  const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g, rec = base + P.rec;
+  const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g;
 #pragma unroll kGemvUnroll
   for (int c = 0; c < nch; ++c) {
     uint4 A[NR];
@@ -958,12 +950,12 @@ __device__ __forceinline__ uint32_t nv_operand(uint32_t sel, uint32_t sgn, int g
 // an exact integer dot product (8 dp2a), scaled by the block's E4M3 scale; the activation factor
 // per chunk; the matrices' tensor scales come at the unit's end.
 template <int TN, int NR, int CMAX>
-__device__ __forceinline__ void gemv_stage_nv(const unsigned char *st, const RingPlan &P, int nch,
+__device__ __forceinline__ void gemv_stage_nv(const unsigned char *st, const RingPlan &P, int nch, uint32_t rec,
                                               float (&acc)[2][kUnitTok]) {
   constexpr uint32_t kRec = sizeof(ActRec);
   const int r = threadIdx.x;
   const uint32_t base = smem_u32(st);
-  const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g, rec = base + P.rec;
+  const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g;
 #pragma unroll 1
   for (int c = 0; c < nch; ++c) {
     uint32_t A[NR][8];
@@ -1026,20 +1018,20 @@ __device__ __forceinline__ void gemv_stage_nv(const unsigned char *st, const Rin
 // 1 .. kUnitTok tokens (a unit serves at most kUnitTok tokens).
 template <int FMT, int NR, int CMAX>
 __device__ __forceinline__ void gemv_dispatch(int nt, const unsigned char *st, const RingPlan &P, int nch,
-                                              uint32_t tab, float (&acc)[2][kUnitTok]) {
+                                              uint32_t tab, uint32_t rec, float (&acc)[2][kUnitTok]) {
   if constexpr (FMT == MOE_FMT_NVFP4_16) {
     static_assert(kUnitTok == 1, "NVFP4 units hold one token");
-    gemv_stage_nv<1, NR, CMAX>(st, P, nch, acc);
+    gemv_stage_nv<1, NR, CMAX>(st, P, nch, rec, acc);
   } else {
     if (kUnitTok <= 2 || nt <= 2) {
       if (nt == 1)
-        gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, acc);
+        gemv_stage<FMT, 0, 1, NR, CMAX>(st, P, nch, tab, rec, acc);
       else
-        gemv_stage<FMT, 0, (kUnitTok < 2 ? kUnitTok : 2), NR, CMAX>(st, P, nch, tab, acc);
+        gemv_stage<FMT, 0, (kUnitTok < 2 ? kUnitTok : 2), NR, CMAX>(st, P, nch, tab, rec, acc);
     } else if (nt == 3) {
-      gemv_stage<FMT, 0, (kUnitTok < 3 ? kUnitTok : 3), NR, CMAX>(st, P, nch, tab, acc);
+      gemv_stage<FMT, 0, (kUnitTok < 3 ? kUnitTok : 3), NR, CMAX>(st, P, nch, tab, rec, acc);
     } else {
-      gemv_stage<FMT, 0, (kUnitTok < 4 ? kUnitTok : 4), NR, CMAX>(st, P, nch, tab, acc);
+      gemv_stage<FMT, 0, (kUnitTok < 4 ? kUnitTok : 4), NR, CMAX>(st, P, nch, tab, rec, acc);
     }
   }
 }
@@ -1080,37 +1072,52 @@ __device__ __forceinline__ void cons_fail(const DecodeArgs &a, RingHdr *H) {
 
 
 // largest u with first-task(u) <= r (first tasks increase with u, first-task(0) = 0)
-template <bool GU>
 __device__ __forceinline__ int find_expert(const int *tb, int na, int r) {
   int lo = 0, hi = na - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (tb[kTabHead + mid * kTabInts + (GU ? 10 : 12)] <= r) lo = mid;
+    if (tb[kTabHead + mid * kTabInts + 10] <= r) lo = mid;
     else hi = mid - 1;
   }
   return lo;
 }
 
-// The producer warp: one work queue of gate/up pieces (tasks < n_gu) then down pieces ->
-// bulk copies into the ring.  A down piece issues its weight copies at once and its h records
-// once every gate/up tile of its expert and token group has written h (a counter the gate/up
-// epilogue raises); gate/up pieces wait for nothing but their own copies, and all CTAs of the
-// grid are resident, so that wait always ends.  Every stage the warp arms is waited for
-// (bounded) before it leaves, so no copy is in flight when the CTA exits.
+// Plane pl (A, S, G) of matrix slot m of a stage: nch chunk slots of 128 rows from slot0 on.
+template <int FMT>
+__device__ __forceinline__ void copy_plane(unsigned char *st, const RingPlan &P, int m, int pl, const ExpertGroup &G,
+                                           int64_t mat, int64_t slot0, int nch, uint64_t pol, uint64_t *bar) {
+  constexpr int kAB = plane_a_bytes(FMT);
+  constexpr int cmax = kGuStageChunks;
+  if (pl == 0)
+    bulk_g2s_hint(st + P.a + m * cmax * kTileRows * kAB, G.a + mat * G.a_mat + slot0 * kAB, nch * kTileRows * kAB,
+                  bar, pol);
+  else if (pl == 1)
+    bulk_g2s_hint(st + P.s + m * cmax * kTileRows * 4, G.s + mat * G.s_mat + slot0, nch * kTileRows * 4, bar, pol);
+  else
+    bulk_g2s_hint(st + P.g + m * cmax * kTileRows * 8, G.g + mat * G.g_mat + slot0, nch * kTileRows * 8, bar, pol);
+}
+
+// The producer warp: one work queue of pieces (active expert u, gate/up tile j, token group,
+// run of K segments) -> bulk copies into the ring.  A piece is its gate/up stages (the gate and
+// up rows of tile j, two chunks of each per stage, with the activation records of the unit's
+// tokens), then its down stages: the piece's share of the output tiles over K-slice j (the 128
+// rows of h that tile j makes), two tiles of two chunks per stage, weights only -- the consumers
+// write h into shared memory themselves.  No copy waits for another CTA, and every stage the
+// warp arms is waited for (bounded) before it leaves, so no copy is in flight when the CTA
+// exits.
 template <int FMT>
 __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H,
                                          int first_task) {
   constexpr int RING = ring_depth(FMT);
   constexpr int kPlanes = has_plane_g(FMT) ? 3 : 2;
-  constexpr int kAB = plane_a_bytes(FMT);
+  constexpr int kPB = plane_bytes(FMT);
   const int lane = threadIdx.x & 31;
-  const int D = a.sh.d, E = a.sh.e, TD = D / kTileRows;
+  const int D = a.sh.d, E = a.sh.e, TD = D / kTileRows, nc = D / kChunk;
   const int *tb = reinterpret_cast<const int *>(smem + P.table);
   unsigned *ctr = a.ws.counters;
   int task = first_task;
-  const int na = tb[0], n_gu = tb[1], n_dn = tb[2] * TD;
+  const int na = tb[0], n_tasks = tb[1];
   fence_proxy_async_smem();  // the tables' scratch (generic stores) becomes ring stages (bulk copies)
-  const int n_tasks = n_gu + n_dn;
   bool ok = true;
   const uint64_t pol = l2_evict_first_policy();
   int slot = 0;
@@ -1121,105 +1128,80 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
   while (ok && task < n_tasks) {
     int nxt = 0;
     if (lane == 0) nxt = static_cast<int>(atomicAdd(ctr, 1u));  // fetched while this piece is issued
-    const bool gu = task < n_gu;
-    int u, mt, grp, piece;
-    const int *tr = tb + kTabHead;
-    if (gu) {
-      u = find_expert<true>(tb, na, task);
-      const int pieces = (tr[u * kTabInts + 11] >> 8) & 0xFF, ng = tr[u * kTabInts + 14];
-      const int r = task - tr[u * kTabInts + 10];
-      mt = r / (ng * pieces);
-      const int q = r - mt * ng * pieces;
-      grp = q / pieces;
-      piece = q - grp * pieces;
-    } else {  // expert-major, like the gate/up pieces, so that the first down pieces find h early
-      const int t2 = task - n_gu;
-      u = find_expert<false>(tb, na, t2 / TD);
-      const int pieces = (tr[u * kTabInts + 13] >> 8) & 0xFF, ng = tr[u * kTabInts + 14];
-      const int r = t2 - tr[u * kTabInts + 12] * TD;
-      mt = r / (ng * pieces);
-      const int q = r - mt * ng * pieces;
-      grp = q / pieces;
-      piece = q - grp * pieces;
-    }
-    const int *row = tr + u * kTabInts;
+    const int u = find_expert(tb, na, task);
+    const int *row = tb + kTabHead + u * kTabInts;
+    const int pk = row[11], ng = row[14];
+    const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
+    const int r = task - row[10];
+    const int j = r / (ng * pieces);
+    const int q = r - j * ng * pieces;
+    const int grp = q / pieces, piece = q - grp * pieces;
     const int e = row[0];
     const int gsz = tok_group_size(row[1]), tok0 = grp * gsz;
     const int ntok = min(gsz, row[1] - tok0);  // tokens of this unit: slots tok0 .. tok0 + ntok - 1
-    const int pk = row[gu ? 11 : 13];
-    const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
     const bool shared = a.sh.n_shared && e == E;
     const ExpertGroup &G = shared ? a.L.shared : a.L.routed;
-    const int eidx = shared ? 0 : e;
-    const int nr = gu ? 2 : 1, cmax = gu ? kGuStageChunks : kDnStageChunks;
-    const int nc = gu ? D / kChunk : G.f / kChunk;
+    const int64_t mat0 = static_cast<int64_t>(shared ? 0 : e) * 3;
+    const int ncd = G.f / kChunk;
     const int cbeg = piece * len * seg, cend = min(nseg, (piece + 1) * len) * seg;
-    const int sch = gu ? kGuStageChunks : seg;
-    bool h_ready = gu;
-    for (int c0 = cbeg; c0 < cend; c0 += sch) {
+    const int d0 = piece * TD / pieces, d1 = (piece + 1) * TD / pieces;  // this piece's down tiles
+    const int n_gu = (cend - cbeg + kGuStageChunks - 1) / kGuStageChunks, n_st = n_gu + (d1 - d0 + 1) / 2;
+    for (int si = 0; si < n_st; ++si) {
       if (round > 0) ok = ring_wait(H, &H->empty[slot], (round - 1) & 1u, a.spin_limit);
       if (!ok) break;
-      const int nch = min(sch, cend - c0);
-      const uint32_t wbytes = nch * kTileRows * plane_bytes(FMT);
-      const uint32_t rbytes = nch * static_cast<uint32_t>(sizeof(ActRec));
-      if (lane == 0) {
-        StageInfo &in = H->info[slot];
-        in.task = task;
-        in.u = u;
-        in.mt = mt;
-        in.seg = c0 / seg;
-        in.ntok = ntok;
-        in.nch = nch;
-        in.flags = (c0 == cbeg ? kPieceStart : 0) | (c0 % seg == 0 ? kSegStart : 0) |
-                   ((c0 + nch) % seg == 0 ? kSegEnd : 0) | (c0 + nch == cend ? kPieceEnd : 0) | (pieces << 8) |
-                   (nseg << 16) | (tok0 << 24);
-        in.c0 = c0;
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&H->full[slot], nr * wbytes + ntok * rbytes);
-      }
-      __syncwarp();
       unsigned char *st = smem + P.stage0 + slot * P.stage;
-      // copy l of the stage, issued by lane l: nr x (A, S[, G]) weight planes, then one run of
-      // records per token (chunk slot of matrix m, chunk c: m * cmax + c)
-      if (lane < nr * kPlanes) {
-        const int m = lane / kPlanes, pl = lane - m * kPlanes;
-        const int64_t mat = static_cast<int64_t>(eidx) * 3 + (gu ? m : 2);
-        const int64_t slot0 = (static_cast<int64_t>(mt) * nc + c0) * kTileRows;
-        if (pl == 0)
-          bulk_g2s_hint(st + P.a + m * cmax * kTileRows * kAB, G.a + mat * G.a_mat + slot0 * kAB,
-                        nch * kTileRows * kAB, &H->full[slot], pol);
-        else if (pl == 1)
-          bulk_g2s_hint(st + P.s + m * cmax * kTileRows * 4, G.s + mat * G.s_mat + slot0, nch * kTileRows * 4,
-                        &H->full[slot], pol);
-        else
-          bulk_g2s_hint(st + P.g + m * cmax * kTileRows * 8, G.g + mat * G.g_mat + slot0, nch * kTileRows * 8,
-                        &H->full[slot], pol);
-      }
-      if (!h_ready) {  // down: the expert's h (this token group, all tiles) must be complete
-        bool hok = true;
+      if (si < n_gu) {
+        const int c0 = cbeg + si * kGuStageChunks, nch = min(kGuStageChunks, cend - c0);
+        const uint32_t rbytes = nch * static_cast<uint32_t>(sizeof(ActRec));
         if (lane == 0) {
-          const unsigned *cnt = a.ws.h_done + u * kMaxTokGroups + grp;
-          const unsigned target = static_cast<unsigned>(G.f / kTileRows * kConsWarps);  // every warp of every tile
-          const long long t0 = clock64();
-          while (ld_acquire_u32(cnt) < target) {
-            if (H->abort || static_cast<uint64_t>(clock64() - t0) > a.spin_limit) {
-              hok = false;
-              break;
-            }
-            __nanosleep(64);
-          }
+          StageInfo &in = H->info[slot];
+          in.task = task;
+          in.u = u;
+          in.mt = j;
+          in.seg = c0 / seg;
+          in.ntok = ntok;
+          in.nch = nch;
+          in.flags = (c0 == cbeg ? kPieceStart : 0) | (c0 % seg == 0 ? kSegStart : 0) |
+                     ((c0 + nch) % seg == 0 ? kSegEnd : 0) | (c0 + nch == cend ? kPieceEnd : 0) | (pieces << 8) |
+                     (nseg << 16) | (tok0 << 24);
+          in.c0 = c0;
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&H->full[slot], 2 * nch * kTileRows * kPB + ntok * rbytes);
         }
-        ok = __shfl_sync(0xffffffffu, hok, 0);
         __syncwarp();
-        asm volatile("fence.proxy.async.global;" ::: "memory");  // h was written by generic stores
-        h_ready = true;
-      }
-      const int i = lane - nr * kPlanes;
-      if (i >= 0 && i < ntok) {
-        const ActRec *srcr = gu ? a.ws.xrec + static_cast<int64_t>(row[2 + tok0 + i]) * (D / kChunk) + c0
-                                : a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + i) * (a.ws.fmax / kChunk) + c0;
-        // (after a failed h wait the copy still goes out, so that the stage completes and drains)
-        bulk_g2s(st + P.rec + i * cmax * static_cast<int>(sizeof(ActRec)), srcr, rbytes, &H->full[slot]);
+        // copy l of the stage, issued by lane l: 2 x (A, S[, G]) weight planes, then one run of
+        // records per token (chunk slot of matrix m, chunk c: m * 2 + c)
+        if (lane < 2 * kPlanes) {
+          const int m = lane / kPlanes;
+          copy_plane<FMT>(st, P, m, lane - m * kPlanes, G, mat0 + m, (static_cast<int64_t>(j) * nc + c0) * kTileRows,
+                          nch, pol, &H->full[slot]);
+        }
+        const int i = lane - 2 * kPlanes;
+        if (i >= 0 && i < ntok)
+          bulk_g2s(st + P.rec + i * kGuStageChunks * static_cast<int>(sizeof(ActRec)),
+                   a.ws.xrec + static_cast<int64_t>(row[2 + tok0 + i]) * nc + c0, rbytes, &H->full[slot]);
+      } else {
+        // output tiles t0 (and t0 + 1) of the down matrix over K-slice j = chunks 2j, 2j + 1
+        const int t0 = d0 + 2 * (si - n_gu), nt = min(2, d1 - t0);
+        if (lane == 0) {
+          StageInfo &in = H->info[slot];
+          in.task = task;
+          in.u = u;
+          in.mt = t0;
+          in.seg = j;
+          in.ntok = ntok;
+          in.nch = 2;
+          in.flags = kDnStage | (nt == 2 ? kDnPair : 0) | (pieces << 8) | (tok0 << 24);
+          in.c0 = 0;
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&H->full[slot], nt * 2 * kTileRows * kPB);
+        }
+        __syncwarp();
+        if (lane < nt * kPlanes) {
+          const int m = lane / kPlanes;
+          copy_plane<FMT>(st, P, m, lane - m * kPlanes, G, mat0 + 2,
+                          (static_cast<int64_t>(t0 + m) * ncd + 2 * j) * kTileRows, 2, pol, &H->full[slot]);
+        }
       }
 #pragma unroll
       for (int s = 0; s < RING; ++s) last_round[s] = s == slot ? static_cast<int>(round) : last_round[s];
@@ -1227,7 +1209,6 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
         slot = 0;
         ++round;
       }
-      if (!ok) break;
     }
     task = __shfl_sync(0xffffffffu, nxt, 0);
   }
@@ -1252,7 +1233,7 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
   }
 }
 
-// Sums of a split unit's segment partials in segment order (the last piece of the unit), row r:
+// Sums of a split unit's segment partials in segment order, row r:
 // tot[m][t] = sum_j part[j][m][t][r].  32 loads are in flight at a time.
 template <int NR>
 __device__ __forceinline__ void sum_segments(const float *part, int nseg, int ntok, float (&tot)[2][kUnitTok]) {
@@ -1286,7 +1267,7 @@ __device__ __forceinline__ void sum_segments(const float *part, int nseg, int nt
 }
 
 // ------------------------------------------------------------------------------------------
-// consumers: gate/up epilogue (SwiGLU + h quantisation) and down epilogue (o + combine)
+// consumers: gate/up epilogue (SwiGLU + h quantisation into shared memory) and down stages
 // ------------------------------------------------------------------------------------------
 struct ConsState {
   uint32_t cph;   // parity of the consumer barrier
@@ -1294,20 +1275,30 @@ struct ConsState {
   int nwmax;      // uses of H->wmax
 };
 
-// Ticket of a split unit; true on the piece that arrives last (uniform over the consumers).
-__device__ __forceinline__ bool unit_ticket(const DecodeArgs &a, RingHdr *H, ConsState &cs, unsigned *ticket,
-                                            unsigned target, bool &ok) {
-  ok = cons_sync(H, cs.cph, a.spin_limit);  // every consumer's partial stores precede the ticket
-  if (!ok) return false;
+// All pieces of a split unit meet here once their segment partials are stored: arrive, then
+// wait (bounded) until every piece has arrived; every piece then sums the same partials in the
+// same order.  The counters are cleared by the last piece to leave (every piece has seen the
+// full count by then).  Uniform over the consumers; false when a wait ran out.
+__device__ __forceinline__ bool unit_meet(const DecodeArgs &a, RingHdr *H, ConsState &cs, unsigned *arrive,
+                                          unsigned pieces) {
+  if (!cons_sync(H, cs.cph, a.spin_limit)) return false;  // every consumer's partial stores precede the arrival
   const int fb = cs.nflag++ & 1;
   if (threadIdx.x == 0) {
     __threadfence();
-    const bool last = atomicAdd(ticket, 1u) == target;
-    if (last) __threadfence();
-    H->flag[fb] = last;
+    atomicAdd(arrive, 1u);
+    bool ok = true;
+    const long long t0 = clock64();
+    while (ld_acquire_u32(arrive) < pieces) {
+      if (H->abort || static_cast<uint64_t>(clock64() - t0) > a.spin_limit) {
+        ok = false;
+        break;
+      }
+      __nanosleep(32);
+    }
+    __threadfence();
+    H->flag[fb] = ok;
   }
-  ok = cons_sync(H, cs.cph, a.spin_limit);
-  return ok && H->flag[fb];
+  return cons_sync(H, cs.cph, a.spin_limit) && H->flag[fb];
 }
 
 // expert id of active expert u (E: the shared expert), from the CTA's task table
@@ -1317,8 +1308,12 @@ __device__ __forceinline__ int unit_expert(const RingHdr *H, int u) {
   return tb[kTabHead + u * kTabInts];
 }
 
+// End of a gate/up piece: the unit's full sums (this piece's, or every piece's partials), the
+// SwiGLU, and h of each token quantised over the tile's 128 rows into the CTA's shared h
+// records, which the piece's down stages read.
 template <int FMT>
-__device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in) {
+__device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in,
+                                          ActRec *hrec) {
   const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
   const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags);
   const int nseg = info_nseg(in.flags), tok0 = info_tok0(in.flags);
@@ -1330,15 +1325,16 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
       tot[1][t] = H->tot[1][t][r];
     }
   if (pieces > 1) {
-    unsigned *ticket = a.ws.gu_ticket + (u * a.ws.tmax + mt) * kMaxTokGroups + tok0 / kTokGroup;
-    bool ok;
-    const bool last = unit_ticket(a, H, cs, ticket, static_cast<unsigned>(pieces - 1), ok);
-    if (!ok) return false;
-    if (!last) return true;
+    const int64_t ti = (static_cast<int64_t>(u) * a.ws.tmax + mt) * kMaxTokGroups + tok0 / kTokGroup;
+    if (!unit_meet(a, H, cs, a.ws.gu_ticket + ti, static_cast<unsigned>(pieces))) return false;
     sum_segments<2>(a.ws.gu_part + static_cast<int64_t>(u * a.ws.tmax + mt) * a.ws.gu_nseg * 2 * kPartStride +
                         tok0 * kTileRows, nseg,
                     ntok, tot);
-    if (r == 0) *ticket = 0u;
+    if (!cons_sync(H, cs.cph, a.spin_limit)) return false;  // every consumer's partial loads are done
+    if (r == 0 && atomicAdd(a.ws.gu_depart + ti, 1u) == static_cast<unsigned>(pieces - 1)) {
+      a.ws.gu_ticket[ti] = 0u;
+      a.ws.gu_depart[ti] = 0u;
+    }
   }
   if (FMT == MOE_FMT_NVFP4_16) {  // the gate and up matrices' tensor scales
     const int ex = unit_expert(H, u);
@@ -1351,7 +1347,8 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
       tot[1][t] *= tu;
     }
   }
-  // SwiGLU, then h of each token quantised over the tile's 128 rows
+  // SwiGLU, then h of each token quantised over the tile's 128 rows.  The barrier after the
+  // maxima also orders these h stores after every consumer's reads of the previous unit's h.
   const int wb = cs.nwmax++ & 1;
   float hv[kUnitTok];
 #pragma unroll
@@ -1366,7 +1363,6 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
     }
   }
   if (!cons_sync(H, cs.cph, a.spin_limit)) return false;
-  const int fs = a.ws.fmax / kChunk;
 #pragma unroll
   for (int t = 0; t < kUnitTok; ++t) {
     if (t < ntok) {
@@ -1375,7 +1371,7 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
       for (int w = 1; w < kConsWarps; ++w) mx = fmaxf(mx, H->wmax[wb][w][t]);
       const int e = fix16_exponent(mx);
       const int m = fix16(hv[t], pow2f(e));
-      ActRec *rec = a.ws.hrec + (static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + t) * fs + 2 * mt + (r >> 6);
+      ActRec *rec = hrec + t * (kTileRows / kChunk) + (r >> 6);
       rec->x[r & 63] = static_cast<int16_t>(m);
       int sum = m;  // warp = 32 consecutive rows = one block of the down matrix's K
 #pragma unroll
@@ -1387,56 +1383,39 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
       }
     }
   }
-  // this warp's rows of h are written: count them for the down pieces waiting on the group
-  __syncwarp();
-  if (lane == 0) {
-    __threadfence();
-    atomicAdd(a.ws.h_done + u * kMaxTokGroups + tok0 / kTokGroup, 1u);
-  }
-  return true;
+  return cons_sync(H, cs.cph, a.spin_limit);  // h complete before any down stage reads it
 }
 
-__device__ __forceinline__ bool dn_finish(const DecodeArgs &a, RingHdr *H, ConsState &cs, const StageInfo &in) {
-  const int r = threadIdx.x;
-  const int D = a.sh.d, TD = D / kTileRows;
-  const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags), tok0 = info_tok0(in.flags);
-  float tot[2][kUnitTok];
-#pragma unroll
-  for (int t = 0; t < kUnitTok; ++t)
-    if (t < ntok) tot[0][t] = H->tot[0][t][r];
-  if (pieces > 1) {
-    unsigned *ticket = a.ws.dn_ticket + (u * TD + mt) * kMaxTokGroups + tok0 / kTokGroup;
-    bool ok;
-    const bool last = unit_ticket(a, H, cs, ticket, static_cast<unsigned>(pieces - 1), ok);
-    if (!ok) return false;
-    if (!last) return true;
-    const int nseg = info_nseg(in.flags);
-    sum_segments<1>(a.ws.dn_part + static_cast<int64_t>(u * TD + mt) * a.ws.dn_nseg * kPartStride + tok0 * kTileRows,
-                    nseg, ntok, tot);
-    if (r == 0) *ticket = 0u;
+// A down stage's outputs: o of output tiles mt (and mt + 1) over K-slice j, row r, per token.
+template <int FMT>
+__device__ __forceinline__ void dn_store(const DecodeArgs &a, const RingHdr *H, const StageInfo &in,
+                                         const float (&acc)[2][kUnitTok]) {
+  const int r = threadIdx.x, D = a.sh.d;
+  const int nt = (in.flags & kDnPair) ? 2 : 1, tok0 = info_tok0(in.flags);
+  float td = 1.f;
+  if (FMT == MOE_FMT_NVFP4_16) {  // the down matrix's tensor scale
+    const int ex = unit_expert(H, in.u);
+    td = (ex == a.sh.e ? a.L.shared : a.L.routed).ts[(ex == a.sh.e ? 0 : ex) * 3 + 2];
   }
-  if (a.sh.fmt == MOE_FMT_NVFP4_16) {  // the down matrix's tensor scale
-    const int ex = unit_expert(H, u);
-    const float td = (ex == a.sh.e ? a.L.shared : a.L.routed).ts[(ex == a.sh.e ? 0 : ex) * 3 + 2];
+  float *o = a.ws.o + (static_cast<int64_t>(in.u) * kDecodeMaxTokens + tok0) * a.ws.tmax * D +
+             static_cast<int64_t>(in.seg) * D + in.mt * kTileRows + r;
 #pragma unroll
-    for (int t = 0; t < kUnitTok; ++t) tot[0][t] *= td;
-  }
-  const int row = mt * kTileRows + r;
+  for (int m = 0; m < 2; ++m)
 #pragma unroll
-  for (int t = 0; t < kUnitTok; ++t)
-    if (t < ntok) a.ws.o[(static_cast<int64_t>(u) * kDecodeMaxTokens + tok0 + t) * D + row] = tot[0][t];
-  return true;
+    for (int t = 0; t < kUnitTok; ++t)
+      if (m < nt && t < in.ntok) o[static_cast<int64_t>(t) * a.ws.tmax * D + m * kTileRows] = acc[m][t] * td;
 }
 
-// The consumer warps: stages in ring order; gate/up stages (task below n_gu) take two matrices
-// of two chunks, down stages one matrix of up to four chunks (one K segment).
+// The consumer warps: stages in ring order.  A gate/up stage holds two matrices of two chunks
+// and the tokens' records; a down stage two output tiles (or one) of two chunks over the
+// K-slice whose h the preceding gate/up stages made.
 template <int FMT>
 __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *smem, const RingPlan &P, RingHdr *H) {
   constexpr int RING = ring_depth(FMT);
   const int r = threadIdx.x, lane = r & 31;
-  const int D = a.sh.d, TD = D / kTileRows;
   uint32_t *tab = reinterpret_cast<uint32_t *>(smem + P.tab);
-  const int n_gu = reinterpret_cast<const int *>(smem + P.table)[1];
+  ActRec *hrec = reinterpret_cast<ActRec *>(smem + P.hrec);
+  const uint32_t hrec_s = smem_u32(hrec);
   ConsState cs{0u, 0, 0};
   if (FMT == MOE_FMT_CB35_32) {
     load_grid_table(a.grid, tab, kTileRows);
@@ -1455,50 +1434,56 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
     }
     const StageInfo in = H->info[slot];
     if (in.task < 0) return;
-    const bool gu = in.task < n_gu;
-    const int pieces = info_pieces(in.flags), tok0 = info_tok0(in.flags);
-    if ((in.flags & kPieceStart) && pieces == 1) {
-#pragma unroll
-      for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int t = 0; t < kUnitTok; ++t) H->tot[m][t][r] = 0.f;
-    }
-    if (in.flags & kSegStart) {
-#pragma unroll
-      for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int t = 0; t < kUnitTok; ++t) seg[m][t] = 0.f;
-    }
     const unsigned char *st = smem + P.stage0 + slot * P.stage;
-    if (gu)
-      gemv_dispatch<FMT, 2, kGuStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), seg);
-    else
-      gemv_dispatch<FMT, 1, kDnStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), seg);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&H->empty[slot]);
-    if (in.flags & kSegEnd) {
-      const int nr = gu ? 2 : 1;
-      if (pieces > 1) {
-        // segment sum of a split unit -> partial buffer [segment][matrix][token][row]
-        float *part = gu ? a.ws.gu_part + (static_cast<int64_t>(in.u * a.ws.tmax + in.mt) * a.ws.gu_nseg + in.seg) *
-                                              2 * kPartStride
-                         : a.ws.dn_part + (static_cast<int64_t>(in.u * TD + in.mt) * a.ws.dn_nseg + in.seg) * kPartStride;
+    if (in.flags & kDnStage) {
+      float acc[2][kUnitTok];
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int t = 0; t < kUnitTok; ++t) acc[m][t] = 0.f;
+      if (in.flags & kDnPair)
+        gemv_dispatch<FMT, 2, kGuStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), hrec_s, acc);
+      else
+        gemv_dispatch<FMT, 1, kGuStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), hrec_s, acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&H->empty[slot]);
+      dn_store<FMT>(a, H, in, acc);
+    } else {
+      const int pieces = info_pieces(in.flags), tok0 = info_tok0(in.flags);
+      if ((in.flags & kPieceStart) && pieces == 1) {
 #pragma unroll
         for (int m = 0; m < 2; ++m)
 #pragma unroll
-          for (int t = 0; t < kUnitTok; ++t)
-            if (m < nr && t < in.ntok) part[m * kPartStride + (tok0 + t) * kTileRows + r] = seg[m][t];
-      } else {
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-          for (int t = 0; t < kUnitTok; ++t)
-            if (m < nr && t < in.ntok) H->tot[m][t][r] += seg[m][t];
+          for (int t = 0; t < kUnitTok; ++t) H->tot[m][t][r] = 0.f;
       }
-    }
-    if (in.flags & kPieceEnd) {
-      const bool ok = gu ? gu_finish<FMT>(a, H, cs, in) : dn_finish(a, H, cs, in);
-      if (!ok) {
+      if (in.flags & kSegStart) {
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int t = 0; t < kUnitTok; ++t) seg[m][t] = 0.f;
+      }
+      gemv_dispatch<FMT, 2, kGuStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), smem_u32(st) + P.rec, seg);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&H->empty[slot]);
+      if (in.flags & kSegEnd) {
+        if (pieces > 1) {
+          // segment sum of a split unit -> partial buffer [segment][matrix][token][row]
+          float *part = a.ws.gu_part +
+                        (static_cast<int64_t>(in.u * a.ws.tmax + in.mt) * a.ws.gu_nseg + in.seg) * 2 * kPartStride;
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int t = 0; t < kUnitTok; ++t)
+              if (t < in.ntok) part[m * kPartStride + (tok0 + t) * kTileRows + r] = seg[m][t];
+        } else {
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int t = 0; t < kUnitTok; ++t)
+              if (t < in.ntok) H->tot[m][t][r] += seg[m][t];
+        }
+      }
+      if ((in.flags & kPieceEnd) && !gu_finish<FMT>(a, H, cs, in, hrec)) {
         cons_fail(a, H);
         return;
       }
@@ -1555,41 +1540,60 @@ __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(Deco
 
 // ------------------------------------------------------------------------------------------
 // combine: y[t] = sum_j w_tj o[slot(t, j)] + o_shared[t] (+ x[t]), slots in descending-logit
-// order.  CTA = (token, 128 columns); every load of a thread is issued before the sum.
+// order; each expert output o is the sum of its K-slice outputs in slice order.  CTA = (token,
+// 64 columns): first every thread sums the slices of some (slot, column) pairs into shared
+// memory (all slices of a pair loaded at once), then one thread per column adds the slots.
 // ------------------------------------------------------------------------------------------
-constexpr int kCombineThreads = 128;  // d_model is a multiple of 128
+constexpr int kCombineCols = 64;       // d_model is a multiple of 128
+constexpr int kCombineThreads = 256;
+constexpr int kMaxSlices = 8;          // K-slices of a slot loaded together (more: one at a time)
 __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
   __shared__ int s_pos[kMaxTopK];
   __shared__ float s_w[kMaxTopK];
-  const int D = a.sh.d, K = a.sh.k;
-  const int cpt = D / kCombineThreads;  // CTAs per token
-  const int t = blockIdx.x / cpt, d = (blockIdx.x - t * cpt) * kCombineThreads + threadIdx.x;
+  __shared__ float s_o[(kMaxTopK + 1) * kCombineCols];  // [slot (K: the shared expert)][column]
+  const int D = a.sh.d, K = a.sh.k, tid = threadIdx.x;
+  const int cpt = D / kCombineCols;  // CTAs per token
+  const int t = blockIdx.x / cpt, d0 = (blockIdx.x - t * cpt) * kCombineCols;
   griddep_wait();
   griddep_launch();
-  if (threadIdx.x < K) {
-    s_pos[threadIdx.x] = __ldcg(a.ws.slotpos + t * K + threadIdx.x);
-    s_w[threadIdx.x] = __ldcg(a.ws.route_w + t * K + threadIdx.x);
+  if (tid < K) {
+    s_pos[tid] = __ldcg(a.ws.slotpos + t * K + tid);
+    s_w[tid] = __ldcg(a.ws.route_w + t * K + tid);
   }
-  const int64_t i = static_cast<int64_t>(t) * D + d;
-  const float xs = a.residual ? load_act(a.x, i, a.x_bf16) : 0.f;
-  float sh = a.sh.n_shared ? __ldcg(a.ws.o + i) : 0.f;  // u = 0 serves token t in slot t
-  if (a.sh.shared_gate) sh *= 1.0f / (1.0f + __expf(-__ldcg(a.ws.gate_logit + t)));
   __syncthreads();
-  float v[kMaxTopK];
+  const int TM = a.ws.tmax, ns = a.sh.n_shared ? 1 : 0;
+  const int js = ns ? a.L.shared.f / kTileRows : 0, jr = a.L.routed.f / kTileRows;
+  for (int it = tid; it < (K + ns) * kCombineCols; it += kCombineThreads) {
+    const int j = it / kCombineCols, c = it - j * kCombineCols;
+    const bool sh = j == K;  // u = 0 serves token t in slot t
+    const float *src = a.ws.o + static_cast<int64_t>(sh ? t : s_pos[j]) * TM * D + d0 + c;
+    const int nq = sh ? js : jr;
+    float v[kMaxSlices];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
-    if (j < K) v[j] = __ldcg(a.ws.o + static_cast<int64_t>(s_pos[j]) * D + d);
-  float y = 0.f;
+    for (int q = 0; q < kMaxSlices; ++q)
+      if (q < nq) v[q] = __ldcg(src + static_cast<int64_t>(q) * D);
+    float o = 0.f;
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
-    if (j < K) y = fmaf(s_w[j], v[j], y);
-  y += sh;
-  if (a.residual) y = xs + y;
-  if (a.y_bf16)
-    static_cast<__nv_bfloat16 *>(a.y)[i] = __float2bfloat16_rn(y);
-  else
-    static_cast<float *>(a.y)[i] = y;
-  if (a.y_copy) a.y_copy[i] = y;
+    for (int q = 0; q < kMaxSlices; ++q)
+      if (q < nq) o += v[q];
+    for (int q = kMaxSlices; q < nq; ++q) o += __ldcg(src + static_cast<int64_t>(q) * D);
+    s_o[j * kCombineCols + c] = o;
+  }
+  __syncthreads();
+  if (tid < kCombineCols) {
+    const int64_t i = static_cast<int64_t>(t) * D + d0 + tid;
+    float sh = ns ? s_o[K * kCombineCols + tid] : 0.f;
+    if (a.sh.shared_gate) sh *= 1.0f / (1.0f + __expf(-__ldcg(a.ws.gate_logit + t)));
+    float y = 0.f;
+    for (int j = 0; j < K; ++j) y = fmaf(s_w[j], s_o[j * kCombineCols + tid], y);
+    y += sh;
+    if (a.residual) y = load_act(a.x, i, a.x_bf16) + y;
+    if (a.y_bf16)
+      static_cast<__nv_bfloat16 *>(a.y)[i] = __float2bfloat16_rn(y);
+    else
+      static_cast<float *>(a.y)[i] = y;
+    if (a.y_copy) a.y_copy[i] = y;
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1713,7 +1717,7 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
   // 3. weighted combine
   {
     rec(a, kProfDown, 0, st);
-    err = launch_pdl(k_combine, a.n * (a.sh.d / kCombineThreads), kCombineThreads, 0, st, a);
+    err = launch_pdl(k_combine, a.n * (a.sh.d / kCombineCols), kCombineThreads, 0, st, a);
     if (err != cudaSuccess) return err;
     rec(a, kProfDown, 1, st);
   }

@@ -92,10 +92,12 @@ static_assert(sizeof(ActRec) == 144, "ActRec is 9 x 16 bytes");
 
 // Decode workspace (n <= 8 tokens).  u indexes active experts: u = 0 is the shared expert
 // when there is one, routed active experts follow in ascending expert id.  A GEMV "unit" is one
-// 128-row tile of one active expert's matrix (pair); its K range is cut into fixed segments of
-// 2 or 4 chunks whose fp32 sums are added in segment order, whether one CTA runs the whole
-// unit or several CTAs each take a run of segments (then the segment sums pass through the
-// partial buffers), so results do not depend on how the work was split.
+// 128-row tile j of one active expert's gate/up pair for one token group, followed by the down
+// matrix over K-slice j (the 128 values of h the tile makes).  The gate/up K range is cut into
+// fixed segments of 2 or 4 chunks whose fp32 sums are added in segment order, whether one CTA
+// runs the whole unit or several CTAs each take a run of segments (then the segment sums pass
+// through the partial buffers); the down outputs of each K-slice are kept apart and added in
+// slice order by the combine, so results do not depend on how the work was split.
 struct DecodeWs {
   float *logits;        // [8][E] selection scores (logit + bias)
   float *raw_logits;    // [8][E] unbiased logits (selection-only bias)
@@ -106,25 +108,20 @@ struct DecodeWs {
   float *route_w;       // [8][k]
   int *slotpos;         // [8][k]: u * 8 + i (i = position of the token in expert u's list)
   // (The GEMV kernel's task table lives in each CTA's shared memory: a header [n_active,
-  // gate/up tasks, down pieces per output tile, 0] and one 16-int row per active expert u:
-  // [expert (E = shared), ntok, tokens 0..7, first gate/up task, gate/up split, first down
-  // piece, down split, token groups, 0]; a split packs run length | pieces << 8 | chunks per
-  // segment << 16 | segments << 20.)
+  // tasks, 0, 0] and one 16-int row per active expert u: [expert (E = shared), ntok, tokens
+  // 0..7, first task, split, 0, 0, token groups, 0]; a split packs run length | pieces << 8 |
+  // chunks per segment << 16 | segments << 20.)
   ActRec *xrec;         // [8][D/64]
-  ActRec *hrec;         // [umax][8][fmax/64]
   float *gu_part;       // [umax][tmax][gu_nseg][2][8][128] gate/up segment sums
-  float *dn_part;       // [umax][D/128][dn_nseg][8][128]  down segment sums
-  float *o;             // [umax * 8][D] expert outputs (unweighted)
-  unsigned *gu_ticket;      // [umax][tmax][8] (token groups)
-  unsigned *dn_ticket;      // [umax][D/128][8] (token groups)
-  unsigned *counters;       // [2] work queue of the GEMV kernel (gate/up pieces, then down pieces)
-  unsigned *h_done;         // [umax][8] (token groups): (tile, consumer warp) pairs that wrote h
+  float *o;             // [umax * 8][tmax][D] expert outputs per K-slice of the down matrix (unweighted)
+  unsigned *gu_ticket;  // [umax][tmax][8] (token groups): pieces of a split unit that stored their partials
+  unsigned *gu_depart;  // [umax][tmax][8]: pieces of a split unit that have read every partial
+  unsigned *counters;   // [2] work queue of the GEMV kernel
   int umax;
   int tmax;             // max(F, F_shared) / 128
   int fmax;
   int gu_seg;           // gate/up: chunks per K segment (2 or 4)
   int gu_nseg;          // gate/up: K segments (d_model / 64 / gu_seg)
-  int dn_nseg;          // down: most K segments of any expert
   int grid_gemv;        // persistent grid of the GEMV kernel
   int min_streams;      // the grid: units are cut into floor(grid / units) pieces
 };
