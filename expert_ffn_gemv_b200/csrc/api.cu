@@ -1,4 +1,5 @@
 // api.cu -- the C ABI (include/moe.h): handle lifetime, weight loading, forward calls.
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -607,8 +608,10 @@ moe_status moe_forward(moe_handle *h, int32_t layer, const void *x, void *y, int
   const bool xh = !is_device_ptr(x), yh = !is_device_ptr(y);
   const void *xd = x;
   void *yd = y;
-  if (xh) {
-    cudaError_t e = cudaMemcpyAsync(h->x_stage, x, xbytes, cudaMemcpyHostToDevice, st);
+  // host inputs are uploaded; device inputs off a 16-byte boundary (the kernels read them 16
+  // bytes at a time) are copied into the aligned staging buffer
+  if (xh || (reinterpret_cast<uintptr_t>(x) & 15u)) {
+    cudaError_t e = cudaMemcpyAsync(h->x_stage, x, xbytes, xh ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "input upload");
     xd = h->x_stage;
   }
@@ -645,8 +648,9 @@ moe_status moe_forward_stack(moe_handle *h, int32_t first_layer, int32_t n_layer
   const uint64_t nd = static_cast<uint64_t>(n_tokens) * D;
   const bool xh = !is_device_ptr(x_in), yh = !is_device_ptr(x_out);
   const void *cur = x_in;
-  if (xh) {
-    cudaError_t e = cudaMemcpyAsync(h->x_stage, x_in, nd * dtype_size(g.act_dtype), cudaMemcpyHostToDevice, st);
+  if (xh || (reinterpret_cast<uintptr_t>(x_in) & 15u)) {  // upload, or realign a device input
+    cudaError_t e = cudaMemcpyAsync(h->x_stage, x_in, nd * dtype_size(g.act_dtype),
+                                    xh ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "input upload");
     cur = h->x_stage;
   }

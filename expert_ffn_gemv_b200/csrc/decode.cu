@@ -582,6 +582,307 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------------------------------
+// Router as one cluster of 16 CTAs per token (bf16 router rows; at most 48 rows per CTA and
+// d_model up to 2,048): every CTA bulk-copies its rows of the router into shared memory before
+// it waits for the previous kernel, computes their logits for its token (fp32 sums) and stores
+// them into CTA 0's shared memory over the cluster (distributed shared memory); after one
+// cluster barrier CTA 0 takes the top-k and the fp32 softmax.  No logit crosses global memory
+// and no CTA waits on a global counter.  The same CTAs quantise the token's input into the
+// activation records.
+// ------------------------------------------------------------------------------------------
+constexpr int kClCtas = 16, kClThreads = 512, kClWarps = kClThreads / 32, kClRowsPerWarp = 3;
+constexpr int kClMaxD = 2048, kClMaxExperts = 1024;
+
+struct ClPlan {
+  int R;                           // router rows per CTA
+  int w, x, lg, raw, keys, tk, total;  // byte offsets: rows, x (fp32), logits, raw logits, keys, top-k scratch
+};
+__host__ __device__ inline ClPlan cl_plan(int ER, int D) {
+  ClPlan p;
+  p.R = (ER + kClCtas - 1) / kClCtas;
+  const int er = p.R * kClCtas;
+  p.w = 128;  // [0, 128): the rows' mbarrier
+  p.x = p.w + ((p.R * D * 2 + 127) & ~127);
+  p.lg = p.x + D * 4;
+  p.raw = p.lg + er * 4;
+  p.keys = p.raw + er * 4;
+  p.tk = p.keys + er * 4;
+  p.total = p.tk + kTopkScratch * 4;
+  return p;
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// every thread of every CTA of the cluster: stores before it are visible to loads after it
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Top-k of one token from its logits in shared memory by one warp (lane l holds experts
+// l + 32 q), the rank-count pass of the GEMV path's top-k: T = the K-th largest lane maximum,
+// the candidates (keys >= T) ranked by counting (descending key, ties to the lower expert).
+// Results: sv[j] the j-th selected logit, si[j] its expert.  False when the candidates are too
+// many or too few (equal or non-finite logits).
+template <int VPL>
+__device__ bool cl_topk_rank(const float *lg, int E, int K, int lane, uint32_t *ws, float *sv, int *si) {
+  uint32_t key[VPL];
+#pragma unroll
+  for (int q = 0; q < VPL; ++q) key[q] = lane + 32 * q < E ? order_key(lg[lane + 32 * q]) : 0u;
+  uint32_t mk = key[0];
+#pragma unroll
+  for (int q = 1; q < VPL; ++q) mk = max(mk, key[q]);
+  ws[lane] = mk;
+  __syncwarp();
+  int r = 0;
+#pragma unroll 8
+  for (int l = 0; l < 32; ++l) {
+    const uint32_t o = ws[l];
+    r += (o > mk) || (o == mk && l < lane);
+  }
+  const uint32_t T = __shfl_sync(0xffffffffu, mk, __ffs(__ballot_sync(0xffffffffu, r == K - 1)) - 1);
+  int c = 0;
+#pragma unroll
+  for (int q = 0; q < VPL; ++q) c += (key[q] >= T && lane + 32 * q < E) ? 1 : 0;
+  int inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  const int C = __shfl_sync(0xffffffffu, inc, 31);
+  if (C > kTopkCand || C < K) return false;
+  uint32_t *ck = ws + 32, *ci = ck + kTopkCand;
+  int o = inc - c;
+#pragma unroll
+  for (int q = 0; q < VPL; ++q)
+    if (key[q] >= T && lane + 32 * q < E) {
+      ck[o] = key[q];
+      ci[o] = lane + 32 * q;
+      ++o;
+    }
+  __syncwarp();
+  for (int i = lane; i < C; i += 32) {
+    const uint32_t ki = ck[i];
+    const int ei = static_cast<int>(ci[i]);
+    int rk = 0;
+    for (int j = 0; j < C; ++j) {
+      const uint32_t kj = ck[j];
+      rk += (kj > ki) || (kj == ki && static_cast<int>(ci[j]) < ei);
+    }
+    if (rk < K) {
+      sv[rk] = key_value(ki);
+      si[rk] = ei;
+    }
+  }
+  __syncwarp();
+  return true;
+}
+
+// The same selection by rounds of a warp argmax over keys in shared memory (any logits).
+__device__ void cl_topk_rounds(const float *lg, uint32_t *keys, int E, int K, int lane, float *sv, int *si) {
+  for (int i = lane; i < E; i += 32) keys[i] = order_key(lg[i]);
+  __syncwarp();
+  for (int j = 0; j < K; ++j) {
+    uint32_t bk = 0u;
+    int bi = 0x7fffffff;
+    for (int i = lane; i < E; i += 32) {
+      const uint32_t v = keys[i];
+      if (v > bk) {
+        bk = v;
+        bi = i;
+      }
+    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    bi = __reduce_min_sync(0xffffffffu, bk == m ? bi : 0x7fffffff);
+    if (bi >= E) bi = j;  // cannot happen (K <= E keys >= 1)
+    if (lane == 0) {
+      keys[bi] = 0u;
+      sv[j] = key_value(m);
+      si[j] = bi;
+    }
+    __syncwarp();
+  }
+}
+
+template <bool XBF16>
+__global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char cs[];
+  const int D = a.sh.d, E = a.sh.e, K = a.sh.k, ER = E + a.sh.shared_gate;
+  const ClPlan P = cl_plan(ER, D);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = static_cast<int>(cluster_ctarank());
+  const int t = blockIdx.x / kClCtas;
+  const int r0 = c * P.R, r1 = min(ER, r0 + P.R);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(cs);
+  // this CTA's router rows (written by no kernel) and their biases, while the previous kernel
+  // finishes
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    if (r1 > r0) {
+      const uint32_t bytes = static_cast<uint32_t>((r1 - r0) * D * 2);
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_g2s(cs + P.w, static_cast<const __nv_bfloat16 *>(a.L.router_w) + static_cast<int64_t>(r0) * D, bytes, bar);
+    } else {
+      mbar_arrive(bar);
+    }
+  }
+  float bias_r[kClRowsPerWarp];
+#pragma unroll
+  for (int i = 0; i < kClRowsPerWarp; ++i) {
+    const int row = r0 + warp + kClWarps * i;
+    bias_r[i] = row < r1 && row < E ? __ldg(a.L.bias + row) : 0.f;
+  }
+  griddep_wait();
+  griddep_launch();
+  if (blockIdx.x == 0 && tid < 2) a.ws.counters[tid] = 0u;  // the GEMV kernel's work queue starts empty
+  // token t's input, fp32, in shared memory
+  float *xs = reinterpret_cast<float *>(cs + P.x);
+  if (XBF16) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + static_cast<int64_t>(t) * D);
+    for (int i = tid; i < D / 8; i += kClThreads) {
+      const uint4 q = __ldg(src + i);
+      float4 *dst = reinterpret_cast<float4 *>(xs) + 2 * i;
+      dst[0] = make_float4(__uint_as_float(q.x << 16), __uint_as_float(q.x & 0xFFFF0000u), __uint_as_float(q.y << 16),
+                           __uint_as_float(q.y & 0xFFFF0000u));
+      dst[1] = make_float4(__uint_as_float(q.z << 16), __uint_as_float(q.z & 0xFFFF0000u), __uint_as_float(q.w << 16),
+                           __uint_as_float(q.w & 0xFFFF0000u));
+    }
+  } else {
+    const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + static_cast<int64_t>(t) * D);
+    for (int i = tid; i < D / 4; i += kClThreads) reinterpret_cast<float4 *>(xs)[i] = __ldg(src + i);
+  }
+  __syncthreads();
+  // activation records of token t: warp per 128-column group, lane = 4 columns
+  for (int g = c + kClCtas * warp; g < D / kQGroup; g += kClCtas * kClWarps) {
+    const float4 v = reinterpret_cast<const float4 *>(xs + g * kQGroup)[lane];
+    float mx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const int ex = fix16_exponent(mx);
+    const float sc = pow2f(ex);
+    const int q0 = fix16(v.x, sc), q1 = fix16(v.y, sc), q2 = fix16(v.z, sc), q3 = fix16(v.w, sc);
+    ActRec *rec = a.ws.xrec + static_cast<int64_t>(t) * (D / kChunk) + (g * kQGroup) / kChunk + (lane >> 4);
+    *reinterpret_cast<uint2 *>(&rec->x[(4 * lane) & 63]) =
+        make_uint2((static_cast<uint32_t>(q0) & 0xFFFFu) | (static_cast<uint32_t>(q1) << 16),
+                   (static_cast<uint32_t>(q2) & 0xFFFFu) | (static_cast<uint32_t>(q3) << 16));
+    int sm = q0 + q1 + q2 + q3;  // eight lanes = one 32-column block
+    sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+    sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+    sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+    if ((lane & 7) == 0) rec->m[(lane >> 3) & 1] = a.sh.fmt == MOE_FMT_Q2_32 ? kQ2SumMul * sm : sm;
+    if ((lane & 15) == 0) {
+      rec->f = pow2f(-ex) * rec_factor(a.sh.fmt);
+      rec->pad = 0u;
+    }
+  }
+  // logits of this CTA's rows: warp = rows warp, warp + 16, warp + 32; lane = 8-column groups
+  // lane, lane + 32, ... (fp32 sums over the whole d_model), stored into CTA 0
+  if (!mbar_wait_bounded(bar, 0u, a.spin_limit) && lane == 0) flag_error(a.err, kErrTimeout);
+  const int G8 = D / 256;
+  float xv[kClMaxD / 256][8];
+#pragma unroll
+  for (int j = 0; j < kClMaxD / 256; ++j)
+    if (j < G8) {
+      const float4 *p = reinterpret_cast<const float4 *>(xs + 8 * lane + 256 * j);
+      const float4 u = p[0], w = p[1];
+      xv[j][0] = u.x; xv[j][1] = u.y; xv[j][2] = u.z; xv[j][3] = u.w;
+      xv[j][4] = w.x; xv[j][5] = w.y; xv[j][6] = w.z; xv[j][7] = w.w;
+    }
+  const uint32_t lg0 = mapa_shared(smem_u32(cs + P.lg), 0u), raw0 = mapa_shared(smem_u32(cs + P.raw), 0u);
+  const __nv_bfloat16 *wsm = reinterpret_cast<const __nv_bfloat16 *>(cs + P.w);
+#pragma unroll
+  for (int i = 0; i < kClRowsPerWarp; ++i) {
+    const int rl = warp + kClWarps * i, row = r0 + rl;
+    if (row < r1) {
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < kClMaxD / 256; ++j)
+        if (j < G8) {
+          const uint4 q = *reinterpret_cast<const uint4 *>(wsm + static_cast<int64_t>(rl) * D + 8 * lane + 256 * j);
+          const uint32_t pw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            s = fmaf(__uint_as_float(pw[k2] << 16), xv[j][2 * k2], s);
+            s = fmaf(__uint_as_float(pw[k2] & 0xFFFF0000u), xv[j][2 * k2 + 1], s);
+          }
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) {
+        if (row < E) {
+          st_cluster_f32(lg0 + 4u * row, s + bias_r[i]);
+          st_cluster_f32(raw0 + 4u * row, s);
+        } else {
+          a.ws.gate_logit[t] = s;  // the shared expert's gate row
+        }
+      }
+    }
+  }
+  cluster_sync_all();
+  if (c != 0) return;
+  // top-k + softmax of token t by warp 0 of CTA 0
+  if (warp != 0) return;
+  const float *lg = reinterpret_cast<const float *>(cs + P.lg), *raw = reinterpret_cast<const float *>(cs + P.raw);
+  uint32_t *ws = reinterpret_cast<uint32_t *>(cs + P.tk);
+  float *sv = reinterpret_cast<float *>(ws + 32 + 2 * kTopkCand);
+  int *si = reinterpret_cast<int *>(sv + kMaxTopK);
+  {
+    bool done;
+    if (E <= 128) done = cl_topk_rank<4>(lg, E, K, lane, ws, sv, si);
+    else if (E <= 256) done = cl_topk_rank<8>(lg, E, K, lane, ws, sv, si);
+    else if (E <= 512) done = cl_topk_rank<16>(lg, E, K, lane, ws, sv, si);
+    else done = cl_topk_rank<32>(lg, E, K, lane, ws, sv, si);
+    if (!done)
+      cl_topk_rounds(lg, reinterpret_cast<uint32_t *>(cs + P.keys), E, K, lane, sv, si);
+    __syncwarp();
+  }
+  int my_i = lane < K ? si[lane] : 0;
+  if (my_i < 0 || my_i >= E) {  // cannot happen: keep the index in range
+    flag_error(a.err, kErrBadIndex);
+    my_i = 0;
+  }
+  // weights: softmax over the selected logits (selection-only bias: over their unbiased logits)
+  float my_l = lane < K ? (a.sh.bias_select ? raw[my_i] : sv[lane]) : -INFINITY;
+  float l0 = my_l;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l0 = fmaxf(l0, __shfl_xor_sync(0xffffffffu, l0, o));
+  if (lane == 0 && !(l0 > -INFINITY && l0 < INFINITY)) flag_error(a.err, kErrBadIndex);
+  float w = lane < K ? __expf(my_l - l0) : 0.f;
+  float sum = w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < K) {
+    w = w / sum;
+    a.ws.sel[t * K + lane] = my_i;
+    a.ws.route_idx[t * K + lane] = my_i;
+    a.ws.route_w[t * K + lane] = w;
+    if (a.out_idx) a.out_idx[t * K + lane] = my_i;
+    if (a.out_w) a.out_w[t * K + lane] = w;
+  }
+}
+
+// Whether the cluster router serves this layer shape (set up once by configure_decode_kernels).
+static bool g_route_cluster = false;
+static bool route_cluster_fits(const Shape &sh) {
+  const int ER = sh.e + sh.shared_gate;
+  return g_route_cluster && sh.router_bf16 && sh.d <= kClMaxD && sh.d % 256 == 0 && sh.e <= kClMaxExperts &&
+         (ER + kClCtas - 1) / kClCtas <= kClWarps * kClRowsPerWarp && cl_plan(ER, sh.d).total <= 200 * 1024;
+}
+
+// ------------------------------------------------------------------------------------------
 // routing tables, built by every GEMV CTA in its own shared memory
 // ------------------------------------------------------------------------------------------
 // Scratch (the ring's stage area, unused until the tables exist): tokmask [E] (bit t = token t
@@ -1659,7 +1960,58 @@ cudaError_t configure_decode_kernels() {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     if (e != cudaSuccess) return e;
   }
+  // the cluster router: 16-CTA clusters (beyond the portable 8) with up to 200 KB of shared
+  // memory per CTA; used only if the device can schedule such a cluster (MOE_ROUTE_CLUSTER=0 in
+  // the environment turns it off)
+  const char *rc = getenv("MOE_ROUTE_CLUSTER");
+  g_route_cluster = false;
+  if (!(rc && rc[0] == '0') && max_optin >= 200 * 1024) {
+    const void *kc[] = {(const void *)k_route_cl<true>, (const void *)k_route_cl<false>};
+    bool ok = true;
+    for (const void *k : kc) {
+      ok = ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) == cudaSuccess &&
+           cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    }
+    if (ok) {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(kClCtas);
+      cfg.blockDim = dim3(kClThreads);
+      cfg.dynamicSmemBytes = 200 * 1024;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = kClCtas;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int nclusters = 0;
+      ok = cudaOccupancyMaxActiveClusters(&nclusters, (const void *)k_route_cl<true>, &cfg) == cudaSuccess &&
+           nclusters >= 1;
+    }
+    (void)cudaGetLastError();  // a refused query leaves the plain router in place
+    g_route_cluster = ok;
+  }
   return cudaSuccess;
+}
+
+// Launch of the cluster router: n clusters of 16 CTAs, programmatic stream serialization.
+template <bool XBF16>
+static cudaError_t launch_route_cluster(const DecodeArgs &a, cudaStream_t st) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(a.n * kClCtas);
+  cfg.blockDim = dim3(kClThreads);
+  cfg.dynamicSmemBytes = cl_plan(a.sh.e + a.sh.shared_gate, a.sh.d).total;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kClCtas;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, k_route_cl<XBF16>, a);
 }
 
 static int gemv_smem(int fmt, int umax) { return ring_plan(fmt, 1, kStageSlots, umax).total; }
@@ -1695,7 +2047,9 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
     const int grid = (a.sh.e + a.sh.shared_gate + kRouteExperts - 1) / kRouteExperts;
     const int sm = a.sh.e > 1024 ? a.sh.e * 4 : 0;  // one logit row for the shared-memory top-k
     rec(a, kProfRoute, 0, st);
-    if (a.sh.router_bf16)
+    if (route_cluster_fits(a.sh))
+      err = a.x_bf16 ? launch_route_cluster<true>(a, st) : launch_route_cluster<false>(a, st);
+    else if (a.sh.router_bf16)
       err = a.x_bf16 ? launch_pdl(k_route<true, true>, grid, kRouteThreads, sm, st, a)
                      : launch_pdl(k_route<true, false>, grid, kRouteThreads, sm, st, a);
     else

@@ -83,6 +83,19 @@ def test_small_layer_tokens(torch_cuda, fmt, n):
     moe.close()
 
 
+@pytest.mark.parametrize("n_experts,top_k", [(600, 8), (1000, 10), (2048, 16)])
+@pytest.mark.parametrize("n", [1, 8])
+def test_many_experts(torch_cuda, n_experts, top_k, n):
+    """Routers wider than 512 experts (the top-k takes one logit row per token in shared memory)."""
+    torch = torch_cuda
+    wl = synth.small_workload(d_model=256, d_ff=128, n_experts=n_experts, top_k=top_k, n_shared=1, shared_d_ff=128)
+    moe = moe_for(wl, 1, 8, seed=6)
+    load_layer_device(moe, 0, wl, 6, 0)
+    x, y, rb = _run_layer(torch, moe, wl, 6, n)
+    _check_layer(wl, 6, 0, x, y, rb)
+    moe.close()
+
+
 @pytest.mark.parametrize("fmt", FORMATS)
 def test_host_and_device_loads_agree(torch_cuda, fmt):
     torch = torch_cuda

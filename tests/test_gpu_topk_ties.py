@@ -6,6 +6,7 @@ applies.  A zero router makes every token's logits equal to the bias:
                   round-based pass (warp argmax per selection) runs;
   * few_values -- four distinct bias values: the rank-count pass runs with ties among the
                   candidates.
+Both at 128 experts (warp per token) and 1,000 (more than 512: the one-row pass).
 
 Indices are compared in order, the softmax weights and the outputs against the oracle."""
 import numpy as np
@@ -26,11 +27,12 @@ def _bias(pattern: str, e: int) -> np.ndarray:
 
 @pytest.mark.parametrize("pattern", ["all_equal", "few_values"])
 @pytest.mark.parametrize("n", [1, 8])
-def test_topk_exact_ties(pattern, n):
+@pytest.mark.parametrize("n_experts", [128, 1000])
+def test_topk_exact_ties(pattern, n, n_experts):
     import torch
 
     assert torch.cuda.is_available()
-    wl = synth.small_workload(d_model=256, d_ff=128, n_experts=128, top_k=8, n_shared=1, shared_d_ff=128)
+    wl = synth.small_workload(d_model=256, d_ff=128, n_experts=n_experts, top_k=8, n_shared=1, shared_d_ff=128)
     seed = 11
     experts = synth.gen_layer_experts(wl, seed, 0)
     shared = synth.gen_shared(wl, seed, 0)
