@@ -1239,14 +1239,6 @@ __device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float (&f)[4]) {
   f[3] = b.y;
 }
 
-// NVFP4: the int8 operands (2 x E2M1 value) of weights 4q .. 4q+3: the magnitude selector picks
-// bytes of the table {0, 1, 2, 3, 4, 6, 8, 12}; the sign bits negate (never a zero, see the repack).
-__device__ __forceinline__ uint32_t nv_operand(uint32_t sel, uint32_t sgn, int g) {
-  const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, sel & 0x7777u);
-  const uint32_t m = prmt_sign_bytes(sgn << (7 - g));
-  return (mag ^ m) + (m & 0x01010101u);
-}
-
 // NVFP4 GEMV of NR matrices over the nch chunks of a stage, tokens 0 .. TN-1: per 16-weight block
 // an exact integer dot product (8 dp2a), scaled by the block's E4M3 scale; the activation factor
 // per chunk; the matrices' tensor scales come at the unit's end.
@@ -1256,11 +1248,10 @@ __device__ __forceinline__ void gemv_stage_nv(const unsigned char *st, const Rin
   constexpr uint32_t kRec = sizeof(ActRec);
   const int r = threadIdx.x;
   const uint32_t base = smem_u32(st);
-  const uint32_t pa = base + P.a, ps = base + P.s, pg = base + P.g;
+  const uint32_t pa = base + P.a, ps = base + P.s;
 #pragma unroll 1
   for (int c = 0; c < nch; ++c) {
     uint32_t A[NR][8];
-    uint2 G[NR];
     float sc[NR][4];
 #pragma unroll
     for (int m = 0; m < NR; ++m) {
@@ -1268,7 +1259,6 @@ __device__ __forceinline__ void gemv_stage_nv(const unsigned char *st, const Rin
       const uint4 a0 = lds_u128(pa + row * 32), a1 = lds_u128(pa + row * 32 + 16);
       A[m][0] = a0.x; A[m][1] = a0.y; A[m][2] = a0.z; A[m][3] = a0.w;
       A[m][4] = a1.x; A[m][5] = a1.y; A[m][6] = a1.z; A[m][7] = a1.w;
-      G[m] = lds_u64(pg + row * 8);
       e4m3x4_to_float(lds_u32(ps + row * 4), sc[m]);
     }
     float cacc[NR][TN];
@@ -1278,15 +1268,12 @@ __device__ __forceinline__ void gemv_stage_nv(const unsigned char *st, const Rin
       for (int t = 0; t < TN; ++t) cacc[m][t] = 0.f;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {  // 16-weight blocks: groups q = 4b .. 4b+3, words 2b, 2b+1
-      uint32_t v[NR][4];
+      uint32_t v[NR][4];  // groups q = 4b .. 4b+3 = the halves of words 2b, 2b+1
 #pragma unroll
-      for (int m = 0; m < NR; ++m)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int q = 4 * b + j;
-          const uint32_t w = A[m][q >> 1];
-          v[m][j] = nv_operand((q & 1) ? (w >> 16) : w, (q < 8) ? G[m].x : G[m].y, q & 7);
-        }
+      for (int m = 0; m < NR; ++m) {
+        nv_operands(A[m][2 * b], v[m][0], v[m][1]);
+        nv_operands(A[m][2 * b + 1], v[m][2], v[m][3]);
+      }
 #pragma unroll
       for (int t = 0; t < TN; ++t) {
         const uint32_t ra = rec + (t * CMAX + c) * kRec + 32 * b;  // 16 int16 = weights 16b .. 16b+15

@@ -13,10 +13,11 @@
 // codes of weights 16w+4kk .. 16w+4kk+3 as bytes 0..3, the operand order of dp2a.
 // CB35 sign word of a block: byte j, bit g is the sign of weight 4g + j, so shifting left by
 // 7 - g puts the signs of group g in the byte msbs, where prmt can replicate them.
-// NVFP4: plane A holds 32 B per (row, chunk): the E2M1 magnitude indices (0..7) as 4-bit prmt
-// selectors, selector q (bits 16 (q % 2) of word q / 2) = weights 4q .. 4q+3; plane G the sign
-// bits in the CB35 arrangement (negative zero stored as zero); plane S the four E4M3 block
-// scales; the matrices' fp32 tensor scales sit in a small array of their own.
+// NVFP4: plane A holds 32 B per (row, chunk): the E2M1 codes as 4-bit prmt selectors, selector q
+// (bits 16 (q % 2) of word q / 2) = weights 4q .. 4q+3, nibble j = weight 4q + j (magnitude index
+// in bits 0..2, sign in bit 3; a negative zero is stored as zero), so no sign plane is needed
+// and a chunk costs what its interchange blocks do (36 B); plane S the four E4M3 block scales;
+// the matrices' fp32 tensor scales sit in a small array of their own.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -43,13 +44,13 @@ constexpr uint32_t kErrBadIndex = 2u;
 // One group of experts with equal shapes (all routed experts, or the shared expert).
 // device plane bytes per (row, 64-weight chunk)
 __host__ __device__ constexpr int plane_a_bytes(int fmt) { return fmt == MOE_FMT_NVFP4_16 ? 32 : 16; }
-__host__ __device__ constexpr bool has_plane_g(int fmt) { return fmt != MOE_FMT_Q2_32; }
+__host__ __device__ constexpr bool has_plane_g(int fmt) { return fmt == MOE_FMT_CB35_32; }
 __host__ __device__ constexpr int plane_bytes(int fmt) { return plane_a_bytes(fmt) + 4 + (has_plane_g(fmt) ? 8 : 0); }
 
 struct ExpertGroup {
   uint8_t *a;          // plane A of expert 0, matrix 0
   __half2 *s;          // plane S (NVFP4: four E4M3 bytes per slot)
-  uint2 *g;            // plane G (CB35, NVFP4) or nullptr
+  uint2 *g;            // plane G (CB35) or nullptr
   float *ts;           // NVFP4: tensor scales [expert][gate, up, down], else nullptr
   int64_t a_mat;       // bytes of plane A per matrix   = F * D / 4 (NVFP4: F * D / 2)
   int64_t s_mat;       // half2 per matrix              = F * D / 64
@@ -256,6 +257,23 @@ __device__ __forceinline__ uint32_t prmt_sign_bytes(uint32_t t) {
   uint32_t r;
   asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(r) : "r"(t));
   return r;
+}
+
+// NVFP4: the int8 operands (2 x E2M1 value) of the two selectors of word w (weights 4q .. 4q+3 in
+// the low half, 4q+4 .. 4q+7 in the high half): the magnitude bits pick bytes of the table
+// {0, 1, 2, 3, 4, 6, 8, 12}; byte masks of the sign bits (bit 3 of each nibble) come from one prmt
+// each -- bytes 0, 1 (2, 3) of w << 4 and of w hold the signs of nibbles 0, 2 and 1, 3 of the low
+// (high) half in their msbs -- and negate by two's complement (never a zero: the repack stores a
+// negative zero as zero).
+__device__ __forceinline__ void nv_operands(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  const uint32_t ml = __byte_perm(0x03020100u, 0x0C080604u, w & 0x7777u);
+  const uint32_t mh = __byte_perm(0x03020100u, 0x0C080604u, (w >> 16) & 0x7777u);
+  const uint32_t w4 = w << 4;
+  uint32_t sl, sh;
+  asm("prmt.b32 %0, %1, %2, 0xD9C8;" : "=r"(sl) : "r"(w4), "r"(w));
+  asm("prmt.b32 %0, %1, %2, 0xFBEA;" : "=r"(sh) : "r"(w4), "r"(w));
+  lo = (ml ^ sl) + (sl & 0x01010101u);
+  hi = (mh ^ sh) + (sh & 0x01010101u);
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }

@@ -631,7 +631,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
             // gives v s / 2 exactly (the tensor scale is applied in the epilogue)
             const uint4 Aw = reinterpret_cast<const uint4 *>(rm)[2 * r + h];
             const uint32_t aw[4] = {Aw.x, Aw.y, Aw.z, Aw.w};
-            const uint32_t sgn = reinterpret_cast<const uint32_t *>(rm + PL::kRawA + PL::kRawS)[2 * r + h];
             const uint32_t sw = reinterpret_cast<const uint32_t *>(rm + PL::kRawA)[r];
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
@@ -642,14 +641,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_pf_gemm(const __grid_constant
               const __nv_bfloat162 s2 = __floats2bfloat162_rn(0.5f * sf, 0.5f * sf);
               const __nv_bfloat162 c2 = __floats2bfloat162_rn(-96.0f * sf, -96.0f * sf);
               uint32_t o[4];
+              uint32_t vv[2];  // groups 2cc, 2cc + 1 of the half = the two selectors of word cc
+              nv_operands(aw[cc], vv[0], vv[1]);
 #pragma unroll
               for (int gg = 0; gg < 2; ++gg) {
-                const int g = 2 * cc + gg;  // group of 4 weights within the half
-                const uint32_t w = aw[g >> 1];
-                const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, ((g & 1) ? (w >> 16) : w) & 0x7777u);
-                const uint32_t mk = prmt_sign_bytes(sgn << (7 - g));
-                const uint32_t v = (mag ^ mk) + (mk & 0x01010101u);
-                const uint32_t u = (v ^ 0x80808080u) - 0x40404040u;  // v + 64 per byte, in 52 .. 76
+                const uint32_t u = (vv[gg] ^ 0x80808080u) - 0x40404040u;  // v + 64 per byte, in 52 .. 76
                 const uint32_t lo = __byte_perm(u, 0x43434343u, 0x5140), hi = __byte_perm(u, 0x43434343u, 0x5342);
                 const __nv_bfloat162 r0 = __hfma2(*reinterpret_cast<const __nv_bfloat162 *>(&lo), s2, c2);
                 const __nv_bfloat162 r1 = __hfma2(*reinterpret_cast<const __nv_bfloat162 *>(&hi), s2, c2);

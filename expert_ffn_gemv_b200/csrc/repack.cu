@@ -4,13 +4,13 @@
 
 namespace moe {
 
-// NVFP4: one thread per (matrix, row, chunk of 64 weights = interchange blocks 4c .. 4c+3):
-// magnitude indices into prmt selectors (plane A, 32 B), signs into the CB35 arrangement (plane
-// G; a negative zero is stored as zero), the four E4M3 scale bytes (plane S); the matrix's
-// tensor scale (its first 4 bytes) goes to ts[mi * ts_stride].
+// NVFP4: one thread per (matrix, row, chunk of 64 weights = interchange blocks 4c .. 4c+3): the
+// E2M1 codes into prmt selectors (plane A, 32 B; a negative zero is stored as zero), the four
+// E4M3 scale bytes (plane S); the matrix's tensor scale (its first 4 bytes) goes to
+// ts[mi * ts_stride].
 __global__ void k_repack_nvfp4(const uint8_t *__restrict__ src, int64_t src_stride, int rows, int cols, int n_mats,
                                int64_t dst_stride, uint8_t *__restrict__ a, uint32_t *__restrict__ s,
-                               uint2 *__restrict__ g, float *__restrict__ ts, int ts_stride) {
+                               float *__restrict__ ts, int ts_stride) {
   const int nc = cols / kChunk;
   const int64_t per_mat = static_cast<int64_t>(rows) * nc;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -27,22 +27,19 @@ __global__ void k_repack_nvfp4(const uint8_t *__restrict__ src, int64_t src_stri
   const uint8_t *b0 = m0 + 4 + (static_cast<int64_t>(row) * (cols / 16) + 4 * c) * 9;
   const int64_t slot = mat * dst_stride + (static_cast<int64_t>(row / kTileRows) * nc + c) * kTileRows +
                        (row % kTileRows);
-  uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sg[2] = {0, 0}, sc = 0;
+  uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sc = 0;
   for (int k = 0; k < 4; ++k) sc |= static_cast<uint32_t>(b0[9 * k]) << (8 * k);
   for (int p = 0; p < 64; ++p) {
     const uint8_t *blk = b0 + 9 * (p >> 4);
     const int i = p & 15;
-    const uint32_t code = (blk[1 + (i >> 1)] >> (4 * (i & 1))) & 15u;
-    const uint32_t mag = code & 7u, neg = mag ? code >> 3 : 0u;
+    uint32_t code = (blk[1 + (i >> 1)] >> (4 * (i & 1))) & 15u;
+    if ((code & 7u) == 0u) code = 0u;  // a negative zero is stored as zero
     const int q = p >> 2, j = p & 3;
-    w[q >> 1] |= mag << (16 * (q & 1) + 4 * j);
-    const int i32 = p & 31;
-    sg[p >> 5] |= neg << (8 * (i32 & 3) + (i32 >> 2));
+    w[q >> 1] |= code << (16 * (q & 1) + 4 * j);
   }
   uint4 *dst = reinterpret_cast<uint4 *>(a) + 2 * slot;
   dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  g[slot] = make_uint2(sg[0], sg[1]);
   s[slot] = sc;
 }
 
@@ -115,7 +112,7 @@ cudaError_t launch_repack(const uint8_t *src, int64_t src_stride, int fmt, int r
   const int64_t blocks = (total + threads - 1) / threads;
   if (fmt == MOE_FMT_NVFP4_16)
     k_repack_nvfp4<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
-        src, src_stride, rows, cols, n_mats, dst_stride, a, reinterpret_cast<uint32_t *>(s), g, ts, ts_stride);
+        src, src_stride, rows, cols, n_mats, dst_stride, a, reinterpret_cast<uint32_t *>(s), ts, ts_stride);
   else if (fmt == MOE_FMT_Q2_32)
     k_repack<MOE_FMT_Q2_32><<<static_cast<unsigned>(blocks), threads, 0, st>>>(
         src, src_stride, rows, cols, n_mats, dst_stride, a, s, g);
