@@ -649,7 +649,10 @@ def bench_prefill(args, rank, world, local):
         roof = {"kernel": "k_pf_gemm<gate/up>", "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
                 "peak_kind": kind, "achieved": gu_gbs, "frac": gu_gbs / pk["hbm_gbs"] if gu_gbs else None,
                 "tflops": gu_tf}
-    roof.update({"avg_launch_us": kms / max(kcnt, 1) * 1e3, "traffic": None,
+    src = source_hash("expert_ffn_gemv_b200/csrc/prefill.cu", "expert_ffn_gemv_b200/csrc/prefill.cuh",
+                      "expert_ffn_gemv_b200/csrc/moe_internal.cuh")
+    roof.update({"avg_launch_us": kms / max(kcnt, 1) * 1e3,
+                 "traffic": profiled_traffic("k_pf_gemm", f"prefill{n}", src, bytes_gu),
                  "algorithmic_bytes_per_launch": bytes_gu, "flop_per_launch": flop_gu,
                  "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge})
     res = _base_result(wl, world, K, W, ms, "tokens/s", sum_over_ranks(n * K / (ms / 1e3), world))
