@@ -582,28 +582,30 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------------------------------
-// Router as one cluster of 16 CTAs per token (bf16 router rows; at most 48 rows per CTA and
-// d_model up to 2,048): every CTA bulk-copies its rows of the router into shared memory before
-// it waits for the previous kernel, computes their logits for its token (fp32 sums) and stores
-// them into CTA 0's shared memory over the cluster (distributed shared memory); after one
-// cluster barrier CTA 0 takes the top-k and the fp32 softmax.  No logit crosses global memory
-// and no CTA waits on a global counter.  The same CTAs quantise the token's input into the
-// activation records.
+// Router as clusters of 16 CTAs, each serving tpc tokens (1, or 2 when the tokens outnumber the
+// clusters the device holds at once; bf16 router rows; at most 48 rows per CTA and d_model up
+// to 2,048): every CTA bulk-copies its rows of the router into shared memory before it waits
+// for the previous kernel, computes their logits for each of its cluster's tokens (fp32 sums)
+// and stores those of token slot s into CTA s's shared memory over the cluster (distributed
+// shared memory); after one cluster barrier CTA s takes token s's top-k and fp32 softmax.  No
+// logit crosses global memory and no CTA waits on a global counter.  The same CTAs quantise
+// the tokens' inputs into the activation records.
 // ------------------------------------------------------------------------------------------
 constexpr int kClCtas = 16, kClThreads = 512, kClWarps = kClThreads / 32, kClRowsPerWarp = 3;
 constexpr int kClMaxD = 2048, kClMaxExperts = 1024;
+constexpr int kClMaxTpc = 2;  // tokens per cluster (at most)
 
 struct ClPlan {
   int R;                           // router rows per CTA
-  int w, x, lg, raw, keys, tk, total;  // byte offsets: rows, x (fp32), logits, raw logits, keys, top-k scratch
+  int w, x, lg, raw, keys, tk, total;  // byte offsets: rows, x (fp32, per token slot), logits, raw logits, keys, top-k scratch
 };
-__host__ __device__ inline ClPlan cl_plan(int ER, int D) {
+__host__ __device__ inline ClPlan cl_plan(int ER, int D, int tpc) {
   ClPlan p;
   p.R = (ER + kClCtas - 1) / kClCtas;
   const int er = p.R * kClCtas;
   p.w = 128;  // [0, 128): the rows' mbarrier
   p.x = p.w + ((p.R * D * 2 + 127) & ~127);
-  p.lg = p.x + D * 4;
+  p.lg = p.x + tpc * D * 4;
   p.raw = p.lg + er * 4;
   p.keys = p.raw + er * 4;
   p.tk = p.keys + er * 4;
@@ -717,13 +719,13 @@ __device__ void cl_topk_rounds(const float *lg, uint32_t *keys, int E, int K, in
 }
 
 template <bool XBF16>
-__global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a) {
+__global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a, int tpc) {
   extern __shared__ __align__(128) unsigned char cs[];
   const int D = a.sh.d, E = a.sh.e, K = a.sh.k, ER = E + a.sh.shared_gate;
-  const ClPlan P = cl_plan(ER, D);
+  const ClPlan P = cl_plan(ER, D, tpc);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = static_cast<int>(cluster_ctarank());
-  const int t = blockIdx.x / kClCtas;
+  const int t0 = (blockIdx.x / kClCtas) * tpc, nt = min(tpc, a.n - t0);  // this cluster's tokens
   const int r0 = c * P.R, r1 = min(ER, r0 + P.R);
   uint64_t *bar = reinterpret_cast<uint64_t *>(cs);
   // this CTA's router rows (written by no kernel) and their biases, while the previous kernel
@@ -748,11 +750,11 @@ __global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a) {
   griddep_wait();
   griddep_launch();
   if (blockIdx.x == 0 && tid < 2) a.ws.counters[tid] = 0u;  // the GEMV kernel's work queue starts empty
-  // token t's input, fp32, in shared memory
+  // the tokens' inputs, fp32, in shared memory (slot s: token t0 + s)
   float *xs = reinterpret_cast<float *>(cs + P.x);
   if (XBF16) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + static_cast<int64_t>(t) * D);
-    for (int i = tid; i < D / 8; i += kClThreads) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + static_cast<int64_t>(t0) * D);
+    for (int i = tid; i < nt * D / 8; i += kClThreads) {
       const uint4 q = __ldg(src + i);
       float4 *dst = reinterpret_cast<float4 *>(xs) + 2 * i;
       dst[0] = make_float4(__uint_as_float(q.x << 16), __uint_as_float(q.x & 0xFFFF0000u), __uint_as_float(q.y << 16),
@@ -761,13 +763,15 @@ __global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a) {
                            __uint_as_float(q.w & 0xFFFF0000u));
     }
   } else {
-    const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + static_cast<int64_t>(t) * D);
-    for (int i = tid; i < D / 4; i += kClThreads) reinterpret_cast<float4 *>(xs)[i] = __ldg(src + i);
+    const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + static_cast<int64_t>(t0) * D);
+    for (int i = tid; i < nt * D / 4; i += kClThreads) reinterpret_cast<float4 *>(xs)[i] = __ldg(src + i);
   }
   __syncthreads();
-  // activation records of token t: warp per 128-column group, lane = 4 columns
-  for (int g = c + kClCtas * warp; g < D / kQGroup; g += kClCtas * kClWarps) {
-    const float4 v = reinterpret_cast<const float4 *>(xs + g * kQGroup)[lane];
+  // activation records of the tokens: warp per (token slot, 128-column group), lane = 4 columns
+  const int GQ = D / kQGroup;
+  for (int gs = c + kClCtas * warp; gs < nt * GQ; gs += kClCtas * kClWarps) {
+    const int sl = gs / GQ, g = gs - sl * GQ, t = t0 + sl;
+    const float4 v = reinterpret_cast<const float4 *>(xs + sl * D + g * kQGroup)[lane];
     float mx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -788,21 +792,24 @@ __global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a) {
       rec->pad = 0u;
     }
   }
-  // logits of this CTA's rows: warp = rows warp, warp + 16, warp + 32; lane = 8-column groups
-  // lane, lane + 32, ... (fp32 sums over the whole d_model), stored into CTA 0
+  // logits of this CTA's rows for token slot sl: warp = rows warp, warp + 16, warp + 32; lane =
+  // 8-column groups lane, lane + 32, ... (fp32 sums over the whole d_model), stored into CTA sl
   if (!mbar_wait_bounded(bar, 0u, a.spin_limit) && lane == 0) flag_error(a.err, kErrTimeout);
   const int G8 = D / 256;
+  const __nv_bfloat16 *wsm = reinterpret_cast<const __nv_bfloat16 *>(cs + P.w);
+#pragma unroll 1
+  for (int sl = 0; sl < nt; ++sl) {
   float xv[kClMaxD / 256][8];
 #pragma unroll
   for (int j = 0; j < kClMaxD / 256; ++j)
     if (j < G8) {
-      const float4 *p = reinterpret_cast<const float4 *>(xs + 8 * lane + 256 * j);
+      const float4 *p = reinterpret_cast<const float4 *>(xs + sl * D + 8 * lane + 256 * j);
       const float4 u = p[0], w = p[1];
       xv[j][0] = u.x; xv[j][1] = u.y; xv[j][2] = u.z; xv[j][3] = u.w;
       xv[j][4] = w.x; xv[j][5] = w.y; xv[j][6] = w.z; xv[j][7] = w.w;
     }
-  const uint32_t lg0 = mapa_shared(smem_u32(cs + P.lg), 0u), raw0 = mapa_shared(smem_u32(cs + P.raw), 0u);
-  const __nv_bfloat16 *wsm = reinterpret_cast<const __nv_bfloat16 *>(cs + P.w);
+  const uint32_t lg0 = mapa_shared(smem_u32(cs + P.lg), static_cast<uint32_t>(sl)),
+                 raw0 = mapa_shared(smem_u32(cs + P.raw), static_cast<uint32_t>(sl));
 #pragma unroll
   for (int i = 0; i < kClRowsPerWarp; ++i) {
     const int rl = warp + kClWarps * i, row = r0 + rl;
@@ -826,15 +833,17 @@ __global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a) {
           st_cluster_f32(lg0 + 4u * row, s + bias_r[i]);
           st_cluster_f32(raw0 + 4u * row, s);
         } else {
-          a.ws.gate_logit[t] = s;  // the shared expert's gate row
+          a.ws.gate_logit[t0 + sl] = s;  // the shared expert's gate row
         }
       }
     }
   }
+  }  // token slots
   cluster_sync_all();
-  if (c != 0) return;
-  // top-k + softmax of token t by warp 0 of CTA 0
+  if (c >= nt) return;
+  // top-k + softmax of token t = t0 + c by warp 0 of CTA c
   if (warp != 0) return;
+  const int t = t0 + c;
   const float *lg = reinterpret_cast<const float *>(cs + P.lg), *raw = reinterpret_cast<const float *>(cs + P.raw);
   uint32_t *ws = reinterpret_cast<uint32_t *>(cs + P.tk);
   float *sv = reinterpret_cast<float *>(ws + 32 + 2 * kTopkCand);
@@ -874,12 +883,14 @@ __global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a) {
   }
 }
 
-// Whether the cluster router serves this layer shape (set up once by configure_decode_kernels).
+// Whether the cluster router serves this layer shape, and how many of its clusters the device
+// holds at once (both set up once by configure_decode_kernels).
 static bool g_route_cluster = false;
+static int g_cl_resident = 1;
 static bool route_cluster_fits(const Shape &sh) {
   const int ER = sh.e + sh.shared_gate;
   return g_route_cluster && sh.router_bf16 && sh.d <= kClMaxD && sh.d % 256 == 0 && sh.e <= kClMaxExperts &&
-         (ER + kClCtas - 1) / kClCtas <= kClWarps * kClRowsPerWarp && cl_plan(ER, sh.d).total <= 200 * 1024;
+         (ER + kClCtas - 1) / kClCtas <= kClWarps * kClRowsPerWarp && cl_plan(ER, sh.d, kClMaxTpc).total <= 200 * 1024;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1949,7 +1960,8 @@ cudaError_t configure_decode_kernels() {
   }
   // the cluster router: 16-CTA clusters (beyond the portable 8) with up to 200 KB of shared
   // memory per CTA; used only if the device can schedule such a cluster (MOE_ROUTE_CLUSTER=0 in
-  // the environment turns it off)
+  // the environment turns it off; =2 gives every cluster two tokens, as on a device that holds
+  // a single cluster at a time)
   const char *rc = getenv("MOE_ROUTE_CLUSTER");
   g_route_cluster = false;
   if (!(rc && rc[0] == '0') && max_optin >= 200 * 1024) {
@@ -1974,6 +1986,7 @@ cudaError_t configure_decode_kernels() {
       int nclusters = 0;
       ok = cudaOccupancyMaxActiveClusters(&nclusters, (const void *)k_route_cl<true>, &cfg) == cudaSuccess &&
            nclusters >= 1;
+      g_cl_resident = ok && !(rc && rc[0] == '2') ? nclusters : 1;
     }
     (void)cudaGetLastError();  // a refused query leaves the plain router in place
     g_route_cluster = ok;
@@ -1981,13 +1994,16 @@ cudaError_t configure_decode_kernels() {
   return cudaSuccess;
 }
 
-// Launch of the cluster router: n clusters of 16 CTAs, programmatic stream serialization.
+// Launch of the cluster router: one token per cluster while the device holds a cluster for every
+// token, else two (a second wave of clusters would start only after the first one ends), 16
+// CTAs per cluster, programmatic stream serialization.
 template <bool XBF16>
 static cudaError_t launch_route_cluster(const DecodeArgs &a, cudaStream_t st) {
+  const int tpc = a.n > g_cl_resident ? kClMaxTpc : 1;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(a.n * kClCtas);
+  cfg.gridDim = dim3((a.n + tpc - 1) / tpc * kClCtas);
   cfg.blockDim = dim3(kClThreads);
-  cfg.dynamicSmemBytes = cl_plan(a.sh.e + a.sh.shared_gate, a.sh.d).total;
+  cfg.dynamicSmemBytes = cl_plan(a.sh.e + a.sh.shared_gate, a.sh.d, tpc).total;
   cfg.stream = st;
   cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -1998,7 +2014,7 @@ static cudaError_t launch_route_cluster(const DecodeArgs &a, cudaStream_t st) {
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = g_pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, k_route_cl<XBF16>, a);
+  return cudaLaunchKernelEx(&cfg, k_route_cl<XBF16>, a, tpc);
 }
 
 static int gemv_smem(int fmt, int umax) { return ring_plan(fmt, 1, kStageSlots, umax).total; }
