@@ -112,11 +112,11 @@ void plan_workspace(moe_handle *h, Carve &c) {
   const moe_config &g = h->cfg;
   const int D = g.d_model, E = g.n_experts, K = g.top_k;
   const int nd = g.max_tokens < kDecodeMaxTokens ? g.max_tokens : kDecodeMaxTokens;
-  const int umax = (nd * K < E ? nd * K : E) + g.n_shared;
+  const int pmax = kDecodeMaxTokens * (K + (g.n_shared ? 1 : 0));
   const int fmax = g.n_shared && g.shared_d_ff > g.d_ff ? g.shared_d_ff : g.d_ff;
   const int tmax = fmax / kTileRows;
   DecodeWs &w = h->dws;
-  w.umax = umax;
+  w.pmax = pmax;
   w.fmax = fmax;
   w.tmax = tmax;
   // router: 256 (else 128) d_model columns per CTA; K segments of 4 (else 2) chunks
@@ -130,13 +130,11 @@ void plan_workspace(moe_handle *h, Carve &c) {
   w.route_sync = c.take<unsigned>(2);
   w.route_idx = c.take<int>(kDecodeMaxTokens * K);
   w.route_w = c.take<float>(kDecodeMaxTokens * K);
-  w.slotpos = c.take<int>(kDecodeMaxTokens * K);
   w.xrec = c.take<ActRec>(static_cast<uint64_t>(kDecodeMaxTokens) * ncd);
-  const uint64_t hrows = static_cast<uint64_t>(umax) * kDecodeMaxTokens;
-  w.gu_part = c.take<float>(static_cast<uint64_t>(umax) * tmax * w.gu_nseg * 2 * kDecodeMaxTokens * kTileRows);
-  w.o = c.take<float>(hrows * tmax * D);
-  w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * kDecodeMaxTokens);  // x token groups of a unit (at most one per token)
-  w.gu_depart = c.take<unsigned>(static_cast<uint64_t>(umax) * tmax * kDecodeMaxTokens);
+  w.gu_part = c.take<float>(static_cast<uint64_t>(pmax) * tmax * w.gu_nseg * 2 * kTileRows);
+  w.o = c.take<float>(static_cast<uint64_t>(pmax) * tmax * D);
+  w.gu_ticket = c.take<unsigned>(static_cast<uint64_t>(pmax) * tmax);
+  w.gu_depart = c.take<unsigned>(static_cast<uint64_t>(pmax) * tmax);
   w.counters = c.take<unsigned>(2);
   const uint64_t nt = static_cast<uint64_t>(g.max_tokens) * D;
   h->res[0] = c.take<float>(nt);
@@ -153,8 +151,8 @@ moe_status check_device_error(moe_handle *h, cudaStream_t st) {
   __atomic_store_n(h->err_host, 0u, __ATOMIC_RELEASE);
   // a kernel that gave up may have left arrival counters set: clear them
   const DecodeWs &w = h->dws;
-  cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.umax * w.tmax * kDecodeMaxTokens, st);
-  cudaMemsetAsync(w.gu_depart, 0, sizeof(unsigned) * w.umax * w.tmax * kDecodeMaxTokens, st);
+  cudaMemsetAsync(w.gu_ticket, 0, sizeof(unsigned) * w.pmax * w.tmax, st);
+  cudaMemsetAsync(w.gu_depart, 0, sizeof(unsigned) * w.pmax * w.tmax, st);
   cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * 2, st);
   cudaMemsetAsync(w.route_sync, 0, sizeof(unsigned) * 2, st);
   if (e & kErrTimeout) return fail(h, MOE_ERR_TIMEOUT, "a device-side bounded wait ran out");
@@ -341,7 +339,7 @@ moe_status moe_create(const moe_config *cfg, moe_handle **out) {
         goto fail_out;
       }
     }
-    cudaError_t ge = decode_grid_sizes(g.fmt, h->dws.umax, &h->dws.grid_gemv, &h->dws.min_streams);
+    cudaError_t ge = decode_grid_sizes(g.fmt, &h->dws.grid_gemv, &h->dws.min_streams);
     if (ge != cudaSuccess) {
       s = cuda_fail(h, ge, "grid sizing");
       goto fail_out;

@@ -69,7 +69,7 @@ constexpr int kGuStageChunks = 2;               // gate/up: chunks per stage
 constexpr int kDnStageChunks = 4;               // down: chunks per stage (one K segment)
 constexpr int kStageSlots = 2 * kGuStageChunks;   // (matrix, chunk) slots of a stage: 4 either way
 static_assert(kStageSlots == kDnStageChunks, "gate/up and down stages share one layout");
-constexpr int kPartStride = kDecodeMaxTokens * kTileRows;  // floats per (segment, matrix)
+constexpr int kPartStride = kTileRows;  // floats per (segment, matrix): the rows of one token
 
 // Q2 block arithmetic.  A block's value is sum_i (q_i - 1.5) m_i = (2S - 3M) / 2 with S = sum q_i m_i
 // and M = sum m_i.  The codes are taken from their words by one mask each, without the shift,
@@ -383,18 +383,12 @@ __device__ __forceinline__ int piece_run(int nseg, int units_total, int ctas) {
   return udiv_small(nseg + p - 1, p);
 }
 
-// Token groups of an active expert: each group of at most kTokGroup of its tokens is a unit of
-// its own over the whole K, so the expert's rows stream once per group (the repeats mostly from
-// L2).  Groups of one token keep every unit's arithmetic equal and the one-token GEMV's registers
-// low enough for four CTAs per SM; MOE_TOK_GROUP=2 (or 4) builds the grouped variant.
-#ifndef MOE_TOK_GROUP
-#define MOE_TOK_GROUP 1
-#endif
-constexpr int kTokGroup = MOE_TOK_GROUP;
-constexpr int kMaxTokGroups = kDecodeMaxTokens / kTokGroup;
-constexpr int kUnitTok = kTokGroup;  // tokens of one GEMV unit (at most)
-__host__ __device__ inline int tok_groups(int ntok) { return (ntok + kTokGroup - 1) / kTokGroup; }
-__host__ __device__ inline int tok_group_size(int ntok) { return ntok < kTokGroup ? ntok : kTokGroup; }
+// A GEMV unit is one (token, expert) pair of the routing -- a token's k-th choice, or its shared
+// expert -- over one 128-row tile of the expert's gate/up rows: an expert chosen by several
+// tokens streams its rows once per token (the repeats mostly from L2).  Units of one token keep
+// every unit's arithmetic equal, the one-token GEMV's registers low enough for four CTAs per SM,
+// and let every CTA find its unit from the router's selections with no shared table.
+constexpr int kUnitTok = 1;  // tokens of one GEMV unit
 
 // Split of one GEMV unit whose K has nc chunks: K segments of 4 (else 2) chunks, cut into
 // pieces of `len` segments.  Returns the packed split; `pieces` the number of pieces.
@@ -406,9 +400,6 @@ __device__ __forceinline__ int unit_split(int nc, int units_total, int min_strea
   return len | (pieces << 8) | (seg << 16) | (nseg << 20);
 }
 
-constexpr int kTabHead = 4;    // ints before the first row of the task table
-constexpr int kTabInts = 16;   // ints per active expert
-constexpr int kMaxActive = kDecodeMaxTokens * kMaxTopK + 1;
 
 template <bool XBF16>
 __device__ __forceinline__ void load_x8(const void *x, int64_t off, float (&v)[8]) {
@@ -894,130 +885,6 @@ static bool route_cluster_fits(const Shape &sh) {
 }
 
 // ------------------------------------------------------------------------------------------
-// routing tables, built by every GEMV CTA in its own shared memory
-// ------------------------------------------------------------------------------------------
-// Scratch (the ring's stage area, unused until the tables exist): tokmask [E] (bit t = token t
-// chose the expert), bitmap and wpre [kMaxExperts / 32] (active experts; active experts before
-// word w), s_idx [8][kMaxTopK], s_cnt [2][kMaxActive], s_misc [4], then one logit row per
-// top-k warp when there are more than 1,024 experts.
-__host__ __device__ constexpr int table_scratch_bytes() {
-  return kMaxExperts * 4 + 2 * (kMaxExperts / 32) * 4 + kDecodeMaxTokens * kMaxTopK * 4 + 2 * kMaxActive * 4 + 16;
-}
-
-// The active-expert rows from the router's selections (u = 0: the shared expert; routed
-// experts follow in ascending id), the K split and the first task of each active expert.  Every
-// thread of the CTA calls it; wr: also write the routing outputs (one CTA does).
-__device__ void build_tables(const DecodeArgs &a, unsigned char *scratch, int *tb, bool wr) {
-  constexpr int kThreads = kGemvThreads;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int D = a.sh.d, E = a.sh.e, K = a.sh.k, n = a.n;
-  uint32_t *tokmask = reinterpret_cast<uint32_t *>(scratch);
-  uint32_t *bitmap = tokmask + E;
-  int *wpre = reinterpret_cast<int *>(bitmap + kMaxExperts / 32);
-  int *s_idx = wpre + kMaxExperts / 32;
-  int *s_cnt = s_idx + kDecodeMaxTokens * kMaxTopK;
-  int *s_misc = s_cnt + 2 * kMaxActive;  // units of gate/up, units of down, routed active
-  const int nw = (E + 31) / 32;
-  for (int i = tid; i < E; i += kThreads) tokmask[i] = 0u;
-  for (int i = tid; i < nw; i += kThreads) bitmap[i] = 0u;
-  if (tid < 4) s_misc[tid] = 0;
-  for (int p = tid; p < n * K; p += kThreads) {  // the router's selections
-    int ex = __ldcg(a.ws.sel + p);
-    if (ex < 0 || ex >= E) {
-      flag_error(a.err, kErrBadIndex);
-      ex = 0;
-    }
-    s_idx[p] = ex;
-  }
-  __syncthreads();
-  for (int p = tid; p < n * K; p += kThreads) {
-    const int ex = s_idx[p];
-    atomicOr(tokmask + ex, 1u << (p / K));
-    atomicOr(bitmap + (ex >> 5), 1u << (ex & 31));
-  }
-  __syncthreads();
-  if (warp == 0) {  // active experts before each bitmap word
-    int run = 0;
-    for (int w0 = 0; w0 < nw; w0 += 32) {
-      const int w = w0 + lane;
-      const int c = w < nw ? __popc(bitmap[w]) : 0;
-      int inc = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += v;
-      }
-      if (w < nw) wpre[w] = run + inc - c;
-      run += __shfl_sync(0xffffffffu, inc, 31);
-    }
-    if (lane == 0) s_misc[2] = run;
-  }
-  __syncthreads();
-  // rows written by the thread of each expert's first token, and the combine's slots
-  const int ns = a.sh.n_shared;
-  const int na = ns + s_misc[2];
-  auto rank_of = [&](int e) { return wpre[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u)); };
-  int ug = 0;
-  for (int p = tid; p < n * K + ns; p += kThreads) {
-    const bool shared = p == n * K;
-    const int t = shared ? 0 : p / K, ex = shared ? E : s_idx[p];
-    uint32_t m = shared ? (1u << n) - 1u : tokmask[ex];
-    const int u = shared ? 0 : ns + rank_of(ex);
-    if (wr && !shared) a.ws.slotpos[p] = u * kDecodeMaxTokens + __popc(m & ((1u << t) - 1u));
-    if (!shared && (m & ((1u << t) - 1u))) continue;  // not the expert's first token
-    const int nt = __popc(m), ng = tok_groups(nt);
-    const int F = shared ? a.L.shared.f : a.L.routed.f;
-    int *row = tb + kTabHead + u * kTabInts;
-    row[0] = ex;
-    row[1] = nt;
-    row[14] = ng;
-    int c = 0;
-    while (m) {
-      row[2 + c++] = __ffs(m) - 1;
-      m &= m - 1u;
-    }
-    s_cnt[kMaxActive + u] = ng;
-    ug += (F / kTileRows) * ng;
-  }
-  if (ug) atomicAdd(&s_misc[0], ug);
-  if (wr && a.out_counts)
-    for (int i = tid; i < E; i += kThreads) a.out_counts[i] = __popc(tokmask[i]);
-  __syncthreads();
-  if (warp == 0) {  // K split, task counts and first task of each active expert (prefix over u)
-    // the split depends on the unit total and d_model only: one split for every unit
-    int pg;
-    const int sg = unit_split(D / kChunk, s_misc[0], a.ws.min_streams, pg);
-    const int tgr = (a.L.routed.f / kTileRows) * pg, tgs = ns ? (a.L.shared.f / kTileRows) * pg : 0;
-    int run0 = 0;
-    for (int u0 = 0; u0 < na; u0 += 32) {
-      const int u = u0 + lane;
-      int c0v = 0;
-      if (u < na) {
-        const bool sh = ns && u == 0;
-        const int ng = s_cnt[kMaxActive + u];
-        tb[kTabHead + u * kTabInts + 11] = sg;
-        c0v = (sh ? tgs : tgr) * ng;
-      }
-      int i0 = c0v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v0 = __shfl_up_sync(0xffffffffu, i0, o);
-        if (lane >= o) i0 += v0;
-      }
-      if (u < na) tb[kTabHead + u * kTabInts + 10] = run0 + i0 - c0v;
-      run0 += __shfl_sync(0xffffffffu, i0, 31);
-    }
-    if (lane == 0) {
-      tb[0] = na;
-      tb[1] = run0;
-      tb[2] = 0;
-      tb[3] = 0;
-    }
-  }
-  __syncthreads();
-}
-
-// ------------------------------------------------------------------------------------------
 // GEMV arithmetic of one ring stage
 // ------------------------------------------------------------------------------------------
 // replicate the 256 x 4 int8 grid 32 times so that lane l reads copy l (bank l): conflict-free
@@ -1108,26 +975,25 @@ __host__ __device__ inline int align128(int v) { return (v + 127) & ~127; }
 // A stage holds, for up to CMAX chunks: plane A [NR][CMAX][128][16 B], plane S [NR][CMAX][128]
 // [4 B], plane G [NR][CMAX][128][8 B] (CB35), then the records [8 tokens][CMAX][144 B].
 struct RingPlan {
-  int table, hrec, stage0, a, s, g, rec, stage, tab, total;
+  int hrec, stage0, a, s, g, rec, stage, tab, total;
 };
 
 // Per-stage description written by the producer before it arms the stage's barrier.
 struct StageInfo {
   int task;    // -1: no more work
-  int u;       // active expert
+  int u;       // the unit's (token, expert) pair: its slot in the outputs
+  int e;       // expert (E: the shared expert)
   int mt;      // 128-row tile
   int seg;     // K segment of the stage
   int ntok;
   int nch;     // chunks in the stage
-  int flags;   // k* bits | pieces of the unit << 8 | K segments of the unit << 16 |
-               // first token slot of the unit's token group << 24
+  int flags;   // k* bits | pieces of the unit << 8 | K segments of the unit << 16
   int c0;      // first chunk of the stage
 };
 constexpr int kPieceStart = 1, kSegStart = 2, kSegEnd = 4, kPieceEnd = 8;
 constexpr int kDnStage = 16, kDnPair = 32;  // a down stage; of two output tiles
 __device__ __forceinline__ int info_pieces(int flags) { return (flags >> 8) & 0xFF; }
 __device__ __forceinline__ int info_nseg(int flags) { return (flags >> 16) & 0xFF; }
-__device__ __forceinline__ int info_tok0(int flags) { return flags >> 24; }
 
 struct RingHdr {
   uint64_t full[kRing];
@@ -1140,10 +1006,9 @@ struct RingHdr {
   float tot[2][kUnitTok][kTileRows];  // running unit sums of an unsplit unit (thread = row)
 };
 
-__host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax, int umax) {
+__host__ __device__ inline RingPlan ring_plan(int fmt, int nr, int cmax) {
   RingPlan p;
-  p.table = align128(static_cast<int>(sizeof(RingHdr)));
-  int off = p.table + align128((kTabHead + kTabInts * umax) * 4);
+  int off = align128(static_cast<int>(sizeof(RingHdr)));
   p.hrec = off;  // h records of the current gate/up unit: [token][2 chunks]
   off += align128(kUnitTok * (kTileRows / kChunk) * static_cast<int>(sizeof(ActRec)));
   p.stage0 = off;
@@ -1370,17 +1235,6 @@ __device__ __forceinline__ void cons_fail(const DecodeArgs &a, RingHdr *H) {
 }
 
 
-// largest u with first-task(u) <= r (first tasks increase with u, first-task(0) = 0)
-__device__ __forceinline__ int find_expert(const int *tb, int na, int r) {
-  int lo = 0, hi = na - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (tb[kTabHead + mid * kTabInts + 10] <= r) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
 // Plane pl (A, S, G) of matrix slot m of a stage: nch chunk slots of 128 rows from slot0 on.
 template <int FMT>
 __device__ __forceinline__ void copy_plane(unsigned char *st, const RingPlan &P, int m, int pl, const ExpertGroup &G,
@@ -1396,10 +1250,13 @@ __device__ __forceinline__ void copy_plane(unsigned char *st, const RingPlan &P,
     bulk_g2s_hint(st + P.g + m * cmax * kTileRows * 8, G.g + mat * G.g_mat + slot0, nch * kTileRows * 8, bar, pol);
 }
 
-// The producer warp: one work queue of pieces (active expert u, gate/up tile j, token group,
-// run of K segments) -> bulk copies into the ring.  A piece is its gate/up stages (the gate and
-// up rows of tile j, two chunks of each per stage, with the activation records of the unit's
-// tokens), then its down stages: the piece's share of the output tiles over K-slice j (the 128
+// The producer warp: one work queue of pieces (pair u, gate/up tile j, run of K segments) ->
+// bulk copies into the ring.  Tasks are numbered from the routing alone: first the shared
+// expert's pairs (u = token t; its rows were prefetched into L2 before the router finished),
+// then the routed pairs (u = n + t K + k for the k-th choice of token t, its expert read from the
+// router's selections), each pair's tiles j, each tile's pieces.  A piece is its gate/up stages
+// (the gate and up rows of tile j, two chunks of each per stage, with the token's activation
+// records), then its down stages: the piece's share of the output tiles over K-slice j (the 128
 // rows of h that tile j makes), two tiles of two chunks per stage, weights only -- the consumers
 // write h into shared memory themselves.  No copy waits for another CTA, and every stage the
 // warp arms is waited for (bounded) before it leaves, so no copy is in flight when the CTA
@@ -1411,12 +1268,16 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
   constexpr int kPlanes = has_plane_g(FMT) ? 3 : 2;
   constexpr int kPB = plane_bytes(FMT);
   const int lane = threadIdx.x & 31;
-  const int D = a.sh.d, E = a.sh.e, TD = D / kTileRows, nc = D / kChunk;
-  const int *tb = reinterpret_cast<const int *>(smem + P.table);
+  const int D = a.sh.d, E = a.sh.e, K = a.sh.k, n = a.n, TD = D / kTileRows, nc = D / kChunk;
+  const int ns = a.sh.n_shared ? 1 : 0;
+  const int tjr = a.L.routed.f / kTileRows, tjs = ns ? a.L.shared.f / kTileRows : 0;
+  // one split for every unit: it depends on the unit count and d_model only
+  int pieces;
+  const int pk = unit_split(nc, ns * n * tjs + n * K * tjr, a.ws.min_streams, pieces);
+  const int len = pk & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
+  const int shared_tasks = ns * n * tjs * pieces, n_tasks = shared_tasks + n * K * tjr * pieces;
   unsigned *ctr = a.ws.counters;
   int task = first_task;
-  const int na = tb[0], n_tasks = tb[1];
-  fence_proxy_async_smem();  // the tables' scratch (generic stores) becomes ring stages (bulk copies)
   bool ok = true;
   const uint64_t pol = l2_evict_first_policy();
   int slot = 0;
@@ -1427,18 +1288,21 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
   while (ok && task < n_tasks) {
     int nxt = 0;
     if (lane == 0) nxt = static_cast<int>(atomicAdd(ctr, 1u));  // fetched while this piece is issued
-    const int u = find_expert(tb, na, task);
-    const int *row = tb + kTabHead + u * kTabInts;
-    const int pk = row[11], ng = row[14];
-    const int len = pk & 0xFF, pieces = (pk >> 8) & 0xFF, seg = (pk >> 16) & 0xF, nseg = pk >> 20;
-    const int r = task - row[10];
-    const int j = r / (ng * pieces);
-    const int q = r - j * ng * pieces;
-    const int grp = q / pieces, piece = q - grp * pieces;
-    const int e = row[0];
-    const int gsz = tok_group_size(row[1]), tok0 = grp * gsz;
-    const int ntok = min(gsz, row[1] - tok0);  // tokens of this unit: slots tok0 .. tok0 + ntok - 1
-    const bool shared = a.sh.n_shared && e == E;
+    const bool shared = task < shared_tasks;
+    const int tpp = (shared ? tjs : tjr) * pieces;           // tasks per pair
+    const int rt = shared ? task : task - shared_tasks;
+    const int q = rt / tpp, rj = rt - q * tpp;               // pair q of its kind
+    const int j = rj / pieces, piece = rj - j * pieces;
+    const int u = shared ? q : ns * n + q, t = shared ? q : q / K;
+    int e = E;
+    if (!shared) {
+      e = __ldcg(a.ws.sel + q);  // the same address in every lane
+      if (e < 0 || e >= E) {
+        if (lane == 0) flag_error(a.err, kErrBadIndex);
+        e = 0;
+      }
+    }
+    constexpr int ntok = kUnitTok;
     const ExpertGroup &G = shared ? a.L.shared : a.L.routed;
     const int64_t mat0 = static_cast<int64_t>(shared ? 0 : e) * 3;
     const int ncd = G.f / kChunk;
@@ -1456,29 +1320,28 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
           StageInfo &in = H->info[slot];
           in.task = task;
           in.u = u;
+          in.e = e;
           in.mt = j;
           in.seg = c0 / seg;
           in.ntok = ntok;
           in.nch = nch;
           in.flags = (c0 == cbeg ? kPieceStart : 0) | (c0 % seg == 0 ? kSegStart : 0) |
                      ((c0 + nch) % seg == 0 ? kSegEnd : 0) | (c0 + nch == cend ? kPieceEnd : 0) | (pieces << 8) |
-                     (nseg << 16) | (tok0 << 24);
+                     (nseg << 16);
           in.c0 = c0;
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(&H->full[slot], 2 * nch * kTileRows * kPB + ntok * rbytes);
         }
         __syncwarp();
-        // copy l of the stage, issued by lane l: 2 x (A, S[, G]) weight planes, then one run of
-        // records per token (chunk slot of matrix m, chunk c: m * 2 + c)
+        // copy l of the stage, issued by lane l: 2 x (A, S[, G]) weight planes, then the run of
+        // the token's records (chunk slot of matrix m, chunk c: m * 2 + c)
         if (lane < 2 * kPlanes) {
           const int m = lane / kPlanes;
           copy_plane<FMT>(st, P, m, lane - m * kPlanes, G, mat0 + m, (static_cast<int64_t>(j) * nc + c0) * kTileRows,
                           nch, pol, &H->full[slot]);
         }
-        const int i = lane - 2 * kPlanes;
-        if (i >= 0 && i < ntok)
-          bulk_g2s(st + P.rec + i * kGuStageChunks * static_cast<int>(sizeof(ActRec)),
-                   a.ws.xrec + static_cast<int64_t>(row[2 + tok0 + i]) * nc + c0, rbytes, &H->full[slot]);
+        if (lane == 2 * kPlanes)
+          bulk_g2s(st + P.rec, a.ws.xrec + static_cast<int64_t>(t) * nc + c0, rbytes, &H->full[slot]);
       } else {
         // output tiles t0 (and t0 + 1) of the down matrix over K-slice j = chunks 2j, 2j + 1
         const int t0 = d0 + 2 * (si - n_gu), nt = min(2, d1 - t0);
@@ -1486,11 +1349,12 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
           StageInfo &in = H->info[slot];
           in.task = task;
           in.u = u;
+          in.e = e;
           in.mt = t0;
           in.seg = j;
           in.ntok = ntok;
           in.nch = 2;
-          in.flags = kDnStage | (nt == 2 ? kDnPair : 0) | (pieces << 8) | (tok0 << 24);
+          in.flags = kDnStage | (nt == 2 ? kDnPair : 0) | (pieces << 8);
           in.c0 = 0;
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(&H->full[slot], nt * 2 * kTileRows * kPB);
@@ -1600,13 +1464,6 @@ __device__ __forceinline__ bool unit_meet(const DecodeArgs &a, RingHdr *H, ConsS
   return cons_sync(H, cs.cph, a.spin_limit) && H->flag[fb];
 }
 
-// expert id of active expert u (E: the shared expert), from the CTA's task table
-__device__ __forceinline__ int unit_expert(const RingHdr *H, int u) {
-  const int *tb = reinterpret_cast<const int *>(reinterpret_cast<const unsigned char *>(H) +
-                                                align128(static_cast<int>(sizeof(RingHdr))));
-  return tb[kTabHead + u * kTabInts];
-}
-
 // End of a gate/up piece: the unit's full sums (this piece's, or every piece's partials), the
 // SwiGLU, and h of each token quantised over the tile's 128 rows into the CTA's shared h
 // records, which the piece's down stages read.
@@ -1615,7 +1472,7 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
                                           ActRec *hrec) {
   const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
   const int u = in.u, mt = in.mt, ntok = in.ntok, pieces = info_pieces(in.flags);
-  const int nseg = info_nseg(in.flags), tok0 = info_tok0(in.flags);
+  const int nseg = info_nseg(in.flags);
   float tot[2][kUnitTok];
 #pragma unroll
   for (int t = 0; t < kUnitTok; ++t)
@@ -1624,11 +1481,9 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
       tot[1][t] = H->tot[1][t][r];
     }
   if (pieces > 1) {
-    const int64_t ti = (static_cast<int64_t>(u) * a.ws.tmax + mt) * kMaxTokGroups + tok0 / kTokGroup;
+    const int64_t ti = static_cast<int64_t>(u) * a.ws.tmax + mt;
     if (!unit_meet(a, H, cs, a.ws.gu_ticket + ti, static_cast<unsigned>(pieces))) return false;
-    sum_segments<2>(a.ws.gu_part + static_cast<int64_t>(u * a.ws.tmax + mt) * a.ws.gu_nseg * 2 * kPartStride +
-                        tok0 * kTileRows, nseg,
-                    ntok, tot);
+    sum_segments<2>(a.ws.gu_part + ti * a.ws.gu_nseg * 2 * kPartStride, nseg, ntok, tot);
     if (!cons_sync(H, cs.cph, a.spin_limit)) return false;  // every consumer's partial loads are done
     if (r == 0 && atomicAdd(a.ws.gu_depart + ti, 1u) == static_cast<unsigned>(pieces - 1)) {
       a.ws.gu_ticket[ti] = 0u;
@@ -1636,7 +1491,7 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
     }
   }
   if (FMT == MOE_FMT_NVFP4_16) {  // the gate and up matrices' tensor scales
-    const int ex = unit_expert(H, u);
+    const int ex = in.e;
     const ExpertGroup &Gp = ex == a.sh.e ? a.L.shared : a.L.routed;
     const int eidx = ex == a.sh.e ? 0 : ex;
     const float tg = Gp.ts[eidx * 3], tu = Gp.ts[eidx * 3 + 1];
@@ -1685,19 +1540,19 @@ __device__ __forceinline__ bool gu_finish(const DecodeArgs &a, RingHdr *H, ConsS
   return cons_sync(H, cs.cph, a.spin_limit);  // h complete before any down stage reads it
 }
 
-// A down stage's outputs: o of output tiles mt (and mt + 1) over K-slice j, row r, per token.
+// A down stage's outputs: o of output tiles mt (and mt + 1) over K-slice j, row r, of the unit's
+// pair (its slot in o).
 template <int FMT>
-__device__ __forceinline__ void dn_store(const DecodeArgs &a, const RingHdr *H, const StageInfo &in,
-                                         const float (&acc)[2][kUnitTok]) {
+__device__ __forceinline__ void dn_store(const DecodeArgs &a, const StageInfo &in, const float (&acc)[2][kUnitTok]) {
   const int r = threadIdx.x, D = a.sh.d;
-  const int nt = (in.flags & kDnPair) ? 2 : 1, tok0 = info_tok0(in.flags);
+  const int nt = (in.flags & kDnPair) ? 2 : 1;
   float td = 1.f;
   if (FMT == MOE_FMT_NVFP4_16) {  // the down matrix's tensor scale
-    const int ex = unit_expert(H, in.u);
+    const int ex = in.e;
     td = (ex == a.sh.e ? a.L.shared : a.L.routed).ts[(ex == a.sh.e ? 0 : ex) * 3 + 2];
   }
-  float *o = a.ws.o + (static_cast<int64_t>(in.u) * kDecodeMaxTokens + tok0) * a.ws.tmax * D +
-             static_cast<int64_t>(in.seg) * D + in.mt * kTileRows + r;
+  float *o = a.ws.o + static_cast<int64_t>(in.u) * a.ws.tmax * D + static_cast<int64_t>(in.seg) * D +
+             in.mt * kTileRows + r;
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -1746,9 +1601,9 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
         gemv_dispatch<FMT, 1, kGuStageChunks>(in.ntok, st, P, in.nch, smem_u32(tab), hrec_s, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&H->empty[slot]);
-      dn_store<FMT>(a, H, in, acc);
+      dn_store<FMT>(a, in, acc);
     } else {
-      const int pieces = info_pieces(in.flags), tok0 = info_tok0(in.flags);
+      const int pieces = info_pieces(in.flags);
       if ((in.flags & kPieceStart) && pieces == 1) {
 #pragma unroll
         for (int m = 0; m < 2; ++m)
@@ -1766,14 +1621,14 @@ __device__ __forceinline__ void consumer(const DecodeArgs &a, unsigned char *sme
       if (lane == 0) mbar_arrive(&H->empty[slot]);
       if (in.flags & kSegEnd) {
         if (pieces > 1) {
-          // segment sum of a split unit -> partial buffer [segment][matrix][token][row]
+          // segment sum of a split unit -> partial buffer [segment][matrix][row]
           float *part = a.ws.gu_part +
                         (static_cast<int64_t>(in.u * a.ws.tmax + in.mt) * a.ws.gu_nseg + in.seg) * 2 * kPartStride;
 #pragma unroll
           for (int m = 0; m < 2; ++m)
 #pragma unroll
             for (int t = 0; t < kUnitTok; ++t)
-              if (t < in.ntok) part[m * kPartStride + (tok0 + t) * kTileRows + r] = seg[m][t];
+              if (t < in.ntok) part[m * kPartStride + t * kTileRows + r] = seg[m][t];
         } else {
 #pragma unroll
           for (int m = 0; m < 2; ++m)
@@ -1807,7 +1662,7 @@ __device__ __forceinline__ void prefetch_share(const void *base, int64_t bytes, 
 template <int FMT>
 __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const RingPlan P = ring_plan(FMT, 1, kStageSlots, a.ws.umax);
+  const RingPlan P = ring_plan(FMT, 1, kStageSlots);
   RingHdr *H = reinterpret_cast<RingHdr *>(smem);
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -1825,11 +1680,11 @@ __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(Deco
     prefetch_share(G.s, 3 * G.s_mat * 4, blockIdx.x, gridDim.x);
     if (G.g) prefetch_share(G.g, 3 * G.g_mat * 8, blockIdx.x, gridDim.x);
   }
-  griddep_wait();  // the router kernel's logits and records
+  __syncthreads();  // the barriers' initialisation precedes every use
+  griddep_wait();   // the router kernel's selections and records
   if (threadIdx.x == 0) griddep_launch();
   int first = 0;
-  if (threadIdx.x == kTileRows) first = static_cast<int>(atomicAdd(a.ws.counters, 1u));  // in flight meanwhile
-  build_tables(a, smem + P.stage0, reinterpret_cast<int *>(smem + P.table), blockIdx.x == 0);
+  if (threadIdx.x == kTileRows) first = static_cast<int>(atomicAdd(a.ws.counters, 1u));
   if (threadIdx.x >= kTileRows) {
     producer<FMT>(a, smem, P, H, __shfl_sync(0xffffffffu, first, 0));
   } else {
@@ -1838,34 +1693,42 @@ __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(Deco
 }
 
 // ------------------------------------------------------------------------------------------
-// combine: y[t] = sum_j w_tj o[slot(t, j)] + o_shared[t] (+ x[t]), slots in descending-logit
-// order; each expert output o is the sum of its K-slice outputs in slice order.  CTA = (token,
-// 64 columns): first every thread sums the slices of some (slot, column) pairs into shared
-// memory (all slices of a pair loaded at once), then one thread per column adds the slots.
+// combine: y[t] = sum_j w_tj o[n + t K + j] + o[t] (+ x[t]) (o[t]: the shared expert's output
+// for token t), the choices j in descending-logit order; each expert output o is the sum of its
+// K-slice outputs in slice order.  CTA = (token, 64 columns): first every thread sums the slices
+// of some (choice, column) pairs into shared memory (all slices of a pair loaded at once), then
+// one thread per column adds the choices.  CTA 0 also writes the optional per-expert counts.
 // ------------------------------------------------------------------------------------------
 constexpr int kCombineCols = 64;       // d_model is a multiple of 128
 constexpr int kCombineThreads = 256;
 constexpr int kMaxSlices = 8;          // K-slices of a slot loaded together (more: one at a time)
 __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
-  __shared__ int s_pos[kMaxTopK];
   __shared__ float s_w[kMaxTopK];
+  __shared__ int s_sel[kDecodeMaxTokens * kMaxTopK];
   __shared__ float s_o[(kMaxTopK + 1) * kCombineCols];  // [slot (K: the shared expert)][column]
   const int D = a.sh.d, K = a.sh.k, tid = threadIdx.x;
   const int cpt = D / kCombineCols;  // CTAs per token
   const int t = blockIdx.x / cpt, d0 = (blockIdx.x - t * cpt) * kCombineCols;
   griddep_wait();
   griddep_launch();
-  if (tid < K) {
-    s_pos[tid] = __ldcg(a.ws.slotpos + t * K + tid);
-    s_w[tid] = __ldcg(a.ws.route_w + t * K + tid);
+  if (tid < K) s_w[tid] = __ldcg(a.ws.route_w + t * K + tid);
+  if (blockIdx.x == 0 && a.out_counts) {  // tokens per expert, from the router's selections
+    const int nk = a.n * K;
+    for (int p = tid; p < nk; p += kCombineThreads) s_sel[p] = __ldcg(a.ws.sel + p);
+    __syncthreads();
+    for (int e = tid; e < a.sh.e; e += kCombineThreads) {
+      int c = 0;
+      for (int p = 0; p < nk; ++p) c += s_sel[p] == e ? 1 : 0;
+      a.out_counts[e] = c;
+    }
   }
   __syncthreads();
   const int TM = a.ws.tmax, ns = a.sh.n_shared ? 1 : 0;
   const int js = ns ? a.L.shared.f / kTileRows : 0, jr = a.L.routed.f / kTileRows;
   for (int it = tid; it < (K + ns) * kCombineCols; it += kCombineThreads) {
     const int j = it / kCombineCols, c = it - j * kCombineCols;
-    const bool sh = j == K;  // u = 0 serves token t in slot t
-    const float *src = a.ws.o + static_cast<int64_t>(sh ? t : s_pos[j]) * TM * D + d0 + c;
+    const bool sh = j == K;
+    const float *src = a.ws.o + static_cast<int64_t>(sh ? t : ns * a.n + t * K + j) * TM * D + d0 + c;
     const int nq = sh ? js : jr;
     float v[kMaxSlices];
 #pragma unroll
@@ -2017,20 +1880,18 @@ static cudaError_t launch_route_cluster(const DecodeArgs &a, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, k_route_cl<XBF16>, a, tpc);
 }
 
-static int gemv_smem(int fmt, int umax) { return ring_plan(fmt, 1, kStageSlots, umax).total; }
+static int gemv_smem(int fmt) { return ring_plan(fmt, 1, kStageSlots).total; }
 
 
 // Persistent grid: SMs x resident CTAs of the GEMV kernel; min_streams = the grid (see piece_run).
-cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_streams) {
+cudaError_t decode_grid_sizes(int fmt, int *grid_gemv, int *min_streams) {
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   // the routing scratch lives in the ring
-  const RingPlan P = ring_plan(fmt, 1, kStageSlots, umax);
-  if (ring_depth(fmt) * P.stage < table_scratch_bytes()) return cudaErrorInvalidConfiguration;
   int occ = 0;
-  const int sm = gemv_smem(fmt, umax);
+  const int sm = gemv_smem(fmt);
   e = fmt == MOE_FMT_Q2_32
           ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<MOE_FMT_Q2_32>, kGemvThreads, sm)
       : fmt == MOE_FMT_CB35_32
@@ -2063,7 +1924,7 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
   }
   // 2. top-k + tables (per CTA), gate/up + SwiGLU, then down (one persistent kernel)
   {
-    const int sm = gemv_smem(a.sh.fmt, a.ws.umax);
+    const int sm = gemv_smem(a.sh.fmt);
     rec(a, kProfGateUp, 0, st);
     err = a.sh.fmt == MOE_FMT_Q2_32     ? launch_pdl(k_gemv<MOE_FMT_Q2_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a)
           : a.sh.fmt == MOE_FMT_CB35_32 ? launch_pdl(k_gemv<MOE_FMT_CB35_32>, a.ws.grid_gemv, kGemvThreads, sm, st, a)

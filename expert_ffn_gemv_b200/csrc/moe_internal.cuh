@@ -107,18 +107,15 @@ struct DecodeWs {
   unsigned *route_sync; // [2] router CTAs done, top-k CTAs done
   int *route_idx;       // [8][k]
   float *route_w;       // [8][k]
-  int *slotpos;         // [8][k]: u * 8 + i (i = position of the token in expert u's list)
-  // (The GEMV kernel's task table lives in each CTA's shared memory: a header [n_active,
-  // tasks, 0, 0] and one 16-int row per active expert u: [expert (E = shared), ntok, tokens
-  // 0..7, first task, split, 0, 0, token groups, 0]; a split packs run length | pieces << 8 |
-  // chunks per segment << 16 | segments << 20.)
+  // Pairs (slots of the GEMV outputs): token t's shared expert is pair t, its k-th routed choice
+  // pair n_shared * n + t * k_top + k (n: tokens of the call); at most pmax = 8 (k + n_shared).
   ActRec *xrec;         // [8][D/64]
-  float *gu_part;       // [umax][tmax][gu_nseg][2][8][128] gate/up segment sums
-  float *o;             // [umax * 8][tmax][D] expert outputs per K-slice of the down matrix (unweighted)
-  unsigned *gu_ticket;  // [umax][tmax][8] (token groups): pieces of a split unit that stored their partials
-  unsigned *gu_depart;  // [umax][tmax][8]: pieces of a split unit that have read every partial
+  float *gu_part;       // [pmax][tmax][gu_nseg][2][128] gate/up segment sums of split units
+  float *o;             // [pmax][tmax][D] expert outputs per K-slice of the down matrix (unweighted)
+  unsigned *gu_ticket;  // [pmax][tmax]: pieces of a split unit that stored their partials
+  unsigned *gu_depart;  // [pmax][tmax]: pieces of a split unit that have read every partial
   unsigned *counters;   // [2] work queue of the GEMV kernel
-  int umax;
+  int pmax;
   int tmax;             // max(F, F_shared) / 128
   int fmax;
   int gu_seg;           // gate/up: chunks per K segment (2 or 4)
@@ -313,7 +310,7 @@ constexpr int kProfDown = 2;      // the combine kernel or the down GEMM + combi
 constexpr int kProfKinds = 3;
 
 cudaError_t configure_decode_kernels();
-cudaError_t decode_grid_sizes(int fmt, int umax, int *grid_gemv, int *min_streams);
+cudaError_t decode_grid_sizes(int fmt, int *grid_gemv, int *min_streams);
 cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_wait_test(unsigned *never_set, uint32_t *err, uint64_t spin_limit, cudaStream_t st);
 
