@@ -1286,8 +1286,8 @@ __device__ __forceinline__ void producer(const DecodeArgs &a, unsigned char *sme
 #pragma unroll
   for (int s = 0; s < RING; ++s) last_round[s] = -1;
   while (ok && task < n_tasks) {
-    int nxt = 0;
-    if (lane == 0) nxt = static_cast<int>(atomicAdd(ctr, 1u));  // fetched while this piece is issued
+    int nxt = 0;  // tasks after the first of every CTA come from the counter, fetched while this piece is issued
+    if (lane == 0) nxt = static_cast<int>(gridDim.x + atomicAdd(ctr, 1u));
     const bool shared = task < shared_tasks;
     const int tpp = (shared ? tjs : tjr) * pieces;           // tasks per pair
     const int rt = shared ? task : task - shared_tasks;
@@ -1683,10 +1683,10 @@ __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(Deco
   __syncthreads();  // the barriers' initialisation precedes every use
   griddep_wait();   // the router kernel's selections and records
   if (threadIdx.x == 0) griddep_launch();
-  int first = 0;
-  if (threadIdx.x == kTileRows) first = static_cast<int>(atomicAdd(a.ws.counters, 1u));
+  // CTA i starts with task i (the grid is every resident CTA, so each split unit's pieces all
+  // run at once); later tasks come from the work queue
   if (threadIdx.x >= kTileRows) {
-    producer<FMT>(a, smem, P, H, __shfl_sync(0xffffffffu, first, 0));
+    producer<FMT>(a, smem, P, H, static_cast<int>(blockIdx.x));
   } else {
     consumer<FMT>(a, smem, P, H);
   }
