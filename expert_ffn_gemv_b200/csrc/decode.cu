@@ -575,28 +575,38 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(DecodeArgs a) {
 // ------------------------------------------------------------------------------------------
 // Router as clusters of 16 CTAs, each serving tpc tokens (1, or 2 when the tokens outnumber the
 // clusters the device holds at once; bf16 router rows; at most 48 rows per CTA and d_model up
-// to 2,048): every CTA bulk-copies its rows of the router into shared memory before it waits
-// for the previous kernel, computes their logits for each of its cluster's tokens (fp32 sums)
-// and stores those of token slot s into CTA s's shared memory over the cluster (distributed
-// shared memory); after one cluster barrier CTA s takes token s's top-k and fp32 softmax.  No
-// logit crosses global memory and no CTA waits on a global counter.  The same CTAs quantise
-// the tokens' inputs into the activation records.
+// to 2,048, a multiple of 256): every CTA bulk-copies its rows of the router into shared memory
+// before it waits for the previous kernel, computes their logits for its cluster's tokens on
+// the tensor cores (bf16 rows x the bf16 hi and lo parts of x, fp32 sums) and stores those of
+// token slot s into CTA s's shared memory over the cluster (distributed shared memory); after
+// one cluster barrier CTA s takes token s's top-k and fp32 softmax.  No logit crosses global
+// memory and no CTA waits on a global counter.  The same CTAs quantise the tokens' inputs into
+// the activation records.
 // ------------------------------------------------------------------------------------------
-constexpr int kClCtas = 16, kClThreads = 512, kClWarps = kClThreads / 32, kClRowsPerWarp = 3;
+constexpr int kClCtas = 16, kClThreads = 512, kClWarps = kClThreads / 32;
 constexpr int kClMaxD = 2048, kClMaxExperts = 1024;
 constexpr int kClMaxTpc = 2;  // tokens per cluster (at most)
 
 struct ClPlan {
-  int R;                           // router rows per CTA
-  int w, x, lg, raw, keys, tk, total;  // byte offsets: rows, x (fp32, per token slot), logits, raw logits, keys, top-k scratch
+  int R;       // router rows per CTA
+  int rs;      // bytes per row of the rows and of the bf16 x parts: d_model x 2 + 16
+  // byte offsets: rows (bf16), x (fp32, per token slot), x parts (bf16: tpc hi rows, then tpc
+  // lo rows), biases, the warps' partial logits [16 warps][48 rows][2 slots], logits, raw
+  // logits, keys, top-k scratch
+  int w, x, xb, bias, red, lg, raw, keys, tk, total;
 };
+constexpr int kClRedRows = 48;  // rows of the three 16-row MMA tiles
 __host__ __device__ inline ClPlan cl_plan(int ER, int D, int tpc) {
   ClPlan p;
   p.R = (ER + kClCtas - 1) / kClCtas;
+  p.rs = D * 2 + 16;  // 16 bytes of padding: the 8 rows of a fragment load fall in distinct banks
   const int er = p.R * kClCtas;
   p.w = 128;  // [0, 128): the rows' mbarrier
-  p.x = p.w + ((p.R * D * 2 + 127) & ~127);
-  p.lg = p.x + tpc * D * 4;
+  p.x = p.w + ((p.R * p.rs + 127) & ~127);
+  p.xb = p.x + tpc * D * 4;
+  p.bias = p.xb + ((2 * tpc * p.rs + 127) & ~127);
+  p.red = p.bias + ((p.R * 4 + 127) & ~127);
+  p.lg = p.red + kClWarps * kClRedRows * kClMaxTpc * 4;
   p.raw = p.lg + er * 4;
   p.keys = p.raw + er * 4;
   p.tk = p.keys + er * 4;
@@ -618,6 +628,17 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
+// D += A B for one m16n8k16 tile: A 16 x 16 bf16 (row-major fragments a0..a3), B 16 x 8 bf16
+// (column fragments b0, b1), D 16 x 8 fp32 (d[0..3])
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // every thread of every CTA of the cluster: stores before it are visible to loads after it
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -724,20 +745,18 @@ __global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a, int tp
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_barrier_init();
-    if (r1 > r0) {
-      const uint32_t bytes = static_cast<uint32_t>((r1 - r0) * D * 2);
-      mbar_arrive_expect_tx(bar, bytes);
-      bulk_g2s(cs + P.w, static_cast<const __nv_bfloat16 *>(a.L.router_w) + static_cast<int64_t>(r0) * D, bytes, bar);
-    } else {
+    if (r1 > r0)
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>((r1 - r0) * D * 2));
+    else
       mbar_arrive(bar);
-    }
   }
-  float bias_r[kClRowsPerWarp];
-#pragma unroll
-  for (int i = 0; i < kClRowsPerWarp; ++i) {
-    const int row = r0 + warp + kClWarps * i;
-    bias_r[i] = row < r1 && row < E ? __ldg(a.L.bias + row) : 0.f;
-  }
+  __syncthreads();  // the barrier is armed before any copy completes on it
+  if (warp == 0)    // one bulk copy per row (lane l: rows l, l + 32), into rows of P.rs bytes
+    for (int rl = lane; rl < r1 - r0; rl += 32)
+      bulk_g2s(cs + P.w + rl * P.rs, static_cast<const __nv_bfloat16 *>(a.L.router_w) + static_cast<int64_t>(r0 + rl) * D,
+               static_cast<uint32_t>(D * 2), bar);
+  float *bias_s = reinterpret_cast<float *>(cs + P.bias);
+  for (int rl = tid; rl < r1 - r0; rl += kClThreads) bias_s[rl] = r0 + rl < E ? __ldg(a.L.bias + r0 + rl) : 0.f;
   griddep_wait();
   griddep_launch();
   if (blockIdx.x == 0 && tid < 2) a.ws.counters[tid] = 0u;  // the GEMV kernel's work queue starts empty
@@ -783,53 +802,83 @@ __global__ void __launch_bounds__(kClThreads, 1) k_route_cl(DecodeArgs a, int tp
       rec->pad = 0u;
     }
   }
-  // logits of this CTA's rows for token slot sl: warp = rows warp, warp + 16, warp + 32; lane =
-  // 8-column groups lane, lane + 32, ... (fp32 sums over the whole d_model), stored into CTA sl
-  if (!mbar_wait_bounded(bar, 0u, a.spin_limit) && lane == 0) flag_error(a.err, kErrTimeout);
-  const int G8 = D / 256;
-  const __nv_bfloat16 *wsm = reinterpret_cast<const __nv_bfloat16 *>(cs + P.w);
-#pragma unroll 1
-  for (int sl = 0; sl < nt; ++sl) {
-  float xv[kClMaxD / 256][8];
-#pragma unroll
-  for (int j = 0; j < kClMaxD / 256; ++j)
-    if (j < G8) {
-      const float4 *p = reinterpret_cast<const float4 *>(xs + sl * D + 8 * lane + 256 * j);
-      const float4 u = p[0], w = p[1];
-      xv[j][0] = u.x; xv[j][1] = u.y; xv[j][2] = u.z; xv[j][3] = u.w;
-      xv[j][4] = w.x; xv[j][5] = w.y; xv[j][6] = w.z; xv[j][7] = w.w;
+  // logits of this CTA's rows on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 sums): the
+  // rows are A (three 16-row tiles), the token slots' x parts the columns of B (x = hi + lo, both
+  // bf16, so x keeps 16 bits of mantissa; columns past the cluster's tokens repeat its last one
+  // and are not used); warp w sums the d_model columns [D w / 16, D (w + 1) / 16), then the 16
+  // partial sums of each (row, slot) are added in warp order and stored into CTA slot's logits.
+  {
+    unsigned char *xb = cs + P.xb;
+    for (int i = tid; i < nt * D; i += kClThreads) {
+      const int sl = i / D, k = i - sl * D;
+      const float v = xs[sl * D + k];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+      *reinterpret_cast<__nv_bfloat16 *>(xb + sl * P.rs + 2 * k) = hi;
+      *reinterpret_cast<__nv_bfloat16 *>(xb + (tpc + sl) * P.rs + 2 * k) = lo;
     }
-  const uint32_t lg0 = mapa_shared(smem_u32(cs + P.lg), static_cast<uint32_t>(sl)),
-                 raw0 = mapa_shared(smem_u32(cs + P.raw), static_cast<uint32_t>(sl));
+  }
+  __syncthreads();
+  if (!mbar_wait_bounded(bar, 0u, a.spin_limit) && lane == 0) flag_error(a.err, kErrTimeout);
+  float *red = reinterpret_cast<float *>(cs + P.red);
+  {
+    const int g = lane >> 2, cq = lane & 3, R = P.R;
+    const int xr = min(g, nt - 1);
+    const uint32_t wb = smem_u32(cs + P.w), xh = smem_u32(cs + P.xb) + xr * P.rs,
+                   xl = smem_u32(cs + P.xb) + (tpc + xr) * P.rs;
+    // fragment rows of the three tiles (rows past this CTA's R repeat its last one)
+    uint32_t ra[3], rb[3];
 #pragma unroll
-  for (int i = 0; i < kClRowsPerWarp; ++i) {
-    const int rl = warp + kClWarps * i, row = r0 + rl;
-    if (row < r1) {
-      float s = 0.f;
+    for (int mt = 0; mt < 3; ++mt) {
+      ra[mt] = wb + min(16 * mt + g, R - 1) * P.rs;
+      rb[mt] = wb + min(16 * mt + g + 8, R - 1) * P.rs;
+    }
+    float acc[3][4];
 #pragma unroll
-      for (int j = 0; j < kClMaxD / 256; ++j)
-        if (j < G8) {
-          const uint4 q = *reinterpret_cast<const uint4 *>(wsm + static_cast<int64_t>(rl) * D + 8 * lane + 256 * j);
-          const uint32_t pw[4] = {q.x, q.y, q.z, q.w};
+    for (int mt = 0; mt < 3; ++mt)
 #pragma unroll
-          for (int k2 = 0; k2 < 4; ++k2) {
-            s = fmaf(__uint_as_float(pw[k2] << 16), xv[j][2 * k2], s);
-            s = fmaf(__uint_as_float(pw[k2] & 0xFFFF0000u), xv[j][2 * k2 + 1], s);
-          }
-        }
+      for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
+    const int kw = D / kClWarps;  // a multiple of 16: d_model is a multiple of 256
+#pragma unroll 2
+    for (int ks = 0; ks < kw; ks += 16) {
+      const uint32_t kb = static_cast<uint32_t>(2 * (warp * kw + ks + 2 * cq));  // byte offset of column k0 + 2 cq
+      const uint32_t bh0 = lds_u32(xh + kb), bh1 = lds_u32(xh + kb + 16);
+      const uint32_t bl0 = lds_u32(xl + kb), bl1 = lds_u32(xl + kb + 16);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) {
-        if (row < E) {
-          st_cluster_f32(lg0 + 4u * row, s + bias_r[i]);
-          st_cluster_f32(raw0 + 4u * row, s);
-        } else {
-          a.ws.gate_logit[t0 + sl] = s;  // the shared expert's gate row
+      for (int mt = 0; mt < 3; ++mt) {
+        if (16 * mt < R) {
+          const uint32_t a0 = lds_u32(ra[mt] + kb), a1 = lds_u32(rb[mt] + kb), a2 = lds_u32(ra[mt] + kb + 16),
+                         a3 = lds_u32(rb[mt] + kb + 16);
+          mma_bf16_16816(acc[mt], a0, a1, a2, a3, bh0, bh1);
+          mma_bf16_16816(acc[mt], a0, a1, a2, a3, bl0, bl1);
         }
       }
     }
+    // columns 0 and 1 (token slots 0, 1) sit in the lanes with cq = 0
+    if (cq == 0) {
+#pragma unroll
+      for (int mt = 0; mt < 3; ++mt) {
+        float *r0p = red + (warp * kClRedRows + 16 * mt + g) * kClMaxTpc;
+        r0p[0] = acc[mt][0];
+        r0p[1] = acc[mt][1];
+        r0p[8 * kClMaxTpc] = acc[mt][2];
+        r0p[8 * kClMaxTpc + 1] = acc[mt][3];
+      }
+    }
   }
-  }  // token slots
+  __syncthreads();
+  for (int i = tid; i < (r1 - r0) * nt; i += kClThreads) {
+    const int rl = i / nt, sl = i - rl * nt, row = r0 + rl;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kClWarps; ++w) sum += red[(w * kClRedRows + rl) * kClMaxTpc + sl];
+    if (row < E) {
+      st_cluster_f32(mapa_shared(smem_u32(cs + P.lg) + 4u * row, static_cast<uint32_t>(sl)), sum + bias_s[rl]);
+      st_cluster_f32(mapa_shared(smem_u32(cs + P.raw) + 4u * row, static_cast<uint32_t>(sl)), sum);
+    } else {
+      a.ws.gate_logit[t0 + sl] = sum;  // the shared expert's gate row
+    }
+  }
   cluster_sync_all();
   if (c >= nt) return;
   // top-k + softmax of token t = t0 + c by warp 0 of CTA c
@@ -881,7 +930,7 @@ static int g_cl_resident = 1;
 static bool route_cluster_fits(const Shape &sh) {
   const int ER = sh.e + sh.shared_gate;
   return g_route_cluster && sh.router_bf16 && sh.d <= kClMaxD && sh.d % 256 == 0 && sh.e <= kClMaxExperts &&
-         (ER + kClCtas - 1) / kClCtas <= kClWarps * kClRowsPerWarp && cl_plan(ER, sh.d, kClMaxTpc).total <= 200 * 1024;
+         (ER + kClCtas - 1) / kClCtas <= kClRedRows && cl_plan(ER, sh.d, kClMaxTpc).total <= 200 * 1024;
 }
 
 // ------------------------------------------------------------------------------------------
