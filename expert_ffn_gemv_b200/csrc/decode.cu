@@ -1752,13 +1752,15 @@ __global__ void __launch_bounds__(kGemvThreads, MOE_GEMV_MIN_BLOCKS) k_gemv(Deco
 // 3,540 -> 3,714 tok/s at 8 tokens), 64 below (one token ran 2.6 % slower at 32)
 constexpr int kCombineCols = 64;       // at most; d_model is a multiple of 128
 __host__ __device__ inline int combine_cols(int n) { return n >= 4 ? 32 : 64; }
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 384;  // at most: 384 below four tokens (two rounds of dependent
+                                       // loads per thread instead of three), 256 from four on
+__host__ __device__ inline int combine_threads(int n) { return n >= 4 ? 256 : kCombineThreads; }
 constexpr int kMaxSlices = 8;          // K-slices of a slot loaded together (more: one at a time)
 __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
   __shared__ float s_w[kMaxTopK];
   __shared__ int s_sel[kDecodeMaxTokens * kMaxTopK];
   __shared__ float s_o[(kMaxTopK + 1) * kCombineCols];  // [slot (K: the shared expert)][column]
-  const int D = a.sh.d, K = a.sh.k, tid = threadIdx.x;
+  const int D = a.sh.d, K = a.sh.k, tid = threadIdx.x, nthr = blockDim.x;
   const int cols = combine_cols(a.n), cpt = D / cols;  // CTAs per token
   const int t = blockIdx.x / cpt, d0 = (blockIdx.x - t * cpt) * cols;
   griddep_wait();
@@ -1766,9 +1768,9 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
   if (tid < K) s_w[tid] = __ldcg(a.ws.route_w + t * K + tid);
   if (blockIdx.x == 0 && a.out_counts) {  // tokens per expert, from the router's selections
     const int nk = a.n * K;
-    for (int p = tid; p < nk; p += kCombineThreads) s_sel[p] = __ldcg(a.ws.sel + p);
+    for (int p = tid; p < nk; p += nthr) s_sel[p] = __ldcg(a.ws.sel + p);
     __syncthreads();
-    for (int e = tid; e < a.sh.e; e += kCombineThreads) {
+    for (int e = tid; e < a.sh.e; e += nthr) {
       int c = 0;
       for (int p = 0; p < nk; ++p) c += s_sel[p] == e ? 1 : 0;
       a.out_counts[e] = c;
@@ -1777,7 +1779,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(DecodeArgs a) {
   __syncthreads();
   const int TM = a.ws.tmax, ns = a.sh.n_shared ? 1 : 0;
   const int js = ns ? a.L.shared.f / kTileRows : 0, jr = a.L.routed.f / kTileRows;
-  for (int it = tid; it < (K + ns) * cols; it += kCombineThreads) {
+  for (int it = tid; it < (K + ns) * cols; it += nthr) {
     const int j = it / cols, c = it - j * cols;
     const bool sh = j == K;
     const float *src = a.ws.o + static_cast<int64_t>(sh ? t : ns * a.n + t * K + j) * TM * D + d0 + c;
@@ -1987,7 +1989,7 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, cudaStream_t st) {
   // 3. weighted combine
   {
     rec(a, kProfDown, 0, st);
-    err = launch_pdl(k_combine, a.n * (a.sh.d / combine_cols(a.n)), kCombineThreads, 0, st, a);
+    err = launch_pdl(k_combine, a.n * (a.sh.d / combine_cols(a.n)), combine_threads(a.n), 0, st, a);
     if (err != cudaSuccess) return err;
     rec(a, kProfDown, 1, st);
   }
