@@ -1,31 +1,32 @@
 // decode.cu -- the dequant-fused GEMV path for 1..8 tokens (decode steps and 1 + 7 token
 // verify batches of the routed-MoE pages: strata-mlx README, "Draft and verify").
 //
-// Three kernels per layer, all on CUDA cores, chained by programmatic dependent launches:
-//   k_route    router GEMV: CTA = 4 experts, warp = (expert, half of d_model), fp32 sums over
-//              the whole d_model (no cross-CTA reduction), logits + bias to global memory.  The
-//              CTAs also quantise the layer input into activation records (int16 + block sums +
-//              a power-of-two factor per 128 columns); the last CTAs to finish take the top-k
-//              of each token (warp per token over order-preserving keys) and the fp32 softmax
-//              over the selected logits.
-//   k_gemv     persistent, one CTA per resident slot.  Every CTA first builds the active-expert
-//              task table in its own shared memory from the selections (all CTAs build the same
-//              table; CTA 0 also writes the routing outputs).  Then a producer warp takes pieces
-//              from one work queue -- a piece is (active expert, 128-row gate/up tile j, token
-//              group, run of K segments) -- and bulk-copies (cp.async.bulk) the rows of the
-//              piece straight from their low-bit planes, with the activation records of the
-//              unit's tokens, into a ring of shared-memory stages, followed by the rows of the
-//              down matrix over K-slice j (the 128 values of h that tile j makes) for the
-//              piece's share of the output tiles.  Four consumer warps (thread = row) unpack the
-//              codes with one ALU op per four weights and multiply them with the int16
-//              activations by dp2a (int16 x int8 -> int32); the exact integer block sums are
-//              scaled by the block scale into fp32 sums, one per K segment, added in segment
-//              order.  At the end of the gate/up tile the consumers apply SwiGLU and quantise h
-//              into records in shared memory (the pieces of a split unit first meet, and each
-//              sums all of their segment partials), then run the down stages against them: no h
-//              leaves the CTA and no down stage waits for another CTA's gate/up work.
-//   k_combine  y = sum_j w_j o_j + o_shared (+ x), slots in descending-logit order; o_j is the
-//              sum of expert j's K-slice outputs in slice order.
+// Three kernels per layer, chained by programmatic dependent launches:
+//   k_route_cl router as clusters of 16 CTAs (one token per cluster, two when the tokens
+//              outnumber the clusters the device holds at once): each CTA copies its router rows
+//              into shared memory before the previous kernel ends, quantises the inputs into
+//              activation records (int16 + block sums + a power-of-two factor per 128 columns),
+//              computes its rows' logits on the tensor cores (mma.sync, bf16 rows x the bf16 hi
+//              and lo parts of x, fp32 sums) and stores each token's logits into one CTA of the
+//              cluster, which takes the top-k and the fp32 softmax.  k_route does the same work
+//              without clusters for the router shapes the cluster kernel does not take.
+//   k_gemv     persistent, one CTA per resident slot.  A unit is one (token, expert) pair of the
+//              routing over one 128-row gate/up tile j; tasks (pieces of units) are numbered
+//              from the selections alone, CTA i starts on task i and later tasks come from a
+//              work-queue counter.  A producer warp bulk-copies (cp.async.bulk) the piece's rows
+//              straight from their low-bit planes, with the token's activation records, into a
+//              ring of shared-memory stages, followed by the rows of the down matrix over
+//              K-slice j (the 128 values of h that tile j makes) for the piece's share of the
+//              output tiles.  Four consumer warps (thread = row) unpack the codes with one ALU
+//              op per four weights and multiply them with the int16 activations by dp2a (int16 x
+//              int8 -> int32); the exact integer block sums are scaled by the block scale into
+//              fp32 sums, one per K segment, added in segment order.  At the end of the gate/up
+//              tile the consumers apply SwiGLU and quantise h into records in shared memory (the
+//              pieces of a split unit first meet, and each sums all of their segment partials),
+//              then run the down stages against them: no h leaves the CTA and no down stage
+//              waits for another CTA's gate/up work.
+//   k_combine  y = sum_j w_j o_j + o_shared (+ x), the choices j in descending-logit order; o_j
+//              is the sum of the pair's K-slice outputs in slice order.
 // No fp32 atomics, and the K segments and slices are fixed by the matrix shapes: results are
 // bit-reproducible and independent of which tokens share a call and of how the work queue
 // split the units among CTAs.
@@ -108,7 +109,7 @@ __device__ __forceinline__ int fix16(float v, float sc) {
 }
 
 // ------------------------------------------------------------------------------------------
-// router + input quantisation + top-k + routing tables
+// router + input quantisation + top-k
 // ------------------------------------------------------------------------------------------
 template <bool RBF16>
 __device__ __forceinline__ void load_row8(const void *w, int64_t off, float (&v)[8]) {
@@ -1020,7 +1021,7 @@ __device__ __forceinline__ int q2_block_dot64(uint32_t w0, uint32_t w1, const in
 __host__ __device__ inline int align128(int v) { return (v + 127) & ~127; }
 
 // Shared memory of the GEMV kernels:
-//   [RingHdr][task table][h records][stage 0] .. [stage kRing-1][grid table (CB35)]
+//   [RingHdr][h records][stage 0] .. [stage kRing-1][grid table (CB35)]
 // A stage holds, for up to CMAX chunks: plane A [NR][CMAX][128][16 B], plane S [NR][CMAX][128]
 // [4 B], plane G [NR][CMAX][128][8 B] (CB35), then the records [8 tokens][CMAX][144 B].
 struct RingPlan {

@@ -91,10 +91,9 @@ struct ActRec {
 };
 static_assert(sizeof(ActRec) == 144, "ActRec is 9 x 16 bytes");
 
-// Decode workspace (n <= 8 tokens).  u indexes active experts: u = 0 is the shared expert
-// when there is one, routed active experts follow in ascending expert id.  A GEMV "unit" is one
-// 128-row tile j of one active expert's gate/up pair for one token group, followed by the down
-// matrix over K-slice j (the 128 values of h the tile makes).  The gate/up K range is cut into
+// Decode workspace (n <= 8 tokens).  A GEMV "unit" is one 128-row tile j of the gate/up pair
+// of one (token, expert) pair of the routing, followed by the down matrix over K-slice j (the
+// 128 values of h the tile makes).  The gate/up K range is cut into
 // fixed segments of 2 or 4 chunks whose fp32 sums are added in segment order, whether one CTA
 // runs the whole unit or several CTAs each take a run of segments (then the segment sums pass
 // through the partial buffers); the down outputs of each K-slice are kept apart and added in
@@ -204,7 +203,7 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes
 }
 
 // L2 policy for data read once (the weight blocks): evict first, so that a pass over the
-// expert blocks does not push the small, reused tensors (activations, routing tables, partial
+// expert blocks does not push the small, reused tensors (activations, selections, partial
 // sums) and the kernels' code out of L2.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
@@ -304,7 +303,7 @@ struct DecodeArgs {
 };
 
 // kernel classes of the per-kernel event timing
-constexpr int kProfRoute = 0;     // router + top-k (+ routing tables / grouping)
+constexpr int kProfRoute = 0;     // router + top-k (+ the prefill's grouping)
 constexpr int kProfGateUp = 1;    // the GEMV kernel (gate/up + SwiGLU + down) or the gate/up GEMM + SwiGLU
 constexpr int kProfDown = 2;      // the combine kernel or the down GEMM + combine
 constexpr int kProfKinds = 3;
