@@ -111,8 +111,7 @@ struct Carve {
 void plan_workspace(moe_handle *h, Carve &c) {
   const moe_config &g = h->cfg;
   const int D = g.d_model, E = g.n_experts, K = g.top_k;
-  const int nd = g.max_tokens < kDecodeMaxTokens ? g.max_tokens : kDecodeMaxTokens;
-  const int pmax = kDecodeMaxTokens * (K + (g.n_shared ? 1 : 0));
+  const int pmax = kDecodeMaxTokens * (K + (g.n_shared ? 1 : 0));  // (token, expert) pairs of a call
   const int fmax = g.n_shared && g.shared_d_ff > g.d_ff ? g.shared_d_ff : g.d_ff;
   const int tmax = fmax / kTileRows;
   DecodeWs &w = h->dws;
